@@ -392,6 +392,7 @@ void orc_block_scores_f64(const uint16_t* q, const uint16_t* k, int BH, int N, i
 /* Steps 6-8: the sparse softmax branch, the linear branch, the projection. */
 /* ------------------------------------------------------------------------ */
 #define ORC_NOQUANT 1 /* test switch: no quantisation anywhere (T3)       */
+#define ORC_WALK 128  /* keys per online-softmax tile of the walk          */
 
 typedef struct {
   int N, d, block, nb, kc;
@@ -409,7 +410,7 @@ static void emul_qblock(const orc_head* H, int i, const int32_t* sel, double* ou
   const double rsd = 1.0 / sqrt((double)d);
   int n0 = i * block, n1 = n0 + block < N ? n0 + block : N;
   double* o = (double*)malloc(sizeof(double) * d);
-  double* sc = (double*)malloc(sizeof(double) * block);
+  double* sc = (double*)malloc(sizeof(double) * (ORC_WALK > block ? ORC_WALK : block));
   double* Hc = NULL;
   double* Zc = NULL;
   uint8_t* in_s = (uint8_t*)calloc(H->nb, 1);
@@ -430,10 +431,16 @@ static void emul_qblock(const orc_head* H, int i, const int32_t* sel, double* ou
     /* --- sparse softmax branch: online over the selected blocks, ascending --- */
     double m = -INFINITY, l = 0.0;
     for (int c = 0; c < d; ++c) o[c] = 0.0;
-    for (int t = 0; t < kc; ++t) {
+    /* The walk takes the selected keys 128 at a time (ORC_WALK / block
+     * consecutive entries of the list): the running max is updated once per
+     * such tile and the tile's P is quantised against it. */
+    const int per_tile = ORC_WALK / block > 0 ? ORC_WALK / block : 1;
+    for (int t0 = 0; t0 < kc; t0 += per_tile) {
+      const int t1 = t0 + per_tile < kc ? t0 + per_tile : kc;
+      double mj = -INFINITY;
+      for (int t = t0; t < t1; ++t) {
       int j = sel[t];
       int k0 = j * block, k1 = k0 + block < N ? k0 + block : N;
-      double mj = -INFINITY;
       for (int kk = k0; kk < k1; ++kk) {
         double s;
         if (H->flags & ORC_NOQUANT) {
@@ -448,15 +455,19 @@ static void emul_qblock(const orc_head* H, int i, const int32_t* sel, double* ou
             acc += (int64_t)H->q8[(int64_t)n * d + c] * (int64_t)H->k8[(int64_t)kk * d + c];
           s = (double)acc * (double)H->sq[n / ORC_QBLK] * (double)H->sk[kk / ORC_QBLK] * rsd;
         }
-        sc[kk - k0] = s;
+        sc[(t - t0) * block + (kk - k0)] = s;
         if (s > mj) mj = s;
       }
+      }
       double mnew = mj > m ? mj : m;
-      double alpha = exp(m - mnew); /* m = -inf on the first block -> 0 */
+      double alpha = exp(m - mnew); /* m = -inf on the first tile -> 0 */
       l *= alpha;
       for (int c = 0; c < d; ++c) o[c] *= alpha;
+      for (int t = t0; t < t1; ++t) {
+      int j = sel[t];
+      int k0 = j * block, k1 = k0 + block < N ? k0 + block : N;
       for (int kk = k0; kk < k1; ++kk) {
-        double p = exp(sc[kk - k0] - mnew);
+        double p = exp(sc[(t - t0) * block + (kk - k0)] - mnew);
         if (H->flags & ORC_NOQUANT) {
           l += p;
           for (int c = 0; c < d; ++c) o[c] += p * (double)bf16_f32(H->v[(int64_t)kk * d + c]);
@@ -468,6 +479,7 @@ static void emul_qblock(const orc_head* H, int i, const int32_t* sel, double* ou
           for (int c = 0; c < d; ++c)
             o[c] += pq * orc_e4m3_decode(H->v8[(int64_t)kk * d + c]);
         }
+      }
       }
       m = mnew;
     }

@@ -174,3 +174,20 @@ def test_external_mask_and_query_selection(orc):
     if not np.array_equal(idx_alt, idx):
         out4, _ = orc.sagesla(q, k, v, w, 64, 0.4, idx=idx_alt)
         assert np.abs(out4[0, :64] - out[0, :64]).max() > 1e-4
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_worked_walk_tile(orc, block):
+    with open(os.path.join(GOLDEN, "worked_walk_tiles.json")) as f:
+        g = json.load(f)
+    N, d = g["N"], g["d"]
+    q = torch.zeros(1, N, d)
+    q[0, :, 0] = g["a"]
+    k = torch.zeros(1, N, d)
+    k[0, 64:, 0] = 2 * g["delta"]
+    v = torch.zeros(1, N, d)
+    v[0, :64, :2] = torch.tensor(g["v_block0"])
+    v[0, 64:, :2] = torch.tensor(g["v_block1"])
+    out, _ = orc.sagesla(q.bfloat16(), k.bfloat16(), v.bfloat16(), None, block, 1.0)
+    for (c, num, den) in g["expect"]:
+        np.testing.assert_allclose(out[0, :, c], num / den, rtol=0, atol=1e-12)
