@@ -1,0 +1,156 @@
+/*
+ * sagesla.h -- C ABI of the SageSLA attention library for NVIDIA B200 (sm_100a).
+ *
+ * SageSLA attention, as the TurboDiffusion pages describe it
+ *   ("揭秘TurboDiffusion：如何让视频生成实现百倍加速？", 支柱一 SageAttention and
+ *    支柱二 SLA; "TurboDiffusion跨模态：图文音视频多模态融合探索", 2.1-2.2;
+ *    量子位 news, 技术解密 1-2):
+ *   - SageAttention: QK^T in INT8 after a smoothing step that removes channel
+ *     outliers (here: the per-head mean of K is subtracted), P.V in FP8;
+ *   - SLA: per query block, only the top-k fraction of key blocks (sla_topk,
+ *     default 0.1) is computed exactly; every other key block contributes
+ *     through a linear-attention branch phi(Q)(phi(K)^T V), phi = elu + 1,
+ *     followed by a d x d projection, added to the sparse output.
+ *
+ * Readings taken where the pages are silent (all stated here once):
+ *   - INT8 Q and K codes per 64-token block with one fp32 scale each
+ *     (amax/127, symmetric, round half to even); FP8 E4M3 V codes with one
+ *     fp32 scale per channel (amax/448); K is smoothed by its per-channel mean
+ *     over the N tokens before quantisation.
+ *   - Block scores: mean-pooled Q_i . mean-pooled (K-mu)_j / sqrt(d) in fp32;
+ *     k = clamp(ceil(topk * Nb), 1, Nb) blocks per query block, ties to the
+ *     lower block index, walked in ascending order.
+ *   - Online softmax: P = exp(S - running max); P~ = e4m3(448 P); the row sum
+ *     is taken over the same P~ that weight V.
+ *   - Linear branch from the raw bf16 Q, K, V: for row r of query block i,
+ *     O_l = phi(q_r) H_i / phi(q_r) Z_i with H_i = sum over unselected key
+ *     blocks j of phi(K_j)^T V_j and Z_i = sum of phi(K_j) rows; y = O_l W^T
+ *     (W = proj_w, [d_out][d_in] row-major, shared by all heads, no bias).
+ *     Empty complement (topk = 1) -> the branch contributes 0.
+ *   - out = bf16(O_s + y), rounded once.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are DEVICE pointers owned by the caller, bf16, contiguous
+ *     [B][H][N][d], 16-byte aligned.  Inputs are never written; rows n >= N
+ *     are never read or written.
+ *   - The call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  It performs no host synchronisation, except that the
+ *     first call needing a larger workspace on a (device, stream) allocates it
+ *     stream-ordered.
+ *   - Supported: d == 128, block in {64, 128}, 0 < topk <= 1, B, H, N >= 1,
+ *     B*H*N*d < 2^40.  Anything else returns SAGESLA_ERR_INVALID without
+ *     launching.  There is no CPU fallback and no alternative backend.
+ *   - The library owns a workspace cache keyed by (device, stream);
+ *     sagesla_release() frees it.
+ */
+#ifndef SAGESLA_H_
+#define SAGESLA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sagesla_stream_t; /* same type as cudaStream_t */
+
+enum {
+  SAGESLA_OK = 0,
+  SAGESLA_ERR_INVALID = -1,        /* bad argument (null, size, d, block, topk, NaN) */
+  SAGESLA_ERR_MISALIGNED = -2,     /* a pointer is not 16-byte aligned */
+  SAGESLA_ERR_OOM = -3,            /* workspace allocation failed */
+  SAGESLA_ERR_LAUNCH = -4,         /* a CUDA launch or runtime call failed */
+  SAGESLA_ERR_DEVICE_TIMEOUT = -5, /* a bounded device-side wait gave up */
+  SAGESLA_ERR_NO_DEVICE = -6       /* current device is not sm_100 */
+};
+
+/*
+ * sagesla_attn: the whole SageSLA path (smoothing + quantisation, pooled
+ * top-k block mask, linear branch, block-sparse INT8/FP8 flash attention with
+ * the linear output and projection added in its epilogue).
+ *   q, k, v  bf16 [B][H][N][d] device.
+ *   proj_w   bf16 [d][d] device, row-major, y = x W^T; NULL turns the linear
+ *            branch off (out = O_s).
+ *   out      bf16 [B][H][N][d] device (written).
+ *   block    64 or 128 (query and key block size of the mask).
+ *   topk     fraction of key blocks computed exactly per query block.
+ * Returns SAGESLA_OK or a negative SAGESLA_ERR_* code (nothing written on an
+ * argument error).
+ */
+int sagesla_attn(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B,
+                 int H, int N, int d, int block, float topk, sagesla_stream_t stream);
+
+/*
+ * dense_int8_attn: the dense reference point of the same kernels, identical
+ * to sagesla_attn(q, k, v, NULL, out, B, H, N, d, 64, 1.0f, stream): every
+ * key block selected, linear branch off.
+ */
+int dense_int8_attn(const void* q, const void* k, const void* v, void* out, int B, int H, int N,
+                    int d, sagesla_stream_t stream);
+
+/*
+ * sagesla_attn_host: sagesla_attn on HOST buffers (pinned memory gives
+ * asynchronous copies).  Copies q, k, v (and proj_w) to the device, runs the
+ * path, copies out back and synchronises `stream` before returning.  Same
+ * shapes and codes as sagesla_attn; proj_w may be NULL.
+ */
+int sagesla_attn_host(const void* q, const void* k, const void* v, const void* proj_w, void* out,
+                      int B, int H, int N, int d, int block, float topk, sagesla_stream_t stream);
+
+/*
+ * sagesla_get_quant: the smoothing + quantisation step alone (for parity).
+ *   q8, k8   int8 [B][H][N][d] device: INT8 codes, row-major.
+ *   v8       uint8 [B][H][N][d] device: FP8 E4M3 codes, row-major.
+ *   sq, sk   float [B][H][ceil(N/64)] device: per-64-token-block scales.
+ *   sv, mu   float [B][H][d] device: per-channel V scale, K mean.
+ */
+int sagesla_get_quant(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                      int8_t* q8, int8_t* k8, uint8_t* v8, float* sq, float* sk, float* sv, float* mu,
+                      sagesla_stream_t stream);
+
+/*
+ * sagesla_get_mask: the block mask alone (for parity).
+ *   idx_out  int32 [B][H][Nb][k] device, Nb = ceil(N/block), k as above;
+ *            each row sorted ascending.
+ *   qbar, kbar  float [B][H][Nb][d] device, or NULL: the pooled means.
+ *   k_out    host int*: receives k (may be NULL).
+ */
+int sagesla_get_mask(const void* q, const void* k, int B, int H, int N, int d, int block,
+                     float topk, int32_t* idx_out, float* qbar, float* kbar, int* k_out,
+                     sagesla_stream_t stream);
+
+/* Number of key blocks kept per query block: clamp(ceil(topk*nb*(1-1e-6)), 1, nb). */
+int sagesla_topk_count(int nb, float topk);
+
+/*
+ * sagesla_sync_status: synchronises `stream` and returns SAGESLA_OK, or
+ * SAGESLA_ERR_DEVICE_TIMEOUT if any bounded device-side wait of an earlier
+ * call on it gave up (the flag is then cleared), or SAGESLA_ERR_LAUNCH.
+ */
+int sagesla_sync_status(sagesla_stream_t stream);
+
+/* Human-readable text for a return code (static storage). */
+const char* sagesla_strerror(int code);
+
+/*
+ * Measurement hooks.  sagesla_profile(1) brackets every kernel the library
+ * launches with CUDA events recorded on the launching stream;
+ * sagesla_profile_read() waits for them and returns, per kernel id, the
+ * summed milliseconds and the number of launches since the last read, then
+ * forgets them.  Kernel ids: 0 stats, 1 stats finalise, 2 quantise,
+ * 3 pooled top-k, 4 linear per-block phi(K)^T V, 5 linear complement sum,
+ * 6 sparse flash, 7 projection-weight tiling.  ms / launches are arrays of
+ * nkernels entries (either may be NULL).  Profiling is off by default.
+ */
+#define SAGESLA_NUM_KERNELS 8
+void sagesla_profile(int enable);
+int sagesla_profile_read(double* ms, int* launches, int nkernels);
+
+/* Frees every cached workspace (synchronises the device first). */
+void sagesla_release(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGESLA_H_ */

@@ -1,0 +1,173 @@
+"""SageSLA attention for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over the C ABI of include/sagesla.h (libsagesla.so,
+built in-tree by `build.py`).  It only marshals arguments: every step of the
+path runs in the library's CUDA kernels.  Tensors are torch CUDA tensors
+(device memory and streams come from PyTorch); there is no CPU fallback --
+a missing library or a non-sm_100 device raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from . import inputs  # noqa: F401  (seeded synthetic inputs, no method arithmetic)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsagesla.so")
+_lib = None
+
+ERRORS = {0: "ok", -1: "invalid argument", -2: "misaligned pointer", -3: "out of memory",
+          -4: "CUDA launch error", -5: "device watchdog timeout", -6: "not an sm_100 device"}
+
+
+class SageSLAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {ERRORS.get(code, 'error')} ({code})")
+
+
+EXPORTS = ["sagesla_attn", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
+           "sagesla_topk_count", "sagesla_sync_status", "sagesla_strerror", "sagesla_release", "sagesla_profile",
+           "sagesla_profile_read"]
+KERNELS = ["stats", "stats_final", "quant", "pool_topk", "linear_kv", "linear_sum", "flash", "w_tile"]
+
+
+def lib():
+    """Load libsagesla.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m sparse_bit_attention_smoothing_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.sagesla_attn.argtypes = [P, P, P, P, P, i, i, i, i, i, f, P]
+        L.dense_int8_attn.argtypes = [P, P, P, P, i, i, i, i, P]
+        L.sagesla_attn_host.argtypes = [P, P, P, P, P, i, i, i, i, i, f, P]
+        L.sagesla_get_quant.argtypes = [P, P, P, i, i, i, i, P, P, P, P, P, P, P, P]
+        L.sagesla_get_mask.argtypes = [P, P, i, i, i, i, i, f, P, P, P, P, P]
+        L.sagesla_topk_count.argtypes = [i, f]
+        L.sagesla_sync_status.argtypes = [P]
+        L.sagesla_strerror.restype = ctypes.c_char_p
+        L.sagesla_strerror.argtypes = [i]
+        L.sagesla_release.restype = None
+        L.sagesla_profile.restype = None
+        L.sagesla_profile.argtypes = [i]
+        L.sagesla_profile_read.argtypes = [P, P, i]
+        for name in EXPORTS:
+            getattr(L, name)
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise SageSLAError(rc, where)
+
+
+def _shape(q):
+    assert q.dim() == 4, "q, k, v must be [B, H, N, d]"
+    return q.shape
+
+
+def topk_count(nb: int, topk: float) -> int:
+    return lib().sagesla_topk_count(nb, ctypes.c_float(topk))
+
+
+def sagesla_attn(q, k, v, proj_w=None, out=None, block: int = 64, topk: float = 0.1, stream=None):
+    """SageSLA attention.  q, k, v: bf16 CUDA [B, H, N, d]; proj_w: bf16 [d, d] or None."""
+    import torch
+    B, H, N, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().sagesla_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(proj_w), _ptr(out), B, H, N, d, block,
+                              ctypes.c_float(topk), _stream(stream)), "sagesla_attn")
+    return out
+
+
+def dense_int8_attn(q, k, v, out=None, stream=None):
+    import torch
+    B, H, N, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().dense_int8_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, _stream(stream)),
+           "dense_int8_attn")
+    return out
+
+
+def sagesla_attn_host(q, k, v, proj_w=None, out=None, block: int = 64, topk: float = 0.1, stream=None):
+    """Same on HOST tensors (pinned for asynchronous copies); returns after the result is in `out`."""
+    import torch
+    B, H, N, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().sagesla_attn_host(_ptr(q), _ptr(k), _ptr(v), _ptr(proj_w), _ptr(out), B, H, N, d, block,
+                                   ctypes.c_float(topk), _stream(stream)), "sagesla_attn_host")
+    return out
+
+
+def sagesla_get_quant(q, k, v, stream=None) -> dict:
+    import torch
+    B, H, N, d = _shape(q)
+    dev = q.device
+    nq = (N + 63) // 64
+    r = dict(q8=torch.empty(B, H, N, d, dtype=torch.int8, device=dev),
+             k8=torch.empty(B, H, N, d, dtype=torch.int8, device=dev),
+             v8=torch.empty(B, H, N, d, dtype=torch.uint8, device=dev),
+             sq=torch.empty(B, H, nq, dtype=torch.float32, device=dev),
+             sk=torch.empty(B, H, nq, dtype=torch.float32, device=dev),
+             sv=torch.empty(B, H, d, dtype=torch.float32, device=dev),
+             mu=torch.empty(B, H, d, dtype=torch.float32, device=dev))
+    _check(lib().sagesla_get_quant(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(r["q8"]), _ptr(r["k8"]),
+                                   _ptr(r["v8"]), _ptr(r["sq"]), _ptr(r["sk"]), _ptr(r["sv"]), _ptr(r["mu"]),
+                                   _stream(stream)), "sagesla_get_quant")
+    return r
+
+
+def sagesla_get_mask(q, k, block: int = 64, topk: float = 0.1, pooled: bool = False, stream=None) -> dict:
+    import torch
+    B, H, N, d = _shape(q)
+    nb = (N + block - 1) // block
+    kc = topk_count(nb, topk)
+    dev = q.device
+    r = dict(idx=torch.empty(B, H, nb, kc, dtype=torch.int32, device=dev), k=kc,
+             qbar=torch.empty(B, H, nb, d, dtype=torch.float32, device=dev) if pooled else None,
+             kbar=torch.empty(B, H, nb, d, dtype=torch.float32, device=dev) if pooled else None)
+    kout = ctypes.c_int(0)
+    _check(lib().sagesla_get_mask(_ptr(q), _ptr(k), B, H, N, d, block, ctypes.c_float(topk), _ptr(r["idx"]),
+                                  _ptr(r["qbar"]), _ptr(r["kbar"]), ctypes.byref(kout), _stream(stream)),
+           "sagesla_get_mask")
+    assert kout.value == kc
+    return r
+
+
+def sync_status(stream=None) -> int:
+    return lib().sagesla_sync_status(_stream(stream))
+
+
+def profile(enable: bool):
+    """Bracket every library kernel launch with CUDA events on its stream."""
+    lib().sagesla_profile(1 if enable else 0)
+
+
+def profile_read() -> dict:
+    """{kernel name: (total ms, launches)} since the last read."""
+    n = len(KERNELS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int * n)()
+    _check(lib().sagesla_profile_read(ms, cnt, n), "sagesla_profile_read")
+    return {KERNELS[i]: (ms[i], cnt[i]) for i in range(n) if cnt[i]}
+
+
+def release():
+    lib().sagesla_release()

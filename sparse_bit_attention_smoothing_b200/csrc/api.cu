@@ -1,0 +1,430 @@
+// api.cu -- the C ABI of include/sagesla.h: argument checks, the workspace
+// cache and the launch sequence of the SageSLA path.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "../../include/sagesla.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sagesla {
+size_t pool_topk_smem(int nb);
+}
+
+using namespace sagesla;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::mutex g_mu;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+std::map<int, int*> g_wd;        // per-device watchdog word
+std::map<int, int> g_dev_ok;     // per-device: 1 = sm_100, 0 = not
+
+int check_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGESLA_ERR_NO_DEVICE;
+  *dev_out = dev;
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_dev_ok.find(dev);
+  if (it == g_dev_ok.end()) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    g_dev_ok[dev] = (major == 10 && minor == 0) ? 1 : 0;
+    it = g_dev_ok.find(dev);
+  }
+  if (!it->second) return SAGESLA_ERR_NO_DEVICE;
+  if (!g_wd.count(dev)) {
+    int* wd = nullptr;
+    if (cudaMalloc(&wd, sizeof(int)) != cudaSuccess) return SAGESLA_ERR_OOM;
+    if (cudaMemset(wd, 0, sizeof(int)) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
+    g_wd[dev] = wd;
+  }
+  return SAGESLA_OK;
+}
+
+int* watchdog(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return g_wd[dev];
+}
+
+// Stream-ordered workspace of at least `bytes`, cached per (device, stream).
+int get_workspace(int dev, cudaStream_t st, size_t bytes, uint8_t** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[std::make_pair(dev, st)];
+  if (w.bytes < bytes) {
+    if (w.ptr) cudaFreeAsync(w.ptr, st);
+    w.ptr = nullptr;
+    w.bytes = 0;
+    if (cudaMallocAsync(&w.ptr, bytes, st) != cudaSuccess) {
+      cudaGetLastError();
+      return SAGESLA_ERR_OOM;
+    }
+    w.bytes = bytes;
+  }
+  *out = static_cast<uint8_t*>(w.ptr);
+  return SAGESLA_OK;
+}
+
+// ------------------------------------------------------------------ profiler
+// When enabled, every kernel launch is bracketed by two CUDA events recorded
+// on the launching stream; sagesla_profile_read() sums the durations per
+// kernel.  Events come from a pool and are reused.
+struct ProfRec {
+  int kernel;
+  cudaEvent_t a, b;
+};
+std::mutex g_pmu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_evpool;
+
+cudaEvent_t ev_get() {
+  if (!g_evpool.empty()) {
+    cudaEvent_t e = g_evpool.back();
+    g_evpool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct ProfScope {
+  int kernel;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr;
+  ProfScope(int k, cudaStream_t s) : kernel(k), st(s) {
+    std::lock_guard<std::mutex> lk(g_pmu);
+    if (g_prof_on) {
+      a = ev_get();
+      cudaEventRecord(a, st);
+    }
+  }
+  ~ProfScope() {
+    if (!a) return;
+    std::lock_guard<std::mutex> lk(g_pmu);
+    cudaEvent_t b = ev_get();
+    cudaEventRecord(b, st);
+    g_prof.push_back({kernel, a, b});
+  }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate(const void* q, const void* k, const void* v, const void* out, int B, int H, int N, int d, int block,
+             float topk) {
+  if (!q || !k || !v || !out) return SAGESLA_ERR_INVALID;
+  if (B < 1 || H < 1 || N < 1 || d != kD) return SAGESLA_ERR_INVALID;
+  if (block != 64 && block != 128) return SAGESLA_ERR_INVALID;
+  if (!(topk > 0.f) || !(topk <= 1.f)) return SAGESLA_ERR_INVALID;  // rejects NaN
+  const long long BH = (long long)B * H;
+  if (BH > 65535) return SAGESLA_ERR_INVALID;
+  if ((double)BH * N * d >= 1099511627776.0) return SAGESLA_ERR_INVALID;
+  const int nb = (N + block - 1) / block;
+  if (sagesla::pool_topk_smem(nb) > 227 * 1024) return SAGESLA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SAGESLA_ERR_MISALIGNED;
+  return SAGESLA_OK;
+}
+
+Geom make_geom(int B, int H, int N, int block, float topk) {
+  Geom g;
+  g.BH = B * H;
+  g.N = N;
+  g.block = block;
+  g.nb = (N + block - 1) / block;
+  g.nq = 2 * ((N + 127) / 128);
+  g.kc = sagesla_topk_count(g.nb, topk);
+  // Row splits for the statistics pass: about 4 CTAs per SM over the grid.
+  int split = (592 + g.BH - 1) / g.BH;
+  const int max_split = (N + 63) / 64;
+  g.split = split < 1 ? 1 : (split > max_split ? max_split : split);
+  return g;
+}
+
+// Carve the workspace.  Every region 256-byte aligned.
+struct Buffers {
+  double* psum;
+  float *pmax, *mu, *sv, *mv;
+  uint8_t *q8t, *k8t, *v8t;
+  float *sq, *sk, *qsum, *ksum;
+  int32_t* idx;
+  size_t total;
+};
+
+Buffers carve(uint8_t* base, const Geom& g) {
+  Buffers b;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base ? base + o : nullptr;
+    o += up(bytes);
+    return p;
+  };
+  const size_t BH = (size_t)g.BH;
+  b.psum = reinterpret_cast<double*>(take(BH * g.split * kD * sizeof(double)));
+  b.pmax = reinterpret_cast<float*>(take(BH * g.split * kD * sizeof(float)));
+  b.mu = reinterpret_cast<float*>(take(BH * kD * sizeof(float)));
+  b.sv = reinterpret_cast<float*>(take(BH * kD * sizeof(float)));
+  b.mv = reinterpret_cast<float*>(take(BH * kD * sizeof(float)));
+  b.q8t = take(BH * g.nq * kTile);
+  b.k8t = take(BH * g.nq * kTile);
+  b.v8t = take(BH * g.nq * kTile);
+  b.sq = reinterpret_cast<float*>(take(BH * g.nq * sizeof(float)));
+  b.sk = reinterpret_cast<float*>(take(BH * g.nq * sizeof(float)));
+  b.qsum = reinterpret_cast<float*>(take(BH * g.nq * kD * sizeof(float)));
+  b.ksum = reinterpret_cast<float*>(take(BH * g.nq * kD * sizeof(float)));
+  b.idx = reinterpret_cast<int32_t*>(take(BH * g.nb * (size_t)g.kc * sizeof(int32_t)));
+  b.total = o;
+  return b;
+}
+
+inline int launch_rc(cudaError_t e) { return e == cudaSuccess ? SAGESLA_OK : SAGESLA_ERR_LAUNCH; }
+
+#define SAGESLA_TRY(x)          \
+  do {                          \
+    int rc_ = (x);              \
+    if (rc_ != SAGESLA_OK) return rc_; \
+  } while (0)
+
+// Stats + quantisation (the front shared by every entry point).
+int run_front(const void* q, const void* k, const void* v, const Geom& g, const Buffers& b, cudaStream_t st) {
+  {
+    ProfScope ps(0, st);
+    SAGESLA_TRY(launch_rc(launch_stats_partial(k, v, g, b.psum, b.pmax, st)));
+  }
+  {
+    ProfScope ps(1, st);
+    SAGESLA_TRY(launch_rc(launch_stats_final(b.psum, b.pmax, g, b.mu, b.sv, b.mv, st)));
+  }
+  {
+    ProfScope ps(2, st);
+    SAGESLA_TRY(launch_rc(
+        launch_quant(q, k, v, b.mu, b.mv, g, b.q8t, b.k8t, b.v8t, b.sq, b.sk, b.qsum, b.ksum, st)));
+  }
+  return SAGESLA_OK;
+}
+
+int run_attn(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B, int H, int N, int d,
+             int block, float topk, cudaStream_t st) {
+  SAGESLA_TRY(validate(q, k, v, out, B, H, N, d, block, topk));
+  if (proj_w && !aligned16(proj_w)) return SAGESLA_ERR_MISALIGNED;
+  int dev = 0;
+  SAGESLA_TRY(check_device(&dev));
+  const Geom g = make_geom(B, H, N, block, topk);
+  const Buffers sizes = carve(nullptr, g);
+  uint8_t* base = nullptr;
+  SAGESLA_TRY(get_workspace(dev, st, sizes.total, &base));
+  const Buffers b = carve(base, g);
+  SAGESLA_TRY(run_front(q, k, v, g, b, st));
+  const bool dense = g.kc == g.nb;
+  if (!dense) {
+    ProfScope ps(3, st);
+    SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, b.idx, nullptr, nullptr, st)));
+  }
+  if (proj_w && !dense) return SAGESLA_ERR_INVALID;  // linear branch: not built yet
+  FlashArgs fa;
+  std::memset(&fa, 0, sizeof(fa));
+  fa.q8t = b.q8t;
+  fa.k8t = b.k8t;
+  fa.v8t = b.v8t;
+  fa.sq = b.sq;
+  fa.sk = b.sk;
+  fa.sv = b.sv;
+  fa.idx = dense ? nullptr : b.idx;
+  fa.out = out;
+  {
+    ProfScope ps(6, st);
+    SAGESLA_TRY(launch_rc(launch_flash(fa, g, st, watchdog(dev))));
+  }
+  return SAGESLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sagesla_topk_count(int nb, float topk) {
+  double t = (double)topk * (double)nb;
+  t -= t * 1e-6;
+  int k = (int)std::ceil(t);
+  if (k < 1) k = 1;
+  if (k > nb) k = nb;
+  return k;
+}
+
+int sagesla_attn(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B, int H, int N,
+                 int d, int block, float topk, sagesla_stream_t stream) {
+  return run_attn(q, k, v, proj_w, out, B, H, N, d, block, topk, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dense_int8_attn(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,
+                    sagesla_stream_t stream) {
+  return run_attn(q, k, v, nullptr, out, B, H, N, d, 64, 1.0f, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int sagesla_attn_host(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B, int H,
+                      int N, int d, int block, float topk, sagesla_stream_t stream) {
+  SAGESLA_TRY(validate(q, k, v, out, B, H, N, d, block, topk));
+  int dev = 0;
+  SAGESLA_TRY(check_device(&dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t E = (size_t)B * H * N * d * 2;  // bytes of one bf16 tensor
+  const size_t W = (size_t)d * d * 2;
+  // Device staging lives in its own cached region, keyed by a distinct stream tag.
+  static std::mutex smu;
+  static std::map<std::pair<int, cudaStream_t>, Workspace> stage;
+  uint8_t* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(smu);
+    Workspace& w = stage[std::make_pair(dev, st)];
+    const size_t need = 4 * up(E) + up(W);
+    if (w.bytes < need) {
+      if (w.ptr) cudaFreeAsync(w.ptr, st);
+      w.ptr = nullptr;
+      w.bytes = 0;
+      if (cudaMallocAsync(&w.ptr, need, st) != cudaSuccess) {
+        cudaGetLastError();
+        return SAGESLA_ERR_OOM;
+      }
+      w.bytes = need;
+    }
+    base = static_cast<uint8_t*>(w.ptr);
+  }
+  uint8_t* dq = base;
+  uint8_t* dk = dq + up(E);
+  uint8_t* dv = dk + up(E);
+  uint8_t* dout = dv + up(E);
+  uint8_t* dw = dout + up(E);
+  if (cudaMemcpyAsync(dq, q, E, cudaMemcpyHostToDevice, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
+  if (cudaMemcpyAsync(dk, k, E, cudaMemcpyHostToDevice, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
+  if (cudaMemcpyAsync(dv, v, E, cudaMemcpyHostToDevice, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
+  if (proj_w && cudaMemcpyAsync(dw, proj_w, W, cudaMemcpyHostToDevice, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
+  SAGESLA_TRY(run_attn(dq, dk, dv, proj_w ? dw : nullptr, dout, B, H, N, d, block, topk, st));
+  if (cudaMemcpyAsync(out, dout, E, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
+  return SAGESLA_OK;
+}
+
+int sagesla_get_quant(const void* q, const void* k, const void* v, int B, int H, int N, int d, int8_t* q8,
+                      int8_t* k8, uint8_t* v8, float* sq, float* sk, float* sv, float* mu, sagesla_stream_t stream) {
+  SAGESLA_TRY(validate(q, k, v, q8, B, H, N, d, 64, 1.0f));
+  if (!k8 || !v8 || !sq || !sk || !sv || !mu) return SAGESLA_ERR_INVALID;
+  int dev = 0;
+  SAGESLA_TRY(check_device(&dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Geom g = make_geom(B, H, N, 64, 1.0f);
+  const Buffers sizes = carve(nullptr, g);
+  uint8_t* base = nullptr;
+  SAGESLA_TRY(get_workspace(dev, st, sizes.total, &base));
+  const Buffers b = carve(base, g);
+  SAGESLA_TRY(run_front(q, k, v, g, b, st));
+  SAGESLA_TRY(launch_rc(launch_untile(b.q8t, b.k8t, b.v8t, g, q8, k8, v8, st)));
+  const int nq64 = (N + 63) / 64;
+  const size_t pitch = (size_t)g.nq * sizeof(float);
+  if (cudaMemcpy2DAsync(sq, nq64 * sizeof(float), b.sq, pitch, nq64 * sizeof(float), g.BH, cudaMemcpyDeviceToDevice,
+                        st) != cudaSuccess)
+    return SAGESLA_ERR_LAUNCH;
+  if (cudaMemcpy2DAsync(sk, nq64 * sizeof(float), b.sk, pitch, nq64 * sizeof(float), g.BH, cudaMemcpyDeviceToDevice,
+                        st) != cudaSuccess)
+    return SAGESLA_ERR_LAUNCH;
+  if (cudaMemcpyAsync(sv, b.sv, (size_t)g.BH * kD * sizeof(float), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return SAGESLA_ERR_LAUNCH;
+  if (cudaMemcpyAsync(mu, b.mu, (size_t)g.BH * kD * sizeof(float), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return SAGESLA_ERR_LAUNCH;
+  return SAGESLA_OK;
+}
+
+int sagesla_get_mask(const void* q, const void* k, int B, int H, int N, int d, int block, float topk,
+                     int32_t* idx_out, float* qbar, float* kbar, int* k_out, sagesla_stream_t stream) {
+  SAGESLA_TRY(validate(q, k, k, idx_out, B, H, N, d, block, topk));
+  int dev = 0;
+  SAGESLA_TRY(check_device(&dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Geom g = make_geom(B, H, N, block, topk);
+  const Buffers sizes = carve(nullptr, g);
+  uint8_t* base = nullptr;
+  SAGESLA_TRY(get_workspace(dev, st, sizes.total, &base));
+  const Buffers b = carve(base, g);
+  // The mask needs only K's mean and the pooled sums; V is read as K here
+  // (its quantised codes are discarded).
+  SAGESLA_TRY(run_front(q, k, k, g, b, st));
+  SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, idx_out, qbar, kbar, st)));
+  if (k_out) *k_out = g.kc;
+  return SAGESLA_OK;
+}
+
+int sagesla_sync_status(sagesla_stream_t stream) {
+  int dev = 0;
+  SAGESLA_TRY(check_device(&dev));
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
+  int* wd = watchdog(dev);
+  int h = 0;
+  if (cudaMemcpy(&h, wd, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
+  if (h) {
+    cudaMemset(wd, 0, sizeof(int));
+    return SAGESLA_ERR_DEVICE_TIMEOUT;
+  }
+  return SAGESLA_OK;
+}
+
+const char* sagesla_strerror(int code) {
+  switch (code) {
+    case SAGESLA_OK: return "ok";
+    case SAGESLA_ERR_INVALID: return "invalid argument";
+    case SAGESLA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case SAGESLA_ERR_OOM: return "workspace allocation failed";
+    case SAGESLA_ERR_LAUNCH: return "CUDA launch or runtime error";
+    case SAGESLA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+    case SAGESLA_ERR_NO_DEVICE: return "current device is not an sm_100 GPU";
+    default: return "unknown error";
+  }
+}
+
+void sagesla_profile(int enable) {
+  std::lock_guard<std::mutex> lk(g_pmu);
+  g_prof_on = enable != 0;
+}
+
+int sagesla_profile_read(double* ms, int* launches, int nkernels) {
+  std::lock_guard<std::mutex> lk(g_pmu);
+  for (int i = 0; i < nkernels; ++i) {
+    if (ms) ms[i] = 0.0;
+    if (launches) launches[i] = 0;
+  }
+  int rc = SAGESLA_OK;
+  for (auto& r : g_prof) {
+    if (cudaEventSynchronize(r.b) != cudaSuccess) rc = SAGESLA_ERR_LAUNCH;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) rc = SAGESLA_ERR_LAUNCH;
+    if (r.kernel >= 0 && r.kernel < nkernels) {
+      if (ms) ms[r.kernel] += t;
+      if (launches) launches[r.kernel] += 1;
+    }
+    g_evpool.push_back(r.a);
+    g_evpool.push_back(r.b);
+  }
+  g_prof.clear();
+  return rc;
+}
+
+void sagesla_release(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  cudaDeviceSynchronize();
+  for (auto& kv : g_ws)
+    if (kv.second.ptr) cudaFree(kv.second.ptr);
+  g_ws.clear();
+}
+
+}  // extern "C"

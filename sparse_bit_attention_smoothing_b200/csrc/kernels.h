@@ -1,0 +1,55 @@
+// kernels.h -- host-side launchers of the SageSLA kernels (internal; the
+// public C ABI is include/sagesla.h).  All launchers are asynchronous on
+// `st` and return the cudaGetLastError() of their launch.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace sagesla {
+
+// Geometry shared by the launchers.
+struct Geom {
+  int BH;      // B*H
+  int N;       // tokens
+  int block;   // 64 or 128 (mask block)
+  int nb;      // ceil(N/block)
+  int nq;      // 64-token quantisation tiles per head, padded: 2*ceil(N/128)
+  int kc;      // key blocks kept per query block
+  int split;   // row splits of the statistics pass
+};
+
+// K1: per-split fp64 sums of K and fp32 max|V| per channel.
+cudaError_t launch_stats_partial(const void* k, const void* v, const Geom& g, double* psum, float* pmax,
+                                 cudaStream_t st);
+// K1b: mu = fl32(sum/N); V scale amax/448 and multiplier 448/amax per channel.
+cudaError_t launch_stats_final(const double* psum, const float* pmax, const Geom& g, float* mu, float* sv,
+                               float* mv, cudaStream_t st);
+// K2: smoothing + INT8 Q/K tiles + FP8 V^T tiles + per-64-row pooled sums.
+cudaError_t launch_quant(const void* q, const void* k, const void* v, const float* mu, const float* mv,
+                         const Geom& g, uint8_t* q8t, uint8_t* k8t, uint8_t* v8t, float* sq, float* sk,
+                         float* qsum, float* ksum, cudaStream_t st);
+// Untile the quantised tiles back to row-major codes (parity entry only).
+cudaError_t launch_untile(const uint8_t* q8t, const uint8_t* k8t, const uint8_t* v8t, const Geom& g, int8_t* q8,
+                          int8_t* k8, uint8_t* v8, cudaStream_t st);
+// K3: pooled block scores and the per-query-block top-k list (ascending).
+cudaError_t launch_pool_topk(const float* qsum, const float* ksum, const Geom& g, int32_t* idx, float* qbar,
+                             float* kbar, cudaStream_t st);
+// K5: block-sparse INT8/FP8 flash attention over the index lists.
+struct FlashArgs {
+  const uint8_t* q8t;
+  const uint8_t* k8t;
+  const uint8_t* v8t;
+  const float* sq;
+  const float* sk;
+  const float* sv;
+  const int32_t* idx;  // [BH][nb][kc]; NULL = dense (every block, ascending)
+  void* out;           // bf16 [BH][N][128]
+  // linear branch (all NULL when off)
+  const void* q;       // bf16 input Q (for phi(Q))
+  const uint16_t* hlin;  // bf16 H_i images [BH][nb][128*128] (B operand layout)
+  const float* zlin;     // fp32 Z_i [BH][nb][128]
+  const uint16_t* wt;    // bf16 proj_w image (B operand layout), 32 KB
+};
+cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int* wd);
+
+}  // namespace sagesla

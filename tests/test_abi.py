@@ -1,0 +1,67 @@
+"""The C-ABI library loads and exports every symbol include/sagesla.h declares;
+host-side argument checks reject bad calls before any CUDA work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_bit_attention_smoothing_b200 import build as sbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    sbuild.build()
+    import sparse_bit_attention_smoothing_b200 as s
+    return s.lib()
+
+
+def declared_functions():
+    txt = open(os.path.join(ROOT, "include", "sagesla.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(?:int|void|const char\*)\s+(\w+)\s*\(", txt)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_topk_count_matches_oracle(L, orc):
+    for nb in (1, 7, 10, 16, 512, 591, 1182, 5000):
+        for t in (0.01, 0.05, 0.1, 0.15, 0.25, 0.3, 0.5, 0.99, 1.0):
+            assert L.sagesla_topk_count(nb, ctypes.c_float(t)) == orc.topk_count(nb, t), (nb, t)
+
+
+def test_strerror(L):
+    for c in (0, -1, -2, -3, -4, -5, -6, -99):
+        assert isinstance(L.sagesla_strerror(c), bytes)
+
+
+F = ctypes.c_float
+
+
+def test_rejects_bad_arguments_without_launch(L):
+    P = ctypes.c_void_p
+    a = P(0x10000)
+    cases = [
+        (None, a, a, None, a, 1, 1, 64, 128, 64, F(0.1)),   # null q
+        (a, a, a, None, a, 1, 1, 64, 64, 64, F(0.1)),       # d != 128
+        (a, a, a, None, a, 1, 1, 64, 128, 32, F(0.1)),      # bad block
+        (a, a, a, None, a, 1, 1, 64, 128, 64, F(0.0)),      # topk = 0
+        (a, a, a, None, a, 1, 1, 64, 128, 64, F(1.5)),      # topk > 1
+        (a, a, a, None, a, 1, 1, 64, 128, 64, F(float("nan"))),
+        (a, a, a, None, a, 0, 1, 64, 128, 64, F(0.1)),      # B = 0
+        (a, a, a, None, a, 1, 1, 0, 128, 64, F(0.1)),       # N = 0
+        (a, a, a, None, a, 300, 300, 64, 128, 64, F(0.1)),  # B*H > 65535
+    ]
+    for c in cases:
+        assert L.sagesla_attn(*c, None) == -1, c
+    m = P(0x10008)
+    assert L.sagesla_attn(a, m, a, None, a, 1, 1, 64, 128, 64, F(0.1), None) == -2
+    assert L.sagesla_attn(a, a, a, m, a, 1, 1, 64, 128, 64, F(0.1), None) == -2
+    assert L.dense_int8_attn(a, a, None, a, 1, 1, 64, 128, None) == -1
