@@ -161,10 +161,17 @@ struct Buffers {
   uint8_t *q8t, *k8t, *v8t;
   float *sq, *sk, *qsum, *ksum;
   int32_t* idx;
+  // linear branch
+  uint8_t* hs;        // mask-GEMM B tiles of h_j (bf16)
+  float* z;           // z_j [BH][nb][128]
+  uint32_t* selbits;  // [BH][nb][2*nbt]
+  float* zl;          // Z_i [BH][nb][128]
+  uint16_t* himg;     // H_i^T images [BH][nb][128*128]
+  uint16_t* wimg;     // proj_w image
   size_t total;
 };
 
-Buffers carve(uint8_t* base, const Geom& g) {
+Buffers carve(uint8_t* base, const Geom& g, bool linear = false) {
   Buffers b;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -186,6 +193,20 @@ Buffers carve(uint8_t* base, const Geom& g) {
   b.qsum = reinterpret_cast<float*>(take(BH * g.nq * kD * sizeof(float)));
   b.ksum = reinterpret_cast<float*>(take(BH * g.nq * kD * sizeof(float)));
   b.idx = reinterpret_cast<int32_t*>(take(BH * g.nb * (size_t)g.kc * sizeof(int32_t)));
+  if (linear) {
+    const size_t nbt = (size_t)(g.nb + 63) / 64;
+    b.hs = take(BH * nbt * 64 * 16384 * 2);
+    b.z = reinterpret_cast<float*>(take(BH * g.nb * kD * sizeof(float)));
+    b.selbits = reinterpret_cast<uint32_t*>(take(BH * g.nb * 2 * nbt * sizeof(uint32_t)));
+    b.zl = reinterpret_cast<float*>(take(BH * g.nb * kD * sizeof(float)));
+    b.himg = reinterpret_cast<uint16_t*>(take(BH * g.nb * 16384 * sizeof(uint16_t)));
+    b.wimg = reinterpret_cast<uint16_t*>(take(16384 * sizeof(uint16_t)));
+  } else {
+    b.hs = nullptr;
+    b.z = b.zl = nullptr;
+    b.selbits = nullptr;
+    b.himg = b.wimg = nullptr;
+  }
   b.total = o;
   return b;
 }
@@ -223,17 +244,32 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
   int dev = 0;
   SAGESLA_TRY(check_device(&dev));
   const Geom g = make_geom(B, H, N, block, topk);
-  const Buffers sizes = carve(nullptr, g);
+  const bool dense = g.kc == g.nb;
+  // An empty complement (every key block selected) makes the linear branch 0.
+  const bool linear = proj_w != nullptr && !dense;
+  const Buffers sizes = carve(nullptr, g, linear);
   uint8_t* base = nullptr;
   SAGESLA_TRY(get_workspace(dev, st, sizes.total, &base));
-  const Buffers b = carve(base, g);
+  const Buffers b = carve(base, g, linear);
   SAGESLA_TRY(run_front(q, k, v, g, b, st));
-  const bool dense = g.kc == g.nb;
+  int* wd = watchdog(dev);
+  if (linear) {
+    {
+      ProfScope ps(7, st);
+      SAGESLA_TRY(launch_rc(launch_w_tile(proj_w, b.wimg, st)));
+    }
+    ProfScope ps(4, st);
+    SAGESLA_TRY(launch_rc(launch_linear_kv(k, v, g, b.hs, b.z, wd, st)));
+  }
   if (!dense) {
     ProfScope ps(3, st);
-    SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, b.idx, nullptr, nullptr, st)));
+    SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, b.idx, nullptr, nullptr, linear ? b.z : nullptr,
+                                           b.selbits, b.zl, st)));
   }
-  if (proj_w && !dense) return SAGESLA_ERR_INVALID;  // linear branch: not built yet
+  if (linear) {
+    ProfScope ps(5, st);
+    SAGESLA_TRY(launch_rc(launch_linear_sum(b.hs, b.selbits, g, b.himg, wd, st)));
+  }
   FlashArgs fa;
   std::memset(&fa, 0, sizeof(fa));
   fa.q8t = b.q8t;
@@ -244,9 +280,15 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
   fa.sv = b.sv;
   fa.idx = dense ? nullptr : b.idx;
   fa.out = out;
+  if (linear) {
+    fa.q = q;
+    fa.hlin = b.himg;
+    fa.zlin = b.zl;
+    fa.wt = b.wimg;
+  }
   {
     ProfScope ps(6, st);
-    SAGESLA_TRY(launch_rc(launch_flash(fa, g, st, watchdog(dev))));
+    SAGESLA_TRY(launch_rc(launch_flash(fa, g, st, wd)));
   }
   return SAGESLA_OK;
 }
@@ -360,7 +402,7 @@ int sagesla_get_mask(const void* q, const void* k, int B, int H, int N, int d, i
   // The mask needs only K's mean and the pooled sums; V is read as K here
   // (its quantised codes are discarded).
   SAGESLA_TRY(run_front(q, k, k, g, b, st));
-  SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, idx_out, qbar, kbar, st)));
+  SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, idx_out, qbar, kbar, nullptr, nullptr, nullptr, st)));
   if (k_out) *k_out = g.kc;
   return SAGESLA_OK;
 }

@@ -49,7 +49,15 @@ struct Params {
   __nv_bfloat16* out;
   int* wd;
   int N, nb, nq, kc, nsteps;
+  // linear branch (linear == 0: off)
+  const uint16_t* qraw;  // bf16 Q [BH][N][128]
+  const uint8_t* himg;   // H_i^T operand images [BH][nb][32 KB]
+  const float* zl;       // Z_i [BH][nb][128]
+  const uint8_t* wimg;   // proj_w operand image, 32 KB
+  int linear;
 };
+constexpr int kImg = 128 * 128 * 2;  // one bf16 128x128 operand image
+constexpr uint32_t kImg_LBO = 128, kImg_SBO = 2048;
 
 template <int MODE>
 struct Cfg {
@@ -63,8 +71,13 @@ struct Cfg {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKStage;
   static constexpr int kOffP = kOffV + kStages * kVStage;
-  static constexpr int kOffBar = kOffP + 2 * kPBuf;
+  static constexpr int kOffW = kOffP + 2 * kPBuf;    // proj_w image (linear branch)
+  static constexpr int kOffBar = kOffW + kImg;
   static constexpr int kSmem = kOffBar + 256 + 1024;  // barriers + alignment slack
+  // After the main loop the K ring holds the H_i images and the V ring the
+  // phi(Q) operand; the P buffers hold O_l.
+  static_assert(kStages * kKStage >= (MODE == 0 ? 2 : 1) * kImg, "K ring too small for H");
+  static_assert(kStages * kVStage >= kQBytes * 2, "V ring too small for phi(Q)");
 };
 
 struct Bars {
@@ -74,6 +87,7 @@ struct Bars {
   uint64_t s_full[2], p_full[2];
   uint64_t o_done;
   uint64_t fin;
+  uint64_t w_full, h_full, phi_ready, n_done, ol_ready, y_done;
   uint32_t tmem;
   int abort;
 };
@@ -113,6 +127,12 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
     }
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->fin, 1);
+    mbar_init(&bars->w_full, 1);
+    mbar_init(&bars->h_full, 1);
+    mbar_init(&bars->phi_ready, kSoftThreads);
+    mbar_init(&bars->n_done, 1);
+    mbar_init(&bars->ol_ready, kSoftThreads);
+    mbar_init(&bars->y_done, 1);
     bars->abort = 0;
     mbar_fence_init();
   }
@@ -143,6 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         bulk_g2s(smem + C::kOffQ + kTile, p.q8t + (head_tiles + ib) * kTile, kTile, &bars->q_full);
       } else {
         bulk_g2s(smem + C::kOffQ, p.q8t + (head_tiles + 2 * iA) * kTile, 2 * kTile, &bars->q_full);
+      }
+      if (p.linear) {
+        mbar_expect_tx(&bars->w_full, kImg);
+        bulk_g2s(smem + C::kOffW, p.wimg, kImg, &bars->w_full);
       }
       int k_issued = 0, v_issued = 0;  // steps whose copies were issued
       for (int s = 0; s < nsteps && !*abort; ++s) {
@@ -189,6 +213,19 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         mbar_wait_drain(&bars->k_full[s % kStages], (s / kStages) & 1, p.wd);
       for (int s = max(0, v_issued - kStages); s < v_issued; ++s)
         mbar_wait_drain(&bars->v_full[s % kStages], (s / kStages) & 1, p.wd);
+      if (p.linear) {
+        // The K ring is free once every MMA of the main loop has completed.
+        if (v_issued == nsteps && mbar_wait(&bars->fin, 0, abort, p.wd)) {
+          const int nh = MODE == 0 ? 2 : 1;
+          mbar_expect_tx(&bars->h_full, nh * kImg);
+          for (int x = 0; x < nh; ++x) {
+            const int i = (x == 0 || !hasB) ? iA : iB;
+            bulk_g2s(smem + C::kOffK + x * kImg, p.himg + ((size_t)bh * p.nb + i) * kImg, kImg, &bars->h_full);
+          }
+          mbar_wait_drain(&bars->h_full, 0, p.wd);
+        }
+        mbar_wait_drain(&bars->w_full, 0, p.wd);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ----------------------------
@@ -266,6 +303,40 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       // Every MMA issued must be complete before TMEM is released.
       mma_commit(&bars->fin);
       mbar_wait_drain(&bars->fin, 0, p.wd);
+      if (p.linear && ok) {
+        // num = phi(Q_i) H_i -> S0 columns;  y = O_l W^T -> S1 columns.
+        const int M = MODE == 0 ? 64 : 128;
+        const uint32_t id = idesc_bf16(M, 128);
+        ok = mbar_wait(&bars->h_full, 0, abort, p.wd) && mbar_wait(&bars->w_full, 0, abort, p.wd) &&
+             mbar_wait(&bars->phi_ready, 0, abort, p.wd);
+        if (ok) {
+          tc_fence_after();
+          for (int x = 0; x < (MODE == 0 ? (hasB ? 2 : 1) : 1); ++x) {
+            const uint8_t* a = smem + C::kOffV + x * (kImg / 2);
+            const uint8_t* b = smem + C::kOffK + x * kImg;
+            const uint32_t d = tmem + kColS0 + ((uint32_t)(x * 16) << 16);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              mma_bf16(d, smem_desc(a + ks * 256, kImg_LBO, kImg_SBO), smem_desc(b + ks * 256, kImg_LBO, kImg_SBO),
+                       id, ks > 0);
+          }
+          mma_commit(&bars->n_done);
+          ok = mbar_wait(&bars->ol_ready, 0, abort, p.wd);
+        }
+        if (ok) {
+          tc_fence_after();
+          for (int x = 0; x < (MODE == 0 ? (hasB ? 2 : 1) : 1); ++x) {
+            const uint8_t* a = smem + C::kOffP + x * (kImg / 2);
+            const uint32_t d = tmem + kColS1 + ((uint32_t)(x * 16) << 16);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              mma_bf16(d, smem_desc(a + ks * 256, kImg_LBO, kImg_SBO),
+                       smem_desc(smem + C::kOffW + ks * 256, kImg_LBO, kImg_SBO), id, ks > 0);
+          }
+          mma_commit(&bars->y_done);
+          mbar_wait_drain(&bars->y_done, 0, p.wd);
+        }
+      }
     }
   } else {
     // ------------------------------ softmax -------------------------------
@@ -396,6 +467,64 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
     // it), which a parity wait cannot tell apart; `fin` has a single phase,
     // committed after the MMA thread's last instruction.
     if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->fin, 0, abort, p.wd));
+    const bool store = active && n < p.N;
+    const uint32_t ybase = tmem + lane_base + kColS1;
+    if (ok && nsteps > 0 && p.linear) {
+      // ---- linear branch: phi(q_r) . H_i / phi(q_r) . Z_i, then . W^T ----
+      const int xo = (MODE == 0 && lane >= 16) ? 1 : 0;  // operand half of this row
+      uint8_t* phiq = smem + C::kOffV + xo * (kImg / 2);
+      uint8_t* olr = smem + C::kOffP + xo * (kImg / 2);
+      const uint4* qrow = reinterpret_cast<const uint4*>(p.qraw + ((size_t)bh * p.N + (store ? n : 0)) * kD);
+      const float* zrow = p.zl + ((size_t)bh * p.nb + (active ? i : 0)) * kD;
+      float den = 0.f;
+#pragma unroll 4
+      for (int ch = 0; ch < 16; ++ch) {  // 8 channels per 16-byte chunk
+        uint4 qq = store ? __ldg(qrow + ch) : make_uint4(0, 0, 0, 0);
+        const uint32_t w4[4] = {qq.x, qq.y, qq.z, qq.w};
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = bf16_lo(w4[e]), b = bf16_hi(w4[e]);
+          const float fa = a > 0.f ? a + 1.f : __expf(a);
+          const float fb = b > 0.f ? b + 1.f : __expf(b);
+          den = fmaf(fa, __ldg(zrow + 8 * ch + 2 * e), den);
+          den = fmaf(fb, __ldg(zrow + 8 * ch + 2 * e + 1), den);
+          const __nv_bfloat162 h = __floats2bfloat162_rn(fa, fb);
+          pk[e] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(phiq + kmajor_off(row, ch * 16, kImg_LBO, kImg_SBO)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->phi_ready);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->n_done, 0, abort, p.wd));
+      if (ok) {
+        tc_fence_after();
+        const float inv_den = (store && den > 0.f) ? 1.f / den : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < kD; c += 16) {
+          uint32_t v16[16];
+          SAGESLA_TMEM_LD16(tmem + lane_base + kColS0 + c, v16);
+          tmem_ld_wait();
+          uint32_t pk[8];
+#pragma unroll
+          for (int z = 0; z < 8; ++z) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v16[2 * z]) * inv_den,
+                                                           __uint_as_float(v16[2 * z + 1]) * inv_den);
+            pk[z] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          *reinterpret_cast<uint4*>(olr + kmajor_off(row, c * 2, kImg_LBO, kImg_SBO)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(olr + kmajor_off(row, c * 2 + 16, kImg_LBO, kImg_SBO)) =
+              make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars->ol_ready);
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_done, 0, abort, p.wd));
+      }
+    }
     if (ok && nsteps > 0) {
       tc_fence_after();
       const uint32_t obase = tmem + lane_base + kColO;
@@ -403,19 +532,25 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       SAGESLA_TMEM_LD16(obase + 128, lw);
       tmem_ld_wait();
       const float inv_l = 1.f / __uint_as_float(lw[0]);
-      const bool store = active && n < p.N;
       __nv_bfloat16* orow = p.out + ((size_t)bh * p.N + (store ? n : 0)) * kD;
 #pragma unroll 1
       for (int c = 0; c < kD; c += 16) {
-        uint32_t o[16];
+        uint32_t o[16], y[16];
         SAGESLA_TMEM_LD16(obase + c, o);
+        if (p.linear) {
+          SAGESLA_TMEM_LD16(ybase + c, y);
+        }
         tmem_ld_wait();
         if (store) {
           uint32_t pk[8];
 #pragma unroll
           for (int z = 0; z < 8; ++z) {
-            const float a = __uint_as_float(o[2 * z]) * inv_l * __ldg(p.sv + (size_t)bh * kD + c + 2 * z);
-            const float b = __uint_as_float(o[2 * z + 1]) * inv_l * __ldg(p.sv + (size_t)bh * kD + c + 2 * z + 1);
+            float a = __uint_as_float(o[2 * z]) * inv_l * __ldg(p.sv + (size_t)bh * kD + c + 2 * z);
+            float b = __uint_as_float(o[2 * z + 1]) * inv_l * __ldg(p.sv + (size_t)bh * kD + c + 2 * z + 1);
+            if (p.linear) {
+              a += __uint_as_float(y[2 * z]);
+              b += __uint_as_float(y[2 * z + 1]);
+            }
             const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
             pk[z] = *reinterpret_cast<const uint32_t*>(&h);
           }
@@ -445,6 +580,11 @@ cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int
   p.nb = g.nb;
   p.nq = g.nq;
   p.kc = g.kc;
+  p.qraw = reinterpret_cast<const uint16_t*>(a.q);
+  p.himg = reinterpret_cast<const uint8_t*>(a.hlin);
+  p.zl = a.zlin;
+  p.wimg = reinterpret_cast<const uint8_t*>(a.wt);
+  p.linear = (a.hlin && a.zlin && a.wt && a.q) ? 1 : 0;
   if (g.block == 64) {
     p.nsteps = (g.kc + 1) / 2;
     const int smem = Cfg<0>::kSmem;

@@ -1,0 +1,368 @@
+// k_linear.cu -- the SLA linear-attention branch, part 1 and 2.
+//
+// "揭秘TurboDiffusion：如何让视频生成实现百倍加速？" 支柱二 SLA and
+// "TurboDiffusion跨模态" 2.2: besides the exactly computed blocks, a light
+// global linear-attention component (kernel-function approximation) covers
+// the rest.  Read as phi(Q)(phi(K)^T V) over the key blocks NOT selected for
+// query block i, phi = elu + 1, from the raw bf16 Q, K, V:
+//   h_j = phi(K_j)^T V_j  (d x d),  z_j = sum of the rows of phi(K_j)
+//   H_i = sum_{j not in S_i} h_j   (a 0/1 complement-mask GEMM per head)
+//
+// K4a linear_kv:  per pair of key blocks, h_j on tcgen05 (kind::f16, both
+//   operands MN-major straight from the token-major rows), fp32 accumulate,
+//   stored in bf16 as the B tiles of the mask GEMM; z_j in fp32.
+// K4b linear_sum: per head, H = (1 - M) . Hstack with tcgen05 (M=128 query
+//   blocks x N=256 columns of the d*d matrices, K = key blocks); the 0/1 A
+//   tiles are expanded in shared memory from the selection bitmask.  Each
+//   output row is the bf16 image of H_i^T in the operand layout the flash
+//   kernel's epilogue MMA reads (so it is one bulk copy there).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sagesla {
+
+namespace {
+
+// Layout of H_i^T as a K-major bf16 B operand [N = cv][K = ck]:
+// element (cv, ck) at (cv/8)*2048 + (ck/8)*128 + (cv%8)*16 + (ck%8)*2 bytes.
+__device__ __forceinline__ uint32_t himg_off(uint32_t cv, uint32_t ck) {
+  return (cv >> 3) * 2048u + (ck >> 3) * 128u + (cv & 7u) * 16u + (ck & 7u) * 2u;
+}
+
+// Mask-GEMM B tiles (64 key blocks x 256 image columns), MN-major: element
+// (j, n) at (n%256/8)*1024 + (j%64/8)*128 + (j%8)*16 + (n%8)*2 within the
+// 32 KB tile of (j/64, n/256).  Tiles ordered [n/256][j/64].
+constexpr int kHsTile = 64 * 256 * 2;  // 32 KB
+constexpr uint32_t kHs_LBO = 128, kHs_SBO = 1024;
+
+__device__ __forceinline__ size_t hs_chunk(int nbt, int j, int chunk) {
+  // chunk = n / 8 (16-byte group of 8 bf16)
+  const int nt = chunk >> 5, c = chunk & 31;
+  return ((size_t)nt * nbt + (j >> 6)) * kHsTile + (size_t)c * kHs_SBO + ((j & 63) >> 3) * kHs_LBO + (j & 7) * 16;
+}
+
+__device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- K4a ----
+// grid (nbt*32, BH): CTA x handles key blocks j = 2x, 2x+1 (zeros past nb).
+// 128 threads; thread 0 issues the MMAs.  Dynamic smem: per block, A (phi(K)
+// rows) and B (V rows) MN-major, BLK x 128 bf16 each; plus the 32 KB image.
+template <int BLK>
+__global__ void __launch_bounds__(128) linear_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int N,
+                                                        int nb, int nbt, uint8_t* __restrict__ hs,
+                                                        float* __restrict__ z, int* wd) {
+  constexpr int kOpBytes = BLK * 128 * 2;  // one operand tile
+  constexpr uint32_t kSBO = (BLK / 8) * 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* img = smem + 4 * kOpBytes;          // 32 KB staging of one h image
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+  __shared__ float zred[4][128];
+  const int bh = blockIdx.y, t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int j0 = 2 * blockIdx.x;
+  const size_t base = (size_t)bh * N * 16;
+  if (t == 0) {
+    mbar_init(&bar, 1);
+    abort_s = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) tmem_alloc(&tmem_s, 256);
+  // Operands: thread t -> channel group cg = t%16 (8 channels), rows t/16 + 8r.
+  const int cg = t & 15, r0 = t >> 4;
+  float zacc[2][8];
+#pragma unroll
+  for (int b = 0; b < 2; ++b)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) zacc[b][c] = 0.f;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    const int j = j0 + b;
+    uint8_t* A = smem + (2 * b) * kOpBytes;
+    uint8_t* B = smem + (2 * b + 1) * kOpBytes;
+    for (int r = r0; r < BLK; r += 8) {
+      const int n = j * BLK + r;
+      uint4 kk = make_uint4(0, 0, 0, 0), vv = kk;
+      const bool valid = j < nb && n < N;
+      if (valid) {
+        kk = __ldg(k + base + (size_t)n * 16 + cg);
+        vv = __ldg(v + base + (size_t)n * 16 + cg);
+      }
+      const uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};
+      uint32_t pw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float f0 = valid ? phi(bf16_lo(kw[e])) : 0.f;
+        const float f1 = valid ? phi(bf16_hi(kw[e])) : 0.f;
+        zacc[b][2 * e] += f0;
+        zacc[b][2 * e + 1] += f1;
+        pw[e] = pack_bf16(f0, f1);
+      }
+      // MN-major core matrix: (m/8)*SBO + (tok/8)*128 + (tok%8)*16 + (m%8)*2
+      const uint32_t off = cg * kSBO + (r >> 3) * 128 + (r & 7) * 16;
+      *reinterpret_cast<uint4*>(A + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+      *reinterpret_cast<uint4*>(B + off) = vv;
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  if (t == 0) {
+    const uint32_t id = idesc_bf16(128, 128, 1) | (1u << 15);  // A and B MN-major
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const uint8_t* A = smem + (2 * b) * kOpBytes;
+      const uint8_t* B = smem + (2 * b + 1) * kOpBytes;
+#pragma unroll
+      for (int ks = 0; ks < BLK / 16; ++ks)
+        mma_bf16(tmem + b * 128, smem_desc(A + ks * 256, 128, kSBO), smem_desc(B + ks * 256, 128, kSBO), id, ks > 0);
+    }
+    mma_commit(&bar);
+  }
+  // z_j: reduce the per-thread channel sums over the 8 row groups.
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    const int j = j0 + b;
+    __syncthreads();
+    if (r0 < 4) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) zred[r0][cg * 8 + c] = zacc[b][c];
+    }
+    __syncthreads();
+    if (r0 >= 4) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) zred[r0 - 4][cg * 8 + c] += zacc[b][c];
+    }
+    __syncthreads();
+    if (j < nb) z[((size_t)bh * nb + j) * kD + t] = (zred[0][t] + zred[1][t]) + (zred[2][t] + zred[3][t]);
+  }
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar, 0, &abort_s, wd));
+  tc_fence_after();
+  // h_j rows: warp w holds ck = 32w + lane; columns cv.  Stage as the bf16
+  // image, then copy 16-byte chunks (8 image columns) to the mask-GEMM tiles.
+  uint4* out0 = nullptr;
+  (void)out0;
+#pragma unroll 1
+  for (int b = 0; b < 2; ++b) {
+    const int j = j0 + b;
+    const int ck = 32 * warp + lane;
+#pragma unroll 1
+    for (int c0 = 0; c0 < 128; c0 += 16) {
+      uint32_t r[16];
+      SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * warp) << 16) + b * 128 + c0, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float val = ok ? __uint_as_float(r[e]) : 0.f;
+        *reinterpret_cast<__nv_bfloat16*>(img + himg_off(c0 + e, ck)) = __float2bfloat16_rn(val);
+      }
+    }
+    __syncthreads();
+    // 2048 chunks of 16 bytes; block j's chunk goes next to block j^1's.
+    for (int c = t; c < 2048; c += 128)
+      *reinterpret_cast<uint4*>(hs + (size_t)bh * nbt * 64 * 16384 * 2 + hs_chunk(nbt, j, c)) =
+          *reinterpret_cast<const uint4*>(img + c * 16);
+    __syncthreads();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------- K4b ----
+// grid (64 n-tiles, ceil(nb/128) i-tiles, BH).  192 threads: warp 0 bulk
+// loads the B tiles, warp 1 issues MMAs, warps 2-5 expand the 0/1 A tiles
+// from the selection bitmask and run the epilogue.  K tiles of 64 key
+// blocks, 2-stage ring; D = 128 x 256 fp32 in TMEM.
+namespace {
+constexpr int kLStages = 2;
+constexpr int kATile = 128 * 64 * 2;  // 16 KB
+struct LBars {
+  uint64_t b_full[kLStages], a_full[kLStages], empty[kLStages], done;
+  uint32_t tmem;
+  int abort;
+};
+}  // namespace
+
+__global__ void __launch_bounds__(192, 1) linear_sum_kernel(const uint8_t* __restrict__ hs,
+                                                             const uint32_t* __restrict__ selbits, int nb, int nbt,
+                                                             int nbw, uint16_t* __restrict__ hout, int* wd) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sB = smem;                               // kLStages x 32 KB
+  uint8_t* sA = smem + kLStages * kHsTile;          // kLStages x 16 KB
+  LBars* bars = reinterpret_cast<LBars*>(sA + kLStages * kATile);
+  volatile int* abort = &bars->abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nt = blockIdx.x, it = blockIdx.y, bh = blockIdx.z;
+  const int i0 = it * 128;
+  const uint8_t* hs_head = hs + (size_t)bh * nbt * 64 * 16384 * 2;
+  if (tid == 0) {
+    for (int s = 0; s < kLStages; ++s) {
+      mbar_init(&bars->b_full[s], 1);
+      mbar_init(&bars->a_full[s], 128);
+      mbar_init(&bars->empty[s], 1);
+    }
+    mbar_init(&bars->done, 1);
+    bars->abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(&bars->tmem, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem;
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int kt = 0; kt < nbt && !*abort; ++kt) {
+        const int st = kt % kLStages;
+        if (kt >= kLStages && !mbar_wait(&bars->empty[st], ((kt / kLStages) - 1) & 1, abort, wd)) break;
+        mbar_expect_tx(&bars->b_full[st], kHsTile);
+        bulk_g2s(sB + st * kHsTile, hs_head + ((size_t)nt * nbt + kt) * kHsTile, kHsTile, &bars->b_full[st]);
+        issued = kt + 1;
+      }
+      for (int kt = (issued > kLStages ? issued - kLStages : 0); kt < issued; ++kt)
+        mbar_wait_drain(&bars->b_full[kt % kLStages], (kt / kLStages) & 1, wd);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id = idesc_bf16(128, 256, 1);  // B MN-major
+      bool ok = true;
+      for (int kt = 0; kt < nbt && ok; ++kt) {
+        const int st = kt % kLStages;
+        ok = mbar_wait(&bars->a_full[st], (kt / kLStages) & 1, abort, wd) &&
+             mbar_wait(&bars->b_full[st], (kt / kLStages) & 1, abort, wd);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_bf16(tmem, smem_desc(sA + st * kATile + ks * 256, kQK_LBO, kQK_SBO),
+                   smem_desc(sB + st * kHsTile + ks * 2 * kHs_LBO, kHs_LBO, kHs_SBO), id, (kt > 0 || ks > 0));
+        mma_commit(&bars->empty[st]);
+      }
+      mma_commit(&bars->done);
+      mbar_wait_drain(&bars->done, 0, wd);
+    }
+  } else {
+    // A producer: thread -> query block row i = i0 + (tid - 64); 64 key
+    // blocks per K tile from two bitmask words; 1 = NOT selected, j < nb.
+    const int r = tid - 64;
+    const int i = i0 + r;
+    bool ok = true;
+    for (int kt = 0; kt < nbt; ++kt) {
+      const int st = kt % kLStages;
+      if (kt >= kLStages) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->empty[st], ((kt / kLStages) - 1) & 1, abort, wd));
+        if (!ok) break;
+      }
+      uint32_t w0 = 0, w1 = 0;
+      if (i < nb) {
+        w0 = selbits[((size_t)bh * nb + i) * nbw + 2 * kt];
+        w1 = selbits[((size_t)bh * nb + i) * nbw + 2 * kt + 1];
+      }
+      uint8_t* A = sA + st * kATile;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {  // 8 keys per 16-byte chunk
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint32_t h2 = 0;
+#pragma unroll
+          for (int z2 = 0; z2 < 2; ++z2) {
+            const int jj = ch * 8 + e * 2 + z2;  // key block within the tile
+            const int j = kt * 64 + jj;
+            const uint32_t bit = jj < 32 ? (w0 >> jj) & 1u : (w1 >> (jj - 32)) & 1u;
+            const bool one = i < nb && j < nb && !bit;
+            h2 |= (one ? 0x3F80u : 0u) << (16 * z2);
+          }
+          pk[e] = h2;
+        }
+        *reinterpret_cast<uint4*>(A + kmajor_off(r, ch * 16, kQK_LBO, kQK_SBO)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->a_full[st]);
+    }
+    // Epilogue: row i of D (256 fp32 columns) -> bf16 image columns.
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, abort, wd));
+    if (ok) {
+      tc_fence_after();
+      const int q = warp & 3;
+      const int row = 32 * q + lane;  // TMEM lane == row of the M=128 tile
+      const int ir = i0 + row;
+      uint16_t* dst = hout + ((size_t)bh * nb + (ir < nb ? ir : 0)) * 16384 + (size_t)nt * 256;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += 16) {
+        uint32_t v16[16];
+        SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * q) << 16) + c0, v16);
+        tmem_ld_wait();
+        if (ir < nb) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(__uint_as_float(v16[2 * e]), __uint_as_float(v16[2 * e + 1]));
+          *reinterpret_cast<uint4*>(dst + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(dst + c0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
+// ------------------------------------------------------------- W image ---
+// proj_w [c_out][c_in] row-major -> K-major B operand image [N=c_out][K=c_in].
+__global__ void w_tile_kernel(const uint16_t* __restrict__ w, uint16_t* __restrict__ wt) {
+  const int co = blockIdx.x, ci = threadIdx.x;
+  wt[himg_off(co, ci) / 2] = w[co * kD + ci];
+}
+
+int linear_kv_smem(int block) { return 4 * block * 128 * 2 + 32768 + 1024; }
+int linear_sum_smem() { return kLStages * (kHsTile + kATile) + (int)sizeof(LBars) + 1024; }
+
+cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_t* hs, float* z, int* wd,
+                             cudaStream_t st) {
+  const int nbt = (g.nb + 63) / 64;
+  const int smem = linear_kv_smem(g.block);
+  cudaError_t e;
+  if (g.block == 64) {
+    e = cudaFuncSetAttribute(linear_kv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    linear_kv_kernel<64><<<dim3(nbt * 32, g.BH), 128, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt, hs,
+                                                                  z, wd);
+  } else {
+    e = cudaFuncSetAttribute(linear_kv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    linear_kv_kernel<128><<<dim3(nbt * 32, g.BH), 128, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt,
+                                                                   hs, z, wd);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_linear_sum(const uint8_t* hs, const uint32_t* selbits, const Geom& g, uint16_t* hout, int* wd,
+                              cudaStream_t st) {
+  const int nbt = (g.nb + 63) / 64;
+  const int smem = linear_sum_smem();
+  cudaError_t e = cudaFuncSetAttribute(linear_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  linear_sum_kernel<<<dim3(64, (g.nb + 127) / 128, g.BH), 192, smem, st>>>(hs, selbits, g.nb, nbt, 2 * nbt, hout, wd);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_w_tile(const void* w, uint16_t* wt, cudaStream_t st) {
+  w_tile_kernel<<<kD, kD, 0, st>>>((const uint16_t*)w, wt);
+  return cudaGetLastError();
+}
+
+}  // namespace sagesla

@@ -36,10 +36,15 @@ __device__ __forceinline__ float pooled(const float* __restrict__ sums, int blk,
   return __fdiv_rn(a, (float)cnt);
 }
 
+// Linear-branch outputs (when zin != NULL): selbits [nb][nbw] words with
+// bit j set when key block j is selected; zout [nb][128] the fp32 sums
+// Z_i = sum_{j not in S_i} z_j, formed as (sum over all j) - (sum over S_i).
 __global__ void __launch_bounds__(256) pool_topk_kernel(const float* __restrict__ qsum, const float* __restrict__ ksum,
                                                         int N, int block, int nb, int nq, int kc,
                                                         int32_t* __restrict__ idx, float* __restrict__ qbar_out,
-                                                        float* __restrict__ kbar_out) {
+                                                        float* __restrict__ kbar_out, const float* __restrict__ zin,
+                                                        uint32_t* __restrict__ selbits, int nbw,
+                                                        float* __restrict__ zout) {
   extern __shared__ __align__(16) float sm[];
   float* qb = sm;                            // [kTQ][128]
   float* kb = qb + kTQ * kD;                 // [kKC][kPad]
@@ -97,6 +102,13 @@ __global__ void __launch_bounds__(256) pool_topk_kernel(const float* __restrict_
       sc[(2 * qg + 1) * nb + j] = a1 * rs;
     }
   }
+  // Total of z over all key blocks of the head (fixed order), for Z_i.
+  __shared__ float ztot[kD];
+  if (zin && t < kD) {
+    float a = 0.f;
+    for (int j = 0; j < nb; ++j) a += zin[((size_t)bh * nb + j) * kD + t];
+    ztot[t] = a;
+  }
   __syncthreads();
   // Phase 2: one warp per query row.
   const int i = i0 + warp;
@@ -128,20 +140,37 @@ __global__ void __launch_bounds__(256) pool_topk_kernel(const float* __restrict_
     const bool sel = j < nb && (key > T || (is_eq && eq_rank < need_eq));
     const unsigned sm_ = __ballot_sync(0xffffffffu, sel);
     if (sel) out[pos + __popc(sm_ & ((1u << lane) - 1u))] = j;
+    if (selbits && lane == 0) selbits[((size_t)bh * nb + i) * nbw + (j0 >> 5)] = sm_;
     pos += __popc(sm_);
     eq_seen += __popc(eqm);
+  }
+  if (selbits)
+    for (int w = ((nb + 31) >> 5) + lane; w < nbw; w += 32) selbits[((size_t)bh * nb + i) * nbw + w] = 0u;
+  if (zin) {
+    __syncwarp();
+    float zs[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) zs[m] = 0.f;
+    for (int tt = 0; tt < kc; ++tt) {
+      const int j = out[tt];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) zs[m] += zin[((size_t)bh * nb + j) * kD + lane + 32 * m];
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) zout[((size_t)bh * nb + i) * kD + lane + 32 * m] = ztot[lane + 32 * m] - zs[m];
   }
 }
 
 size_t pool_topk_smem(int nb) { return sizeof(float) * ((size_t)kTQ * kD + (size_t)kKC * kPad + (size_t)kTQ * nb); }
 
 cudaError_t launch_pool_topk(const float* qsum, const float* ksum, const Geom& g, int32_t* idx, float* qbar,
-                             float* kbar, cudaStream_t st) {
+                             float* kbar, const float* zin, uint32_t* selbits, float* zout, cudaStream_t st) {
   const size_t smem = pool_topk_smem(g.nb);
   cudaError_t e = cudaFuncSetAttribute(pool_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   pool_topk_kernel<<<dim3((g.nb + kTQ - 1) / kTQ, g.BH), 256, smem, st>>>(qsum, ksum, g.N, g.block, g.nb, g.nq, g.kc,
-                                                                           idx, qbar, kbar);
+                                                                           idx, qbar, kbar, zin, selbits,
+                                                                           2 * ((g.nb + 63) / 64), zout);
   return cudaGetLastError();
 }
 

@@ -121,3 +121,31 @@ def test_rows_past_n_untouched(sg):
     assert torch.isfinite(big[:, :, :100].float()).all()
     assert torch.all(big[:, :, 100:] == 7.0)
     assert sg.sync_status() == 0
+
+
+@pytest.mark.parametrize("B,H,N,outl", CASES)
+@pytest.mark.parametrize("block,topk", [(64, 0.25), (64, 0.3), (128, 0.3), (64, 0.05), (128, 0.5)])
+def test_full_path_with_linear_branch_vs_emulation(sg, orc, B, H, N, outl, block, topk):
+    q, k, v, w = _inputs(B, H, N, outl)
+    dq, dk, dv, dw = _dev(q, k, v, w)
+    out = sg.sagesla_attn(dq, dk, dv, dw, block=block, topk=topk)
+    m = sg.sagesla_get_mask(dq, dk, block=block, topk=topk)
+    torch.cuda.synchronize()
+    assert sg.sync_status() == 0
+    qf, kf, vf = (t.reshape(B * H, N, 128) for t in (q, k, v))
+    nb = (N + block - 1) // block
+    idx = m["idx"].cpu().numpy().reshape(B * H, nb, -1)
+    emu, _ = orc.sagesla(qf, kf, vf, w, block, topk, idx=idx)
+    _check_out(out.reshape(B * H, N, 128), emu)
+    # the branch is really there: it moves the result well beyond the tolerance
+    emu0, _ = orc.sagesla(qf, kf, vf, None, block, topk, idx=idx)
+    assert np.abs(emu - emu0).max() > 5e-2
+
+
+def test_linear_branch_topk_one_contributes_nothing(sg):
+    q, k, v, w = _inputs(1, 2, 700, True)
+    dq, dk, dv, dw = _dev(q, k, v, w)
+    a = sg.sagesla_attn(dq, dk, dv, dw, block=64, topk=1.0)
+    b = sg.dense_int8_attn(dq, dk, dv)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
