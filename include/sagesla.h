@@ -139,10 +139,11 @@ const char* sagesla_strerror(int code);
  * summed milliseconds and the number of launches since the last read, then
  * forgets them.  Kernel ids: 0 stats, 1 stats finalise, 2 quantise,
  * 3 pooled top-k, 4 linear per-block phi(K)^T V, 5 linear complement sum,
- * 6 sparse flash, 7 projection-weight tiling.  ms / launches are arrays of
- * nkernels entries (either may be NULL).  Profiling is off by default.
+ * 6 sparse flash, 7 projection-weight tiling, 8 linear output (phi(Q) H,
+ * normalisation, projection).  ms / launches are arrays of nkernels entries
+ * (either may be NULL).  Profiling is off by default.
  */
-#define SAGESLA_NUM_KERNELS 8
+#define SAGESLA_NUM_KERNELS 9
 void sagesla_profile(int enable);
 int sagesla_profile_read(double* ms, int* launches, int nkernels);
 

@@ -30,7 +30,8 @@ class SageSLAError(RuntimeError):
 EXPORTS = ["sagesla_attn", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
            "sagesla_topk_count", "sagesla_sync_status", "sagesla_strerror", "sagesla_release", "sagesla_profile",
            "sagesla_profile_read"]
-KERNELS = ["stats", "stats_final", "quant", "pool_topk", "linear_kv", "linear_sum", "flash", "w_tile"]
+KERNELS = ["stats", "stats_final", "quant", "pool_topk", "linear_kv", "linear_sum", "flash", "w_tile",
+           "linear_apply"]
 
 
 def lib():

@@ -161,6 +161,7 @@ struct Buffers {
   uint8_t *q8t, *k8t, *v8t;
   float *sq, *sk, *qsum, *ksum;
   int32_t* idx;
+  float *qbar, *kbar;  // pooled means [BH][nb][128]
   // linear branch
   uint8_t* hs;        // mask-GEMM B tiles of h_j (bf16)
   float* z;           // z_j [BH][nb][128]
@@ -193,6 +194,8 @@ Buffers carve(uint8_t* base, const Geom& g, bool linear = false) {
   b.qsum = reinterpret_cast<float*>(take(BH * g.nq * kD * sizeof(float)));
   b.ksum = reinterpret_cast<float*>(take(BH * g.nq * kD * sizeof(float)));
   b.idx = reinterpret_cast<int32_t*>(take(BH * g.nb * (size_t)g.kc * sizeof(int32_t)));
+  b.qbar = reinterpret_cast<float*>(take(BH * g.nb * kD * sizeof(float)));
+  b.kbar = reinterpret_cast<float*>(take(BH * g.nb * kD * sizeof(float)));
   if (linear) {
     const size_t nbt = (size_t)(g.nb + 63) / 64;
     b.hs = take(BH * nbt * 64 * 16384 * 2);
@@ -263,12 +266,16 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
   }
   if (!dense) {
     ProfScope ps(3, st);
-    SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, b.idx, nullptr, nullptr, linear ? b.z : nullptr,
+    SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, b.idx, b.qbar, b.kbar, linear ? b.z : nullptr,
                                            b.selbits, b.zl, st)));
   }
   if (linear) {
-    ProfScope ps(5, st);
-    SAGESLA_TRY(launch_rc(launch_linear_sum(b.hs, b.selbits, g, b.himg, wd, st)));
+    {
+      ProfScope ps(5, st);
+      SAGESLA_TRY(launch_rc(launch_linear_sum(b.hs, b.selbits, g, b.himg, wd, st)));
+    }
+    ProfScope ps(8, st);
+    SAGESLA_TRY(launch_rc(launch_linear_apply(q, b.himg, b.zl, b.wimg, g, out, wd, st)));
   }
   FlashArgs fa;
   std::memset(&fa, 0, sizeof(fa));
@@ -280,12 +287,7 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
   fa.sv = b.sv;
   fa.idx = dense ? nullptr : b.idx;
   fa.out = out;
-  if (linear) {
-    fa.q = q;
-    fa.hlin = b.himg;
-    fa.zlin = b.zl;
-    fa.wt = b.wimg;
-  }
+  fa.add_out = linear ? 1 : 0;
   {
     ProfScope ps(6, st);
     SAGESLA_TRY(launch_rc(launch_flash(fa, g, st, wd)));
@@ -402,7 +404,8 @@ int sagesla_get_mask(const void* q, const void* k, int B, int H, int N, int d, i
   // The mask needs only K's mean and the pooled sums; V is read as K here
   // (its quantised codes are discarded).
   SAGESLA_TRY(run_front(q, k, k, g, b, st));
-  SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, idx_out, qbar, kbar, nullptr, nullptr, nullptr, st)));
+  SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, idx_out, qbar ? qbar : b.qbar, kbar ? kbar : b.kbar,
+                                         nullptr, nullptr, nullptr, st)));
   if (k_out) *k_out = g.kc;
   return SAGESLA_OK;
 }

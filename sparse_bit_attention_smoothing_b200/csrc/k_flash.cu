@@ -29,7 +29,7 @@ namespace sagesla {
 namespace {
 
 constexpr int kStages = 2;
-constexpr int kSoftThreads = 128;
+constexpr int kSoftThreads = 256;  // two warps per TMEM lane quadrant
 constexpr int kThreads = 64 + kSoftThreads;
 constexpr int kVSlot = kTile + 1024;  // 8 KB V^T tile + 16 rows of ones (1 KB)
 constexpr uint32_t kOnesE4M3 = 0x38383838u;
@@ -49,15 +49,8 @@ struct Params {
   __nv_bfloat16* out;
   int* wd;
   int N, nb, nq, kc, nsteps;
-  // linear branch (linear == 0: off)
-  const uint16_t* qraw;  // bf16 Q [BH][N][128]
-  const uint8_t* himg;   // H_i^T operand images [BH][nb][32 KB]
-  const float* zl;       // Z_i [BH][nb][128]
-  const uint8_t* wimg;   // proj_w operand image, 32 KB
-  int linear;
+  int add_out;  // 1: out already holds the linear branch (bf16); add O_s to it
 };
-constexpr int kImg = 128 * 128 * 2;  // one bf16 128x128 operand image
-constexpr uint32_t kImg_LBO = 128, kImg_SBO = 2048;
 
 template <int MODE>
 struct Cfg {
@@ -71,13 +64,8 @@ struct Cfg {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKStage;
   static constexpr int kOffP = kOffV + kStages * kVStage;
-  static constexpr int kOffW = kOffP + 2 * kPBuf;    // proj_w image (linear branch)
-  static constexpr int kOffBar = kOffW + kImg;
-  static constexpr int kSmem = kOffBar + 256 + 1024;  // barriers + alignment slack
-  // After the main loop the K ring holds the H_i images and the V ring the
-  // phi(Q) operand; the P buffers hold O_l.
-  static_assert(kStages * kKStage >= (MODE == 0 ? 2 : 1) * kImg, "K ring too small for H");
-  static_assert(kStages * kVStage >= kQBytes * 2, "V ring too small for phi(Q)");
+  static constexpr int kOffBar = kOffP + 2 * kPBuf;
+  static constexpr int kSmem = kOffBar + 256 + 2048 + 1024;  // barriers, max exchange, alignment slack
 };
 
 struct Bars {
@@ -87,7 +75,7 @@ struct Bars {
   uint64_t s_full[2], p_full[2];
   uint64_t o_done;
   uint64_t fin;
-  uint64_t w_full, h_full, phi_ready, n_done, ol_ready, y_done;
+  uint64_t xbar[4][2];  // row-max exchange between the two warps of a quadrant
   uint32_t tmem;
   int abort;
 };
@@ -127,12 +115,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
     }
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->fin, 1);
-    mbar_init(&bars->w_full, 1);
-    mbar_init(&bars->h_full, 1);
-    mbar_init(&bars->phi_ready, kSoftThreads);
-    mbar_init(&bars->n_done, 1);
-    mbar_init(&bars->ol_ready, kSoftThreads);
-    mbar_init(&bars->y_done, 1);
+    for (int qq = 0; qq < 4; ++qq)
+      for (int b = 0; b < 2; ++b) mbar_init(&bars->xbar[qq][b], 64);
     bars->abort = 0;
     mbar_fence_init();
   }
@@ -163,10 +147,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         bulk_g2s(smem + C::kOffQ + kTile, p.q8t + (head_tiles + ib) * kTile, kTile, &bars->q_full);
       } else {
         bulk_g2s(smem + C::kOffQ, p.q8t + (head_tiles + 2 * iA) * kTile, 2 * kTile, &bars->q_full);
-      }
-      if (p.linear) {
-        mbar_expect_tx(&bars->w_full, kImg);
-        bulk_g2s(smem + C::kOffW, p.wimg, kImg, &bars->w_full);
       }
       int k_issued = 0, v_issued = 0;  // steps whose copies were issued
       for (int s = 0; s < nsteps && !*abort; ++s) {
@@ -213,19 +193,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         mbar_wait_drain(&bars->k_full[s % kStages], (s / kStages) & 1, p.wd);
       for (int s = max(0, v_issued - kStages); s < v_issued; ++s)
         mbar_wait_drain(&bars->v_full[s % kStages], (s / kStages) & 1, p.wd);
-      if (p.linear) {
-        // The K ring is free once every MMA of the main loop has completed.
-        if (v_issued == nsteps && mbar_wait(&bars->fin, 0, abort, p.wd)) {
-          const int nh = MODE == 0 ? 2 : 1;
-          mbar_expect_tx(&bars->h_full, nh * kImg);
-          for (int x = 0; x < nh; ++x) {
-            const int i = (x == 0 || !hasB) ? iA : iB;
-            bulk_g2s(smem + C::kOffK + x * kImg, p.himg + ((size_t)bh * p.nb + i) * kImg, kImg, &bars->h_full);
-          }
-          mbar_wait_drain(&bars->h_full, 0, p.wd);
-        }
-        mbar_wait_drain(&bars->w_full, 0, p.wd);
-      }
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ----------------------------
@@ -303,43 +270,14 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       // Every MMA issued must be complete before TMEM is released.
       mma_commit(&bars->fin);
       mbar_wait_drain(&bars->fin, 0, p.wd);
-      if (p.linear && ok) {
-        // num = phi(Q_i) H_i -> S0 columns;  y = O_l W^T -> S1 columns.
-        const int M = MODE == 0 ? 64 : 128;
-        const uint32_t id = idesc_bf16(M, 128);
-        ok = mbar_wait(&bars->h_full, 0, abort, p.wd) && mbar_wait(&bars->w_full, 0, abort, p.wd) &&
-             mbar_wait(&bars->phi_ready, 0, abort, p.wd);
-        if (ok) {
-          tc_fence_after();
-          for (int x = 0; x < (MODE == 0 ? (hasB ? 2 : 1) : 1); ++x) {
-            const uint8_t* a = smem + C::kOffV + x * (kImg / 2);
-            const uint8_t* b = smem + C::kOffK + x * kImg;
-            const uint32_t d = tmem + kColS0 + ((uint32_t)(x * 16) << 16);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-              mma_bf16(d, smem_desc(a + ks * 256, kImg_LBO, kImg_SBO), smem_desc(b + ks * 256, kImg_LBO, kImg_SBO),
-                       id, ks > 0);
-          }
-          mma_commit(&bars->n_done);
-          ok = mbar_wait(&bars->ol_ready, 0, abort, p.wd);
-        }
-        if (ok) {
-          tc_fence_after();
-          for (int x = 0; x < (MODE == 0 ? (hasB ? 2 : 1) : 1); ++x) {
-            const uint8_t* a = smem + C::kOffP + x * (kImg / 2);
-            const uint32_t d = tmem + kColS1 + ((uint32_t)(x * 16) << 16);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-              mma_bf16(d, smem_desc(a + ks * 256, kImg_LBO, kImg_SBO),
-                       smem_desc(smem + C::kOffW + ks * 256, kImg_LBO, kImg_SBO), id, ks > 0);
-          }
-          mma_commit(&bars->y_done);
-          mbar_wait_drain(&bars->y_done, 0, p.wd);
-        }
-      }
     }
   } else {
     // ------------------------------ softmax -------------------------------
+    // Two warps per TMEM lane quadrant: group g = 0 (warps 2-5) owns the
+    // first 64-key sub-tile of each step, group 1 (warps 6-9) the second.
+    // The two threads of a row trade their sub-tile maxima through a
+    // double-buffered shared slot and a 64-thread named barrier.
+    const int g = (warp - 2) >> 2;
     const int q = warp & 3;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int row, i, qtile;
@@ -360,93 +298,93 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
     const int n = i * block + row;
     const size_t tb = (size_t)bh * p.nq;
     const float c0 = active ? __ldg(p.sq + tb + qtile) * (kLog2e * 0.08838834764831845f) : 0.f;
-    float m_run = -INFINITY;
+    float* xch = reinterpret_cast<float*>(smem + C::kOffBar + sizeof(Bars));  // [2][2][128]
+    const int xrow = 32 * q + lane;
     uint8_t* prow_base = smem + C::kOffP + (MODE == 0 && lane >= 16 ? kTile : 0);
-    const int prow = row;
+    // Metadata of this thread's sub-tile, one step ahead of use.
+    auto tile_of = [&](int s) -> int {
+      if (MODE == 0) {
+        const int t = 2 * s + g;
+        return (active && t < p.kc) ? list_at(p, bh, i, t) : -1;
+      }
+      return 2 * list_at(p, bh, i, s) + g;
+    };
+    int kt_cur = tile_of(0);
+    float sk_cur = kt_cur >= 0 ? __ldg(p.sk + tb + kt_cur) : 0.f;
+    int kt_next = nsteps > 1 ? tile_of(1) : -1;
+    float m_run = -INFINITY;
     bool ok = true;
     for (int s = 0; s < nsteps; ++s) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[s & 1], (s >> 1) & 1, abort, p.wd));
       if (!ok) break;
       tc_fence_after();
       const int nsub = MODE == 0 ? min(2, p.kc - 2 * s) : 2;
-      uint32_t acc[128];
-      const uint32_t sbase = tmem + lane_base + ((s & 1) ? kColS1 : kColS0);
-      SAGESLA_TMEM_LD16(sbase + 0, acc + 0);
-      SAGESLA_TMEM_LD16(sbase + 16, acc + 16);
-      SAGESLA_TMEM_LD16(sbase + 32, acc + 32);
-      SAGESLA_TMEM_LD16(sbase + 48, acc + 48);
-      if (nsub == 2) {
-        SAGESLA_TMEM_LD16(sbase + 64, acc + 64);
-        SAGESLA_TMEM_LD16(sbase + 80, acc + 80);
-        SAGESLA_TMEM_LD16(sbase + 96, acc + 96);
-        SAGESLA_TMEM_LD16(sbase + 112, acc + 112);
+      const bool have = g < nsub && active && kt_cur >= 0;
+      const int nvalid = have ? max(0, min(64, p.N - kt_cur * 64)) : 0;
+      const float cu = c0 * sk_cur;
+      uint32_t acc[64];
+      if (g < nsub) {
+        const uint32_t sbase = tmem + lane_base + ((s & 1) ? kColS1 : kColS0) + 64 * g;
+        SAGESLA_TMEM_LD16(sbase + 0, acc + 0);
+        SAGESLA_TMEM_LD16(sbase + 16, acc + 16);
+        SAGESLA_TMEM_LD16(sbase + 32, acc + 32);
+        SAGESLA_TMEM_LD16(sbase + 48, acc + 48);
+        tmem_ld_wait();
       }
-      tmem_ld_wait();
-      // Per 64-key sub-tile: scale and number of valid keys.
-      float cu[2], mu_[2];
-      int nvalid[2], mx[2];
-      float m_new = m_run;
+      // Prefetch the key scale of the next step (its list entry arrived).
+      const float sk_next = kt_next >= 0 ? __ldg(p.sk + tb + kt_next) : 0.f;
+      const int kt_after = (s + 2 < nsteps) ? tile_of(s + 2) : -1;
+      int mx = INT_MIN;
+      if (nvalid == 64) {
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        cu[u] = 0.f;
-        nvalid[u] = 0;
-        if (u < nsub && active) {
-          int ktile;
-          if (MODE == 0) {
-            ktile = list_at(p, bh, i, 2 * s + u);
-          } else {
-            ktile = 2 * list_at(p, bh, i, s) + u;
-          }
-          cu[u] = c0 * __ldg(p.sk + tb + ktile);
-          nvalid[u] = max(0, min(64, p.N - ktile * 64));
-          int m_i = INT_MIN;
+        for (int c = 0; c < 64; ++c) mx = max(mx, (int)acc[c]);
+      } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < nvalid[u]) m_i = max(m_i, (int)acc[64 * u + c]);
-          mx[u] = m_i;
-          mu_[u] = __int2float_rn(m_i) * cu[u];
-          if (nvalid[u] > 0) m_new = fmaxf(m_new, mu_[u]);
-        }
+        for (int c = 0; c < 64; ++c)
+          if (c < nvalid) mx = max(mx, (int)acc[c]);
       }
+      const float mu = nvalid > 0 ? __int2float_rn(mx) * cu : -INFINITY;
+      xch[((s & 1) * 2 + g) * 128 + xrow] = mu;
+      mbar_arrive(&bars->xbar[q][s & 1]);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->xbar[q][s & 1], (s >> 1) & 1, abort, p.wd));
+      if (!ok) break;
+      const float mo = xch[((s & 1) * 2 + (g ^ 1)) * 128 + xrow];
+      const float m_new = fmaxf(m_run, fmaxf(mu, mo));
       const float alpha = (m_run == -INFINITY) ? 1.f : ex2(m_run - m_new);
-      // exponent of 448*P: (acc - max_u) * c_u + (m_u - m_new) + log2(448); the
-      // integer difference is exact, so values near the running max keep full
-      // precision however large the scores are.
-      float off[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) off[u] = nvalid[u] > 0 ? (mu_[u] - m_new) + kLog2_448 : 0.f;
-      // P~ codes, packed 4 per word, written into the row of the P buffer.
+      // exponent of 448*P: (acc - max_u) * c_u + (m_u - m_new) + log2(448);
+      // the integer difference is exact, so values near the running max keep
+      // full precision however large the scores are.
+      const float off = nvalid > 0 ? (mu - m_new) + kLog2_448 : 0.f;
       uint8_t* pbuf = prow_base + (s & 1) * C::kPBuf;
+      if (g < nsub) {
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        if (u < nsub) {
+        for (int ch = 0; ch < 4; ++ch) {  // 16-key chunks
+          uint32_t w[4];
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {  // 16-key chunks
-            uint32_t w[4];
+          for (int e = 0; e < 4; ++e) {
+            const int c = 16 * ch + 4 * e;
+            float x[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 16 * ch + 4 * e;
-              float x[4];
-#pragma unroll
-              for (int z = 0; z < 4; ++z)
-                x[z] = (c + z < nvalid[u])
-                           ? ex2(fmaf(__int2float_rn((int)acc[64 * u + c + z] - mx[u]), cu[u], off[u]))
-                           : 0.f;
-              w[e] = e4m3x2(x[0], x[1]) | (e4m3x2(x[2], x[3]) << 16);
-            }
-            *reinterpret_cast<uint4*>(pbuf + kmajor_off(prow, 64 * u + 16 * ch, kQK_LBO, kQK_SBO)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+            for (int z = 0; z < 4; ++z)
+              x[z] = (nvalid == 64 || c + z < nvalid)
+                         ? ex2(fmaf(__int2float_rn((int)acc[c + z] - mx), cu, off))
+                         : 0.f;
+            w[e] = e4m3x2(x[0], x[1]) | (e4m3x2(x[2], x[3]) << 16);
           }
+          *reinterpret_cast<uint4*>(pbuf + kmajor_off(row, 64 * g + 16 * ch, kQK_LBO, kQK_SBO)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      // Rescale O (and its row-sum columns) when the running max moved.
+      // Rescale O (and its row-sum columns) when the running max moved.  The
+      // two groups split the 144 columns: 0-79 and 80-143.
       if (s > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (s - 1) & 1, abort, p.wd));
         if (!ok) break;
         tc_fence_after();
         const uint32_t obase = tmem + lane_base + kColO;
+        const int cbeg = g == 0 ? 0 : 80, cend = g == 0 ? 80 : kNO;
 #pragma unroll 1
-        for (int c = 0; c < kNO; c += 16) {
+        for (int c = cbeg; c < cend; c += 16) {
           uint32_t o[16];
           SAGESLA_TMEM_LD16(obase + c, o);
           tmem_ld_wait();
@@ -457,74 +395,25 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         tmem_st_wait();
       }
       m_run = m_new;
+      kt_cur = kt_next;
+      sk_cur = sk_next;
+      kt_next = kt_after;
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->p_full[s & 1]);
     }
-    // Epilogue: O_s = O / l * s_v -> bf16.
+    // Epilogue: O_s = O / l * s_v (+ the linear branch already in out) -> bf16.
     // The last PV steps may still be in flight here, and o_done may be more
     // than one phase behind (a step that skips its rescale never waits on
     // it), which a parity wait cannot tell apart; `fin` has a single phase,
     // committed after the MMA thread's last instruction.
-    if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->fin, 0, abort, p.wd));
     const bool store = active && n < p.N;
-    const uint32_t ybase = tmem + lane_base + kColS1;
-    if (ok && nsteps > 0 && p.linear) {
-      // ---- linear branch: phi(q_r) . H_i / phi(q_r) . Z_i, then . W^T ----
-      const int xo = (MODE == 0 && lane >= 16) ? 1 : 0;  // operand half of this row
-      uint8_t* phiq = smem + C::kOffV + xo * (kImg / 2);
-      uint8_t* olr = smem + C::kOffP + xo * (kImg / 2);
-      const uint4* qrow = reinterpret_cast<const uint4*>(p.qraw + ((size_t)bh * p.N + (store ? n : 0)) * kD);
-      const float* zrow = p.zl + ((size_t)bh * p.nb + (active ? i : 0)) * kD;
-      float den = 0.f;
-#pragma unroll 4
-      for (int ch = 0; ch < 16; ++ch) {  // 8 channels per 16-byte chunk
-        uint4 qq = store ? __ldg(qrow + ch) : make_uint4(0, 0, 0, 0);
-        const uint32_t w4[4] = {qq.x, qq.y, qq.z, qq.w};
-        uint32_t pk[4];
+    __nv_bfloat16* orow = p.out + ((size_t)bh * p.N + (store ? n : 0)) * kD + 64 * g;
+    uint4 yrow[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = bf16_lo(w4[e]), b = bf16_hi(w4[e]);
-          const float fa = a > 0.f ? a + 1.f : __expf(a);
-          const float fb = b > 0.f ? b + 1.f : __expf(b);
-          den = fmaf(fa, __ldg(zrow + 8 * ch + 2 * e), den);
-          den = fmaf(fb, __ldg(zrow + 8 * ch + 2 * e + 1), den);
-          const __nv_bfloat162 h = __floats2bfloat162_rn(fa, fb);
-          pk[e] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        *reinterpret_cast<uint4*>(phiq + kmajor_off(row, ch * 16, kImg_LBO, kImg_SBO)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars->phi_ready);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->n_done, 0, abort, p.wd));
-      if (ok) {
-        tc_fence_after();
-        const float inv_den = (store && den > 0.f) ? 1.f / den : 0.f;
-#pragma unroll 1
-        for (int c = 0; c < kD; c += 16) {
-          uint32_t v16[16];
-          SAGESLA_TMEM_LD16(tmem + lane_base + kColS0 + c, v16);
-          tmem_ld_wait();
-          uint32_t pk[8];
-#pragma unroll
-          for (int z = 0; z < 8; ++z) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v16[2 * z]) * inv_den,
-                                                           __uint_as_float(v16[2 * z + 1]) * inv_den);
-            pk[z] = *reinterpret_cast<const uint32_t*>(&h);
-          }
-          *reinterpret_cast<uint4*>(olr + kmajor_off(row, c * 2, kImg_LBO, kImg_SBO)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(olr + kmajor_off(row, c * 2 + 16, kImg_LBO, kImg_SBO)) =
-              make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&bars->ol_ready);
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_done, 0, abort, p.wd));
-      }
-    }
+    for (int c = 0; c < 8; ++c)
+      yrow[c] = (p.add_out && store) ? *reinterpret_cast<const uint4*>(orow + 8 * c) : make_uint4(0, 0, 0, 0);
+    if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->fin, 0, abort, p.wd));
     if (ok && nsteps > 0) {
       tc_fence_after();
       const uint32_t obase = tmem + lane_base + kColO;
@@ -532,25 +421,19 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       SAGESLA_TMEM_LD16(obase + 128, lw);
       tmem_ld_wait();
       const float inv_l = 1.f / __uint_as_float(lw[0]);
-      __nv_bfloat16* orow = p.out + ((size_t)bh * p.N + (store ? n : 0)) * kD;
-#pragma unroll 1
-      for (int c = 0; c < kD; c += 16) {
-        uint32_t o[16], y[16];
-        SAGESLA_TMEM_LD16(obase + c, o);
-        if (p.linear) {
-          SAGESLA_TMEM_LD16(ybase + c, y);
-        }
+#pragma unroll
+      for (int c = 0; c < 64; c += 16) {
+        uint32_t o[16];
+        SAGESLA_TMEM_LD16(obase + 64 * g + c, o);
         tmem_ld_wait();
         if (store) {
           uint32_t pk[8];
 #pragma unroll
           for (int z = 0; z < 8; ++z) {
-            float a = __uint_as_float(o[2 * z]) * inv_l * __ldg(p.sv + (size_t)bh * kD + c + 2 * z);
-            float b = __uint_as_float(o[2 * z + 1]) * inv_l * __ldg(p.sv + (size_t)bh * kD + c + 2 * z + 1);
-            if (p.linear) {
-              a += __uint_as_float(y[2 * z]);
-              b += __uint_as_float(y[2 * z + 1]);
-            }
+            const uint32_t yw = z < 4 ? (&yrow[c / 8].x)[z] : (&yrow[c / 8 + 1].x)[z - 4];
+            const int ch = 64 * g + c + 2 * z;
+            const float a = __uint_as_float(o[2 * z]) * inv_l * __ldg(p.sv + (size_t)bh * kD + ch) + bf16_lo(yw);
+            const float b = __uint_as_float(o[2 * z + 1]) * inv_l * __ldg(p.sv + (size_t)bh * kD + ch + 1) + bf16_hi(yw);
             const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
             pk[z] = *reinterpret_cast<const uint32_t*>(&h);
           }
@@ -580,11 +463,7 @@ cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int
   p.nb = g.nb;
   p.nq = g.nq;
   p.kc = g.kc;
-  p.qraw = reinterpret_cast<const uint16_t*>(a.q);
-  p.himg = reinterpret_cast<const uint8_t*>(a.hlin);
-  p.zl = a.zlin;
-  p.wimg = reinterpret_cast<const uint8_t*>(a.wt);
-  p.linear = (a.hlin && a.zlin && a.wt && a.q) ? 1 : 0;
+  p.add_out = a.add_out;
   if (g.block == 64) {
     p.nsteps = (g.kc + 1) / 2;
     const int smem = Cfg<0>::kSmem;

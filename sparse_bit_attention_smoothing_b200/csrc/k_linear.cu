@@ -321,6 +321,189 @@ __global__ void __launch_bounds__(192, 1) linear_sum_kernel(const uint8_t* __res
   if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
+// ---------------------------------------------------------------- K4c ----
+// linear_apply: y_r = (phi(q_r) H_i / phi(q_r) Z_i) W^T for every row r of
+// query block i, written (bf16) into `out`; the flash kernel adds O_s to it.
+// Block 64: two query blocks per CTA whose M=64 accumulators share TMEM at
+// lane offsets 0 / 16 (all 128 threads hold a row); block 128: M = 128.
+// 128 threads; thread 0 issues the copies and MMAs.  TMEM: num (128 cols) and
+// y (128 cols).  Shared: H images, W image, phi(Q) (reused for O_l).
+template <int MODE>
+__global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __restrict__ q,
+                                                           const uint8_t* __restrict__ himg,
+                                                           const float* __restrict__ zl,
+                                                           const uint8_t* __restrict__ wimg, int N, int nb,
+                                                           __nv_bfloat16* __restrict__ out, int* wd) {
+  constexpr int kImg = 32768;
+  constexpr int nH = MODE == 0 ? 2 : 1;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sH = smem;                       // nH x 32 KB
+  uint8_t* sW = smem + nH * kImg;           // 32 KB
+  uint8_t* sA = sW + kImg;                  // 32 KB: phi(Q), then O_l
+  __shared__ uint64_t bar_in, bar_n, bar_y;
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int bh = blockIdx.y;
+  const int iA = MODE == 0 ? 2 * (int)blockIdx.x : (int)blockIdx.x;
+  const int iB = MODE == 0 ? iA + 1 : -1;
+  const bool hasB = MODE == 0 && iB < nb;
+  if (t == 0) {
+    mbar_init(&bar_in, 1);
+    mbar_init(&bar_n, 1);
+    mbar_init(&bar_y, 1);
+    abort_s = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) tmem_alloc(&tmem_s, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  if (t == 0) {
+    mbar_expect_tx(&bar_in, (nH + 1) * kImg);
+    for (int x = 0; x < nH; ++x) {
+      const int i = (x == 0 || !hasB) ? iA : iB;
+      bulk_g2s(sH + x * kImg, himg + ((size_t)bh * nb + i) * kImg, kImg, &bar_in);
+    }
+    bulk_g2s(sW, wimg, kImg, &bar_in);
+  }
+  // Row of this thread (same TMEM lane mapping as the flash kernel).
+  int row, i;
+  bool active;
+  if (MODE == 0) {
+    row = 16 * warp + (lane & 15);
+    i = lane >= 16 ? iB : iA;
+    active = lane >= 16 ? hasB : true;
+  } else {
+    row = 32 * warp + lane;
+    i = iA;
+    active = true;
+  }
+  const int blk = MODE == 0 ? 64 : 128;
+  const int n = i * blk + row;
+  const bool store = active && n < N;
+  const int xo = (MODE == 0 && lane >= 16) ? 1 : 0;
+  uint8_t* arow = sA + xo * (kImg / 2);
+  const uint4* qrow = reinterpret_cast<const uint4*>(q + ((size_t)bh * N + (store ? n : 0)) * kD);
+  const float4* zrow = reinterpret_cast<const float4*>(zl + ((size_t)bh * nb + (active ? i : 0)) * kD);
+  float den = 0.f;
+  uint4 qq[16];
+#pragma unroll
+  for (int ch = 0; ch < 16; ++ch) qq[ch] = store ? __ldg(qrow + ch) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int ch = 0; ch < 16; ++ch) {
+    const uint32_t w4[4] = {qq[ch].x, qq[ch].y, qq[ch].z, qq[ch].w};
+    const float4 z0 = __ldg(zrow + 2 * ch), z1 = __ldg(zrow + 2 * ch + 1);
+    const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+    uint32_t pk[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a = phi(bf16_lo(w4[e])), b = phi(bf16_hi(w4[e]));
+      den = fmaf(a, zz[2 * e], den);
+      den = fmaf(b, zz[2 * e + 1], den);
+      pk[e] = pack_bf16(a, b);
+    }
+    *reinterpret_cast<uint4*>(arow + kmajor_off(row, ch * 16, 128, 2048)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  const int M = MODE == 0 ? 64 : 128;
+  const uint32_t id = idesc_bf16(M, 128);
+  const int nx = MODE == 0 ? (hasB ? 2 : 1) : 1;
+  if (t == 0) {
+    if (mbar_wait(&bar_in, 0, &abort_s, wd)) {
+      tc_fence_after();
+      for (int x = 0; x < nx; ++x) {
+        const uint32_t d = tmem + ((uint32_t)(x * 16) << 16);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16(d, smem_desc(sA + x * (kImg / 2) + ks * 256, 128, 2048), smem_desc(sH + x * kImg + ks * 256, 128, 2048),
+                   id, ks > 0);
+      }
+    }
+    mma_commit(&bar_n);
+  }
+  bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_n, 0, &abort_s, wd));
+  tc_fence_after();
+  const uint32_t lb = (uint32_t)(32 * warp) << 16;
+  {
+    const float inv_den = (store && den > 0.f) ? 1.f / den : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < kD; c += 16) {
+      uint32_t v16[16];
+      SAGESLA_TMEM_LD16(tmem + lb + c, v16);
+      tmem_ld_wait();
+      uint32_t pk[8];
+#pragma unroll
+      for (int z2 = 0; z2 < 8; ++z2)
+        pk[z2] = pack_bf16(ok ? __uint_as_float(v16[2 * z2]) * inv_den : 0.f,
+                           ok ? __uint_as_float(v16[2 * z2 + 1]) * inv_den : 0.f);
+      *reinterpret_cast<uint4*>(arow + kmajor_off(row, c * 2, 128, 2048)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4*>(arow + kmajor_off(row, c * 2 + 16, 128, 2048)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (t == 0) {
+    tc_fence_after();
+    if (ok) {
+      for (int x = 0; x < nx; ++x) {
+        const uint32_t d = tmem + 128 + ((uint32_t)(x * 16) << 16);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16(d, smem_desc(sA + x * (kImg / 2) + ks * 256, 128, 2048), smem_desc(sW + ks * 256, 128, 2048), id,
+                   ks > 0);
+      }
+    }
+    mma_commit(&bar_y);
+  }
+  ok = __all_sync(0xffffffffu, mbar_wait(&bar_y, 0, &abort_s, wd)) && ok;
+  tc_fence_after();
+  __nv_bfloat16* orow = out + ((size_t)bh * N + (store ? n : 0)) * kD;
+#pragma unroll 1
+  for (int c = 0; c < kD; c += 16) {
+    uint32_t v16[16];
+    SAGESLA_TMEM_LD16(tmem + lb + 128 + c, v16);
+    tmem_ld_wait();
+    if (store) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int z2 = 0; z2 < 8; ++z2)
+        pk[z2] = pack_bf16(ok ? __uint_as_float(v16[2 * z2]) : 0.f, ok ? __uint_as_float(v16[2 * z2 + 1]) : 0.f);
+      *reinterpret_cast<uint4*>(orow + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4*>(orow + c + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+  }
+  // The inputs' bulk copies must have landed before the CTA exits.
+  if (t == 0) mbar_wait_drain(&bar_in, 0, wd);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+int linear_apply_smem(int block) { return (block == 64 ? 4 : 3) * 32768 + 1024; }
+
+cudaError_t launch_linear_apply(const void* q, const uint16_t* himg, const float* zl, const uint16_t* wimg,
+                                const Geom& g, void* out, int* wd, cudaStream_t st) {
+  const int smem = linear_apply_smem(g.block);
+  cudaError_t e;
+  if (g.block == 64) {
+    e = cudaFuncSetAttribute(linear_apply_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    linear_apply_kernel<0><<<dim3((g.nb + 1) / 2, g.BH), 128, smem, st>>>(
+        (const uint16_t*)q, (const uint8_t*)himg, zl, (const uint8_t*)wimg, g.N, g.nb, (__nv_bfloat16*)out, wd);
+  } else {
+    e = cudaFuncSetAttribute(linear_apply_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    linear_apply_kernel<1><<<dim3(g.nb, g.BH), 128, smem, st>>>(
+        (const uint16_t*)q, (const uint8_t*)himg, zl, (const uint8_t*)wimg, g.N, g.nb, (__nv_bfloat16*)out, wd);
+  }
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------- W image ---
 // proj_w [c_out][c_in] row-major -> K-major B operand image [N=c_out][K=c_in].
 __global__ void w_tile_kernel(const uint16_t* __restrict__ w, uint16_t* __restrict__ wt) {

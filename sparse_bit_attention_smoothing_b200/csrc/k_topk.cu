@@ -36,13 +36,20 @@ __device__ __forceinline__ float pooled(const float* __restrict__ sums, int blk,
   return __fdiv_rn(a, (float)cnt);
 }
 
+// Pooled means of every attention block, once: grid (nb, BH), 128 threads.
+__global__ void pool_means_kernel(const float* __restrict__ qsum, const float* __restrict__ ksum, int N, int block,
+                                  int nb, int nq, float* __restrict__ qbar, float* __restrict__ kbar) {
+  const int i = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+  qbar[((size_t)bh * nb + i) * kD + c] = pooled(qsum + (size_t)bh * nq * kD, i, block, N, c);
+  kbar[((size_t)bh * nb + i) * kD + c] = pooled(ksum + (size_t)bh * nq * kD, i, block, N, c);
+}
+
 // Linear-branch outputs (when zin != NULL): selbits [nb][nbw] words with
 // bit j set when key block j is selected; zout [nb][128] the fp32 sums
 // Z_i = sum_{j not in S_i} z_j, formed as (sum over all j) - (sum over S_i).
-__global__ void __launch_bounds__(256) pool_topk_kernel(const float* __restrict__ qsum, const float* __restrict__ ksum,
-                                                        int N, int block, int nb, int nq, int kc,
-                                                        int32_t* __restrict__ idx, float* __restrict__ qbar_out,
-                                                        float* __restrict__ kbar_out, const float* __restrict__ zin,
+__global__ void __launch_bounds__(256) pool_topk_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
+                                                        int nb, int kc, int32_t* __restrict__ idx,
+                                                        const float* __restrict__ zin,
                                                         uint32_t* __restrict__ selbits, int nbw,
                                                         float* __restrict__ zout) {
   extern __shared__ __align__(16) float sm[];
@@ -51,31 +58,25 @@ __global__ void __launch_bounds__(256) pool_topk_kernel(const float* __restrict_
   float* sc = kb + kKC * kPad;               // [kTQ][nb]
   const int bh = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int i0 = blockIdx.x * kTQ;
-  const float* qs = qsum + (size_t)bh * nq * kD;
-  const float* ks = ksum + (size_t)bh * nq * kD;
+  const float* qh = qbar + (size_t)bh * nb * kD;
+  const float* kh = kbar + (size_t)bh * nb * kD;
   const float rs = 1.0f / sqrtf((float)kD);
 
   for (int e = t; e < kTQ * kD; e += 256) {
-    const int r = e / kD, c = e % kD;
-    const int i = i0 + r;
-    const float val = i < nb ? pooled(qs, i, block, N, c) : 0.f;
-    qb[e] = val;
-    if (qbar_out && i < nb) qbar_out[((size_t)bh * nb + i) * kD + c] = val;
+    const int r = e / kD;
+    qb[e] = i0 + r < nb ? qh[(size_t)i0 * kD + e] : 0.f;
   }
   // Phase 1: scores.  Thread -> key block jj = t % 64 of the chunk, query
   // rows 2*(t/64) and 2*(t/64)+1.
   const int jj = t & 63, qg = t >> 6;
   for (int j0 = 0; j0 < nb; j0 += kKC) {
     __syncthreads();
-    for (int e = t; e < kKC * kD; e += 256) {
-      const int r = e / kD, c = e % kD;
+    for (int e = t; e < kKC * kD / 4; e += 256) {
+      const int r = e / (kD / 4), c4 = e % (kD / 4);
       const int j = j0 + r;
-      float val = 0.f;
-      if (j < nb) {
-        val = pooled(ks, j, block, N, c);
-        if (kbar_out && blockIdx.x == 0) kbar_out[((size_t)bh * nb + j) * kD + c] = val;
-      }
-      kb[r * kPad + c] = val;
+      const float4 val = j < nb ? *reinterpret_cast<const float4*>(kh + (size_t)j * kD + 4 * c4)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(kb + r * kPad + 4 * c4) = val;
     }
     __syncthreads();
     const int j = j0 + jj;
@@ -165,11 +166,13 @@ size_t pool_topk_smem(int nb) { return sizeof(float) * ((size_t)kTQ * kD + (size
 
 cudaError_t launch_pool_topk(const float* qsum, const float* ksum, const Geom& g, int32_t* idx, float* qbar,
                              float* kbar, const float* zin, uint32_t* selbits, float* zout, cudaStream_t st) {
-  const size_t smem = pool_topk_smem(g.nb);
-  cudaError_t e = cudaFuncSetAttribute(pool_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  pool_means_kernel<<<dim3(g.nb, g.BH), kD, 0, st>>>(qsum, ksum, g.N, g.block, g.nb, g.nq, qbar, kbar);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  pool_topk_kernel<<<dim3((g.nb + kTQ - 1) / kTQ, g.BH), 256, smem, st>>>(qsum, ksum, g.N, g.block, g.nb, g.nq, g.kc,
-                                                                           idx, qbar, kbar, zin, selbits,
+  const size_t smem = pool_topk_smem(g.nb);
+  e = cudaFuncSetAttribute(pool_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  pool_topk_kernel<<<dim3((g.nb + kTQ - 1) / kTQ, g.BH), 256, smem, st>>>(qbar, kbar, g.nb, g.kc, idx, zin, selbits,
                                                                            2 * ((g.nb + 63) / 64), zout);
   return cudaGetLastError();
 }

@@ -31,7 +31,8 @@ cudaError_t launch_quant(const void* q, const void* k, const void* v, const floa
 // Untile the quantised tiles back to row-major codes (parity entry only).
 cudaError_t launch_untile(const uint8_t* q8t, const uint8_t* k8t, const uint8_t* v8t, const Geom& g, int8_t* q8,
                           int8_t* k8, uint8_t* v8, cudaStream_t st);
-// K3: pooled block scores and the per-query-block top-k list (ascending).
+// K3: pooled block means (written to qbar/kbar, [BH][nb][128], required),
+// then block scores and the per-query-block top-k list (ascending).
 // With zin != NULL also writes the selection bitmask (2*ceil(nb/64) words
 // per query block) and Z_i = sum of z_j over the unselected key blocks.
 cudaError_t launch_pool_topk(const float* qsum, const float* ksum, const Geom& g, int32_t* idx, float* qbar,
@@ -42,6 +43,9 @@ cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_
 // K4b: H_i = sum over unselected j of h_j, as bf16 operand images [nb][128*128].
 cudaError_t launch_linear_sum(const uint8_t* hs, const uint32_t* selbits, const Geom& g, uint16_t* hout, int* wd,
                               cudaStream_t st);
+// K4c: y = (phi(Q_i) H_i / phi(Q_i) Z_i) W^T per row, written (bf16) to out.
+cudaError_t launch_linear_apply(const void* q, const uint16_t* himg, const float* zl, const uint16_t* wimg,
+                                const Geom& g, void* out, int* wd, cudaStream_t st);
 // proj_w [d][d] -> the bf16 B-operand image read by the flash epilogue.
 cudaError_t launch_w_tile(const void* w, uint16_t* wt, cudaStream_t st);
 // K5: block-sparse INT8/FP8 flash attention over the index lists.
@@ -54,11 +58,7 @@ struct FlashArgs {
   const float* sv;
   const int32_t* idx;  // [BH][nb][kc]; NULL = dense (every block, ascending)
   void* out;           // bf16 [BH][N][128]
-  // linear branch (all NULL when off)
-  const void* q;         // bf16 input Q (for phi(Q))
-  const uint16_t* hlin;  // bf16 H_i images [BH][nb][128*128] (B operand layout)
-  const float* zlin;     // fp32 Z_i [BH][nb][128]
-  const uint16_t* wt;    // bf16 proj_w image (B operand layout), 32 KB
+  int add_out;          // 1: out already holds the linear branch y (bf16); add O_s to it
 };
 cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int* wd);
 
