@@ -92,6 +92,23 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def flash_traffic(w):
+    """DRAM bytes of one flash launch from the committed ncu capture, scaled by
+    elements; None when the kernel source changed since the capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "flash_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        t = json.load(f)
+    with open(os.path.join(ROOT, t["source"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != t["source_sha256"]:
+            return None
+    if w.block != 64:
+        return None
+    return t["dram_bytes"] / t["elements"] * (w.B * w.H * w.N * w.d)
+
+
 def flops(w) -> dict:
     """Dense-equivalent and computed-block FLOPs of one call, and algorithmic HBM bytes."""
     from sparse_bit_attention_smoothing_b200 import topk_count
@@ -270,7 +287,7 @@ def main():
             "gpu_launches": launches, "device_status": status,
             "kernels_ms": {kname: round(t / max(1, n), 4) for kname, (t, n) in prof.items()},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak8, "unit": "TFLOP/s",
-                         "frac": (achieved / peak8) if achieved else None, "traffic": None,
+                         "frac": (achieved / peak8) if achieved else None, "traffic": flash_traffic(w),
                          "kernel": "flash", "peak_note": f"8-bit = 2 x {pk['src']} bf16 burst {pk['bf16']}",
                          "path_t_roof_ms": t_roof * 1e3, "path_frac": t_roof * 1e3 / ms},
             "clocks": clocks,
