@@ -119,6 +119,29 @@ int sagesla_get_mask(const void* q, const void* k, int B, int H, int N, int d, i
                      float topk, int32_t* idx_out, float* qbar, float* kbar, int* k_out,
                      sagesla_stream_t stream);
 
+/*
+ * sagesla_smooth_stats_noalloc: the smoothing statistics of the path -- the
+ * per-channel mean of K (mu, as in sagesla_get_quant) and the per-channel FP8
+ * scale of V (sv) -- computed WITHOUT allocating any device memory.  The
+ * pages have no counterpart: this is an interface for callers that cannot
+ * allocate once running (a process that fixes its device-memory budget at
+ * start-up, or code running where an allocation would stall or fail).  The
+ * regular entry points allocate a workspace on first use; this one uses a
+ * fixed 4 MiB scratch array that is part of the library image on every GPU
+ * that loads the library, until the process exits.
+ *   k, v     bf16 [B][H][N][d] device, 16-byte aligned.
+ *   mu, sv   float [B][H][d] device (written).
+ * The first call on a device looks up the scratch array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls share the scratch: calls that
+ * overlap on the GPU (other streams or host threads on the same device) race
+ * and must be serialised by the caller.  Sizes whose partial sums do not fit
+ * the scratch (B*H above about 2000) return SAGESLA_ERR_INVALID without
+ * launching; other argument errors as for sagesla_attn.
+ */
+int sagesla_smooth_stats_noalloc(const void* k, const void* v, int B, int H, int N, int d, float* mu,
+                                 float* sv, sagesla_stream_t stream);
+
 /* Number of key blocks kept per query block: clamp(ceil(topk*nb*(1-1e-6)), 1, nb). */
 int sagesla_topk_count(int nb, float topk);
 
