@@ -30,7 +30,7 @@ __host__ __device__ __forceinline__ uint32_t kmajor_off(uint32_t r, uint32_t c, 
 // Watchdog: every device-side wait is bounded; on expiry the kernel records
 // the failure in a device word of the workspace (`wd`) and returns.  The
 // host reads and clears it in sagesla_sync_status().
-constexpr long kSpinLimit = 1L << 24;  // try_wait iterations (each may suspend briefly)
+constexpr long kSpinLimit = 1L << 24;  // try_wait probes (each may suspend briefly)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -60,10 +60,21 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of a phase (cheap when it has already completed).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait.  Returns false if it gave up: then it raises `abort` (a
 // CTA-shared flag, so that every role of the CTA stops) and the global
 // watchdog word `wd`.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* wd) {
+  if (mbar_test(bar, parity)) return true;
   for (long i = 0; i < kSpinLimit; ++i) {
     if (mbar_try(bar, parity)) return true;
     if ((i & 255) == 255 && *abort) return false;
@@ -76,6 +87,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // Bounded wait that ignores the abort flag: used to drain work that always
 // completes on its own (issued copies, issued MMAs) before the CTA exits.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int* wd) {
+  if (mbar_test(bar, parity)) return true;
   for (long i = 0; i < kSpinLimit; ++i)
     if (mbar_try(bar, parity)) return true;
   atomicExch(wd, 1);
@@ -120,6 +132,10 @@ __device__ __forceinline__ uint64_t smem_desc(const void* p, uint32_t lbo, uint3
   d |= (uint64_t)1 << 46;
   return d;
 }
+// Descriptor of smem offset `off` from a base descriptor (the start-address
+// field holds address >> 4 in 14 bits; shared memory is < 256 KB, so adding
+// off >> 4 to the low word never carries out of the field).
+__device__ __forceinline__ uint64_t desc_at(uint64_t base, uint32_t off) { return base + (uint64_t)(off >> 4); }
 // Instruction descriptors.  kind::i8 s8 x s8 -> s32; kind::f8f6f4 e4m3 x e4m3
 // -> f32; kind::f16 bf16 x bf16 -> f32.  Both operands K-major unless b_mn.
 __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {

@@ -9,18 +9,32 @@
 // smoothing on integer tensor cores) and 支柱二 (only the selected blocks are
 // computed exactly); 量子位 news 技术解密 1 (SageAttention2++).
 //
-// Layout on the SM (192 threads, 1 CTA/SM):
-//   warp 0  producer: bulk copies of Q^, K^ and V^T tiles (pre-tiled in HBM
-//           by the quantiser, so one cp.async.bulk moves a whole 8 KB tile);
-//   warp 1  MMA issuer (one thread) + TMEM owner;
-//   warps 2-5  softmax / rescale / epilogue, one query row per thread.
+// Roles on the SM (15 warps, 1 CTA/SM):
+//   warp 0     producer: bulk copies of Q^, K^ and V^T tiles (pre-tiled in
+//              HBM by the quantiser, so one cp.async.bulk moves a whole tile);
+//   warp 1     QK^T issuer (one thread) and TMEM owner;
+//   warp 2     PV issuer (one thread) -- two issuers keep the tensor pipe fed
+//              while either of them waits;
+//   warps 3-10 softmax: two warps per TMEM lane quadrant, each owning one
+//              64-key sub-tile of the 128-key step of every row;
+//   warps 11-14 correction: one warp per quadrant; rescales O by
+//              exp(m_old - m_new) between PV steps, off the softmax path, and
+//              runs the epilogue.
 // Mode 64 (block 64): a CTA owns two query blocks A and B.  Their M=64
 //   accumulators share TMEM columns at lane offsets 0 and 16, so all 128
-//   softmax threads hold a row.  Each step takes two key blocks per query
-//   block (S tile N = 128), PV is M=64, N=144 (128 V channels + 16 rows of
-//   ones whose product is the row sum of P~).
+//   lanes hold a row.  Each step takes two key blocks per query block (S tile
+//   N = 128); PV is M=64, N=144 (128 V channels + 16 rows of ones whose
+//   product is the row sum of P~).
 // Mode 128 (block 128): one query block of 128 rows per CTA, M = 128.
 // TMEM: S double buffer (2 x 128 cols) + O (144 cols) of 512 allocated.
+//
+// Step hand-offs (s = step): S(s) -> s_full -> softmax(s) -> p_full(s) ->
+// correction(s) [waits PV(s-1)] -> s_free(s), o_ready(s) -> PV(s) -> o_done.
+// QK^T for step s+2 waits s_free(s) (its S buffer and alpha slot are then
+// free); P is triple-buffered, so the buffer softmax(s+3) writes was read by
+// PV(s), which correction(s+1) saw complete before s_free(s+1) released
+// QK^T(s+3).  Every parity wait below is at most one phase behind its
+// barrier (o_ready has the PV issuer as its only waiter).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -29,8 +43,11 @@ namespace sagesla {
 namespace {
 
 constexpr int kStages = 2;
-constexpr int kSoftThreads = 256;  // two warps per TMEM lane quadrant
-constexpr int kThreads = 64 + kSoftThreads;
+constexpr int kPBufs = 3;
+constexpr int kSoftThreads = 256;
+constexpr int kCorrThreads = 128;
+constexpr int kWarpSoft0 = 3, kWarpCorr0 = 11;
+constexpr int kThreads = 32 * 3 + kSoftThreads + kCorrThreads;  // 480
 constexpr int kVSlot = kTile + 1024;  // 8 KB V^T tile + 16 rows of ones (1 KB)
 constexpr uint32_t kOnesE4M3 = 0x38383838u;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -64,8 +81,11 @@ struct Cfg {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKStage;
   static constexpr int kOffP = kOffV + kStages * kVStage;
-  static constexpr int kOffBar = kOffP + 2 * kPBuf;
-  static constexpr int kSmem = kOffBar + 256 + 2048 + 1024;  // barriers, max exchange, alignment slack
+  static constexpr int kOffBar = kOffP + kPBufs * kPBuf;
+  static constexpr int kBarBytes = 512;
+  static constexpr int kOffX = kOffBar + kBarBytes;      // row-max exchange [2][2][128] f32
+  static constexpr int kOffA = kOffX + 2 * 2 * 128 * 4;  // alpha [2][128] f32
+  static constexpr int kSmem = kOffA + 2 * 128 * 4 + 1024;  // + alignment slack
 };
 
 struct Bars {
@@ -73,12 +93,14 @@ struct Bars {
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], p_full[2];
-  uint64_t o_done;
+  uint64_t o_ready, o_done;
+  uint64_t s_free[2];
   uint64_t fin;
-  uint64_t xbar[4][2];  // row-max exchange between the two warps of a quadrant
+  uint64_t xbar[4][2];  // row-max exchange between the two softmax warps of a quadrant
   uint32_t tmem;
   int abort;
 };
+static_assert(sizeof(Bars) <= 512, "barrier block");
 
 // key block (mask block index) of list entry t for query block i
 __device__ __forceinline__ int list_at(const Params& p, int bh, int i, int t) {
@@ -93,6 +115,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
+  float* xch = reinterpret_cast<float*>(smem + C::kOffX);
+  float* alpha_s = reinterpret_cast<float*>(smem + C::kOffA);
   volatile int* abort = &bars->abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y;
@@ -100,6 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
   const int iA = MODE == 0 ? 2 * (int)blockIdx.x : (int)blockIdx.x;
   const int iB = MODE == 0 ? 2 * (int)blockIdx.x + 1 : -1;
   const bool hasB = MODE == 0 && iB < p.nb;
+  const int nsteps = p.nsteps;
 
   if (tid == 0) {
     mbar_init(&bars->q_full, 1);
@@ -113,8 +138,11 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       mbar_init(&bars->s_full[b], 1);
       mbar_init(&bars->p_full[b], kSoftThreads);
     }
+    mbar_init(&bars->o_ready, kCorrThreads);
+    mbar_init(&bars->s_free[0], kCorrThreads);
+    mbar_init(&bars->s_free[1], kCorrThreads);
     mbar_init(&bars->o_done, 1);
-    mbar_init(&bars->fin, 1);
+    mbar_init(&bars->fin, 2);
     for (int qq = 0; qq < 4; ++qq)
       for (int b = 0; b < 2; ++b) mbar_init(&bars->xbar[qq][b], 64);
     bars->abort = 0;
@@ -123,10 +151,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
   // Rows of ones under every V slot (PV's extra 16 output columns = row sum).
   for (int e = tid; e < kStages * (C::kVStage / kVSlot) * 64; e += kThreads) {
     const int slot = e / 64, w = e % 64;
-    reinterpret_cast<uint32_t*>(smem + C::kOffV + slot * kVSlot + kTile)[w * 4 + 0] = kOnesE4M3;
-    reinterpret_cast<uint32_t*>(smem + C::kOffV + slot * kVSlot + kTile)[w * 4 + 1] = kOnesE4M3;
-    reinterpret_cast<uint32_t*>(smem + C::kOffV + slot * kVSlot + kTile)[w * 4 + 2] = kOnesE4M3;
-    reinterpret_cast<uint32_t*>(smem + C::kOffV + slot * kVSlot + kTile)[w * 4 + 3] = kOnesE4M3;
+    *reinterpret_cast<uint4*>(smem + C::kOffV + slot * kVSlot + kTile + w * 16) =
+        make_uint4(kOnesE4M3, kOnesE4M3, kOnesE4M3, kOnesE4M3);
   }
   fence_proxy_async_smem();
   if (warp == 1) tmem_alloc(&bars->tmem, kTmemCols);
@@ -134,7 +160,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
-  const int nsteps = p.nsteps;
 
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
@@ -151,32 +176,34 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       int k_issued = 0, v_issued = 0;  // steps whose copies were issued
       for (int s = 0; s < nsteps && !*abort; ++s) {
         const int st = s % kStages;
+        int jj[2][2] = {{-1, -1}, {-1, -1}};
+        if (MODE == 0) {
+          const int nsub = min(2, p.kc - 2 * s);
+          for (int x = 0; x < 2; ++x) {
+            const int i = (x == 0 || !hasB) ? iA : iB;
+            for (int u = 0; u < nsub; ++u) jj[x][u] = list_at(p, bh, i, 2 * s + u);
+          }
+        } else {
+          jj[0][0] = list_at(p, bh, iA, s);
+        }
         if (s >= kStages && !mbar_wait(&bars->k_empty[st], ((s / kStages) - 1) & 1, abort, p.wd)) break;
         uint8_t* kd = smem + C::kOffK + st * C::kKStage;
         uint8_t* vd = smem + C::kOffV + st * C::kVStage;
         if (MODE == 0) {
           const int nsub = min(2, p.kc - 2 * s);
           mbar_expect_tx(&bars->k_full[st], 2 * nsub * kTile);
-          for (int x = 0; x < 2; ++x) {
-            const int i = (x == 0 || !hasB) ? iA : iB;
-            for (int u = 0; u < nsub; ++u) {
-              const int j = list_at(p, bh, i, 2 * s + u);
-              bulk_g2s(kd + (2 * x + u) * kTile, p.k8t + (head_tiles + j) * kTile, kTile, &bars->k_full[st]);
-            }
-          }
+          for (int x = 0; x < 2; ++x)
+            for (int u = 0; u < nsub; ++u)
+              bulk_g2s(kd + (2 * x + u) * kTile, p.k8t + (head_tiles + jj[x][u]) * kTile, kTile, &bars->k_full[st]);
           k_issued = s + 1;
           if (s >= kStages && !mbar_wait(&bars->v_empty[st], ((s / kStages) - 1) & 1, abort, p.wd)) break;
           mbar_expect_tx(&bars->v_full[st], 2 * nsub * kTile);
-          for (int x = 0; x < 2; ++x) {
-            const int i = (x == 0 || !hasB) ? iA : iB;
-            for (int u = 0; u < nsub; ++u) {
-              const int j = list_at(p, bh, i, 2 * s + u);
-              bulk_g2s(vd + (2 * x + u) * kVSlot, p.v8t + (head_tiles + j) * kTile, kTile, &bars->v_full[st]);
-            }
-          }
+          for (int x = 0; x < 2; ++x)
+            for (int u = 0; u < nsub; ++u)
+              bulk_g2s(vd + (2 * x + u) * kVSlot, p.v8t + (head_tiles + jj[x][u]) * kTile, kTile, &bars->v_full[st]);
           v_issued = s + 1;
         } else {
-          const int j = list_at(p, bh, iA, s);
+          const int j = jj[0][0];
           mbar_expect_tx(&bars->k_full[st], 2 * kTile);
           bulk_g2s(kd, p.k8t + (head_tiles + 2 * j) * kTile, 2 * kTile, &bars->k_full[st]);
           k_issued = s + 1;
@@ -195,89 +222,86 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         mbar_wait_drain(&bars->v_full[s % kStages], (s / kStages) & 1, p.wd);
     }
   } else if (warp == 1) {
-    // ------------------------------ MMA issuer ----------------------------
+    // ------------------------------ QK^T issuer ---------------------------
     if (lane == 0) {
-      const uint32_t id_s = MODE == 0 ? 0u : idesc_i8(128, 128);
-      const uint32_t id_pv = idesc_e4m3(MODE == 0 ? 64 : 128, kNO);
+      const uint64_t dqk = smem_desc(smem, kQK_LBO, kQK_SBO);
       bool ok = mbar_wait(&bars->q_full, 0, abort, p.wd);
-      auto issue_s = [&](int s) {
+      for (int s = 0; ok && s < nsteps; ++s) {
         const int st = s % kStages;
+        if (!(ok = mbar_wait(&bars->k_full[st], (s / kStages) & 1, abort, p.wd))) break;
+        // S buffer s&1 and alpha slot s&1 are free once step s-2 is corrected.
+        if (s >= 2) {
+          if (!(ok = mbar_wait(&bars->s_free[s & 1], ((s - 2) >> 1) & 1, abort, p.wd))) break;
+          tc_fence_after();
+        }
         const uint32_t dS = tmem + ((s & 1) ? kColS1 : kColS0);
-        const uint8_t* kd = smem + C::kOffK + st * C::kKStage;
+        const uint32_t koff = C::kOffK + st * C::kKStage;
         if (MODE == 0) {
-          const int nsub = min(2, p.kc - 2 * s);
-          const uint32_t id = idesc_i8(64, 64 * nsub);
-          for (int x = 0; x < (hasB ? 2 : 1); ++x) {
-            const uint8_t* qa = smem + C::kOffQ + x * kTile;
-            const uint8_t* kb = kd + 2 * x * kTile;
+          const uint32_t id = p.kc - 2 * s >= 2 ? idesc_i8(64, 128) : idesc_i8(64, 64);
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            if (x == 1 && !hasB) break;
             const uint32_t d = dS + ((uint32_t)(x * 16) << 16);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_i8(d, smem_desc(qa + kk * 256, kQK_LBO, kQK_SBO), smem_desc(kb + kk * 256, kQK_LBO, kQK_SBO), id,
+              mma_i8(d, desc_at(dqk, C::kOffQ + x * kTile + kk * 256), desc_at(dqk, koff + 2 * x * kTile + kk * 256), id,
                      kk > 0);
           }
         } else {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_i8(dS, smem_desc(smem + C::kOffQ + kk * 256, kQK_LBO, kQK_SBO),
-                   smem_desc(kd + kk * 256, kQK_LBO, kQK_SBO), id_s, kk > 0);
+            mma_i8(dS, desc_at(dqk, C::kOffQ + kk * 256), desc_at(dqk, koff + kk * 256), idesc_i8(128, 128), kk > 0);
         }
         mma_commit(&bars->s_full[s & 1]);
         mma_commit(&bars->k_empty[st]);
-      };
-      if (ok && nsteps > 0) {
-        ok = mbar_wait(&bars->k_full[0], 0, abort, p.wd);
-        if (ok) {
-          tc_fence_after();
-          issue_s(0);
-        }
       }
+      mma_commit(&bars->fin);
+    }
+  } else if (warp == 2) {
+    // ------------------------------ PV issuer -----------------------------
+    if (lane == 0) {
+      const uint64_t dqk = smem_desc(smem, kQK_LBO, kQK_SBO);
+      const uint64_t dv = smem_desc(smem, kV_LBO, kV_SBO);
+      const uint32_t id_pv = idesc_e4m3(MODE == 0 ? 64 : 128, kNO);
+      bool ok = true;
       for (int s = 0; ok && s < nsteps; ++s) {
-        if (s + 1 < nsteps) {
-          const int st1 = (s + 1) % kStages;
-          if (!(ok = mbar_wait(&bars->k_full[st1], ((s + 1) / kStages) & 1, abort, p.wd))) break;
-          tc_fence_after();
-          issue_s(s + 1);
-        }
         const int st = s % kStages;
-        if (!(ok = mbar_wait(&bars->p_full[s & 1], (s >> 1) & 1, abort, p.wd))) break;
         if (!(ok = mbar_wait(&bars->v_full[st], (s / kStages) & 1, abort, p.wd))) break;
+        if (!(ok = mbar_wait(&bars->o_ready, s & 1, abort, p.wd))) break;
         tc_fence_after();
-        const uint8_t* vd = smem + C::kOffV + st * C::kVStage;
-        const uint8_t* pb = smem + C::kOffP + (s & 1) * C::kPBuf;
+        const uint32_t voff = C::kOffV + st * C::kVStage;
+        const uint32_t poff = C::kOffP + (s % kPBufs) * C::kPBuf;
         if (MODE == 0) {
-          const int nsub = min(2, p.kc - 2 * s);
-          for (int x = 0; x < (hasB ? 2 : 1); ++x) {
+          const int nk = p.kc - 2 * s >= 2 ? 4 : 2;
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            if (x == 1 && !hasB) break;
             const uint32_t d = tmem + kColO + ((uint32_t)(x * 16) << 16);
-            for (int kk = 0; kk < 2 * nsub; ++kk) {
-              const uint8_t* a = pb + x * kTile + kk * 256;
-              const uint8_t* b = vd + (2 * x + (kk >> 1)) * kVSlot + (kk & 1) * 256;
-              mma_e4m3(d, smem_desc(a, kQK_LBO, kQK_SBO), smem_desc(b, kV_LBO, kV_SBO), id_pv, (s > 0 || kk > 0));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (kk >= nk) break;
+              mma_e4m3(d, desc_at(dqk, poff + x * kTile + kk * 256),
+                       desc_at(dv, voff + (2 * x + (kk >> 1)) * kVSlot + (kk & 1) * 256), id_pv, (s > 0 || kk > 0));
             }
           }
         } else {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint8_t* a = pb + kk * 256;
-            const uint8_t* b = vd + (kk >> 1) * kVSlot + (kk & 1) * 256;
-            mma_e4m3(tmem + kColO, smem_desc(a, kQK_LBO, kQK_SBO), smem_desc(b, kV_LBO, kV_SBO), id_pv,
-                     (s > 0 || kk > 0));
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_e4m3(tmem + kColO, desc_at(dqk, poff + kk * 256), desc_at(dv, voff + (kk >> 1) * kVSlot + (kk & 1) * 256),
+                     id_pv, (s > 0 || kk > 0));
         }
         mma_commit(&bars->o_done);
         mma_commit(&bars->v_empty[st]);
       }
-      // Every MMA issued must be complete before TMEM is released.
       mma_commit(&bars->fin);
-      mbar_wait_drain(&bars->fin, 0, p.wd);
     }
-  } else {
+  } else if (warp < kWarpCorr0) {
     // ------------------------------ softmax -------------------------------
-    // Two warps per TMEM lane quadrant: group g = 0 (warps 2-5) owns the
-    // first 64-key sub-tile of each step, group 1 (warps 6-9) the second.
-    // The two threads of a row trade their sub-tile maxima through a
-    // double-buffered shared slot and a 64-thread named barrier.
-    const int g = (warp - 2) >> 2;
+    // Two warps per TMEM lane quadrant: group g = 0 owns the first 64-key
+    // sub-tile of each step, group 1 the second.  The two threads of a row
+    // trade their sub-tile maxima through a double-buffered shared slot and a
+    // per-quadrant mbarrier (bounded wait).
+    const int g = (warp - kWarpSoft0) >> 2;
     const int q = warp & 3;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int row, i, qtile;
@@ -294,12 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       active = true;
       qtile = 2 * iA + (row >> 6);
     }
-    const int block = MODE == 0 ? 64 : 128;
-    const int n = i * block + row;
     const size_t tb = (size_t)bh * p.nq;
     const float c0 = active ? __ldg(p.sq + tb + qtile) * (kLog2e * 0.08838834764831845f) : 0.f;
-    float* xch = reinterpret_cast<float*>(smem + C::kOffBar + sizeof(Bars));  // [2][2][128]
-    const int xrow = 32 * q + lane;
+    const int xrow = 32 * q + lane;  // TMEM lane of this row
     uint8_t* prow_base = smem + C::kOffP + (MODE == 0 && lane >= 16 ? kTile : 0);
     // Metadata of this thread's sub-tile, one step ahead of use.
     auto tile_of = [&](int s) -> int {
@@ -313,9 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
     float sk_cur = kt_cur >= 0 ? __ldg(p.sk + tb + kt_cur) : 0.f;
     int kt_next = nsteps > 1 ? tile_of(1) : -1;
     float m_run = -INFINITY;
-    bool ok = true;
     for (int s = 0; s < nsteps; ++s) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[s & 1], (s >> 1) & 1, abort, p.wd));
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[s & 1], (s >> 1) & 1, abort, p.wd));
       if (!ok) break;
       tc_fence_after();
       const int nsub = MODE == 0 ? min(2, p.kc - 2 * s) : 2;
@@ -350,49 +370,52 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       if (!ok) break;
       const float mo = xch[((s & 1) * 2 + (g ^ 1)) * 128 + xrow];
       const float m_new = fmaxf(m_run, fmaxf(mu, mo));
-      const float alpha = (m_run == -INFINITY) ? 1.f : ex2(m_run - m_new);
-      // exponent of 448*P: (acc - max_u) * c_u + (m_u - m_new) + log2(448);
-      // the integer difference is exact, so values near the running max keep
-      // full precision however large the scores are.
+      if (g == 0) alpha_s[(s & 1) * 128 + xrow] = (m_run == -INFINITY) ? 1.f : ex2(m_run - m_new);
+      // exponent of 448*P: (acc - max_u) * c_u + (m_u - m_new) + log2(448); the
+      // integer difference is exact, so values near the running max keep full
+      // precision however large the scores are.
       const float off = nvalid > 0 ? (mu - m_new) + kLog2_448 : 0.f;
-      uint8_t* pbuf = prow_base + (s & 1) * C::kPBuf;
-      if (g < nsub) {
+      uint8_t* pbuf = prow_base + (s % kPBufs) * C::kPBuf;
+      // acc - max is an integer in [-2^22, 0]; adding it to the bit pattern of
+      // 1.5*2^23 and subtracting 1.5*2^23 converts it to float exactly on the
+      // ALU/FMA pipes (the integer-to-float instruction would share the pipe
+      // that evaluates ex2).
+      const int bias_i = 0x4B400000 - mx;
+      if (g < nsub && nvalid == 64) {
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {  // 16-key chunks
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float x[4];
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+              const float dif = __int_as_float((int)acc[16 * ch + 4 * e + z] + bias_i) - 12582912.0f;
+              x[z] = ex2(fmaf(dif, cu, off));
+            }
+            w[e] = __byte_perm(e4m3x2(x[0], x[1]), e4m3x2(x[2], x[3]), 0x5410);
+          }
+          *reinterpret_cast<uint4*>(pbuf + kmajor_off(row, 64 * g + 16 * ch, kQK_LBO, kQK_SBO)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      } else if (g < nsub) {
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = 16 * ch + 4 * e;
             float x[4];
 #pragma unroll
-            for (int z = 0; z < 4; ++z)
-              x[z] = (nvalid == 64 || c + z < nvalid)
-                         ? ex2(fmaf(__int2float_rn((int)acc[c + z] - mx), cu, off))
-                         : 0.f;
-            w[e] = e4m3x2(x[0], x[1]) | (e4m3x2(x[2], x[3]) << 16);
+            for (int z = 0; z < 4; ++z) {
+              const float dif = __int_as_float((int)acc[c + z] + bias_i) - 12582912.0f;
+              x[z] = c + z < nvalid ? ex2(fmaf(dif, cu, off)) : 0.f;
+            }
+            w[e] = __byte_perm(e4m3x2(x[0], x[1]), e4m3x2(x[2], x[3]), 0x5410);
           }
           *reinterpret_cast<uint4*>(pbuf + kmajor_off(row, 64 * g + 16 * ch, kQK_LBO, kQK_SBO)) =
               make_uint4(w[0], w[1], w[2], w[3]);
         }
-      }
-      // Rescale O (and its row-sum columns) when the running max moved.  The
-      // two groups split the 144 columns: 0-79 and 80-143.
-      if (s > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (s - 1) & 1, abort, p.wd));
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t obase = tmem + lane_base + kColO;
-        const int cbeg = g == 0 ? 0 : 80, cend = g == 0 ? 80 : kNO;
-#pragma unroll 1
-        for (int c = cbeg; c < cend; c += 16) {
-          uint32_t o[16];
-          SAGESLA_TMEM_LD16(obase + c, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int z = 0; z < 16; ++z) o[z] = __float_as_uint(__uint_as_float(o[z]) * alpha);
-          SAGESLA_TMEM_ST16(obase + c, o);
-        }
-        tmem_st_wait();
       }
       m_run = m_new;
       kt_cur = kt_next;
@@ -402,36 +425,85 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       tc_fence_before();
       mbar_arrive(&bars->p_full[s & 1]);
     }
-    // Epilogue: O_s = O / l * s_v (+ the linear branch already in out) -> bf16.
-    // The last PV steps may still be in flight here, and o_done may be more
-    // than one phase behind (a step that skips its rescale never waits on
-    // it), which a parity wait cannot tell apart; `fin` has a single phase,
-    // committed after the MMA thread's last instruction.
+  } else {
+    // ------------------------------ correction ----------------------------
+    // One warp per quadrant; thread = TMEM lane (one row of A/B or of the
+    // 128-row block).  Between PV(s-1) and PV(s) it multiplies the row's O
+    // and row-sum columns by alpha(s) when the running max moved.
+    const int q = warp & 3;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const uint32_t obase = tmem + lane_base + kColO;
+    const int xrow = 32 * q + lane;
+    int row, i;
+    bool active;
+    if (MODE == 0) {
+      row = 16 * q + (lane & 15);
+      i = lane >= 16 ? iB : iA;
+      active = lane >= 16 ? hasB : true;
+    } else {
+      row = 32 * q + lane;
+      i = iA;
+      active = true;
+    }
+    const int block = MODE == 0 ? 64 : 128;
+    const int n = i * block + row;
     const bool store = active && n < p.N;
-    __nv_bfloat16* orow = p.out + ((size_t)bh * p.N + (store ? n : 0)) * kD + 64 * g;
-    uint4 yrow[8];
+    bool ok = true;
+    for (int s = 0; s < nsteps; ++s) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->p_full[s & 1], (s >> 1) & 1, abort, p.wd));
+      if (!ok) break;
+      tc_fence_after();
+      const float alpha = alpha_s[(s & 1) * 128 + xrow];
+      // PV(s-1) must be complete before O is touched, before PV(s) may start
+      // and before QK^T(s+2) may release the P buffer softmax(s+3) writes.
+      if (s > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (s - 1) & 1, abort, p.wd));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->s_free[s & 1]);
+      if (s > 0) {
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < kNO; c += 16) {
+            uint32_t o[16];
+            SAGESLA_TMEM_LD16(obase + c, o);
+            tmem_ld_wait();
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
+            for (int z = 0; z < 16; ++z) o[z] = __float_as_uint(__uint_as_float(o[z]) * alpha);
+            SAGESLA_TMEM_ST16(obase + c, o);
+          }
+          tmem_st_wait();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->o_ready);
+    }
+    // Epilogue: O_s = O / l * s_v (+ the linear branch already in out) -> bf16.
+    __nv_bfloat16* orow = p.out + ((size_t)bh * p.N + (store ? n : 0)) * kD;
+    uint4 yrow[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
       yrow[c] = (p.add_out && store) ? *reinterpret_cast<const uint4*>(orow + 8 * c) : make_uint4(0, 0, 0, 0);
     if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->fin, 0, abort, p.wd));
     if (ok && nsteps > 0) {
       tc_fence_after();
-      const uint32_t obase = tmem + lane_base + kColO;
       uint32_t lw[16];
       SAGESLA_TMEM_LD16(obase + 128, lw);
       tmem_ld_wait();
       const float inv_l = 1.f / __uint_as_float(lw[0]);
 #pragma unroll
-      for (int c = 0; c < 64; c += 16) {
+      for (int c = 0; c < kD; c += 16) {
         uint32_t o[16];
-        SAGESLA_TMEM_LD16(obase + 64 * g + c, o);
+        SAGESLA_TMEM_LD16(obase + c, o);
         tmem_ld_wait();
         if (store) {
           uint32_t pk[8];
 #pragma unroll
           for (int z = 0; z < 8; ++z) {
             const uint32_t yw = z < 4 ? (&yrow[c / 8].x)[z] : (&yrow[c / 8 + 1].x)[z - 4];
-            const int ch = 64 * g + c + 2 * z;
+            const int ch = c + 2 * z;
             const float a = __uint_as_float(o[2 * z]) * inv_l * __ldg(p.sv + (size_t)bh * kD + ch) + bf16_lo(yw);
             const float b = __uint_as_float(o[2 * z + 1]) * inv_l * __ldg(p.sv + (size_t)bh * kD + ch + 1) + bf16_hi(yw);
             const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -442,6 +514,11 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         }
       }
     }
+  }
+  // Every MMA has completed once `fin` has both issuers' arrivals.
+  if (warp == 1) {
+    if (lane == 0) mbar_wait_drain(&bars->fin, 0, p.wd);
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
