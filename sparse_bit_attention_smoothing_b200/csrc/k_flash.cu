@@ -9,15 +9,18 @@
 // smoothing on integer tensor cores) and 支柱二 (only the selected blocks are
 // computed exactly); 量子位 news 技术解密 1 (SageAttention2++).
 //
-// Roles on the SM (15 warps, 1 CTA/SM):
-//   warp 0     producer: bulk copies of Q^, K^ and V^T tiles (pre-tiled in
+// Roles on the SM (16 warps, 1 CTA/SM):
+//   warp 0     K producer: bulk copies of the Q^ and K^ tiles (pre-tiled in
 //              HBM by the quantiser, so one cp.async.bulk moves a whole tile);
 //   warp 1     QK^T issuer (one thread) and TMEM owner;
 //   warp 2     PV issuer (one thread) -- two issuers keep the tensor pipe fed
 //              while either of them waits;
-//   warps 3-10 softmax: two warps per TMEM lane quadrant, each owning one
+//   warp 3     V producer: bulk copies of the V^T tiles.  K and V have their
+//              own producers so a K copy never queues behind a V stage that
+//              the later PV step still holds;
+//   warps 4-11 softmax: two warps per TMEM lane quadrant, each owning one
 //              64-key sub-tile of the 128-key step of every row;
-//   warps 11-14 correction: one warp per quadrant; rescales O by
+//   warps 12-15 correction: one warp per quadrant; rescales O by
 //              exp(m_old - m_new) between PV steps, off the softmax path, and
 //              runs the epilogue.
 // Mode 64 (block 64): a CTA owns two query blocks A and B.  Their M=64
@@ -46,8 +49,8 @@ constexpr int kStages = 2;
 constexpr int kPBufs = 3;
 constexpr int kSoftThreads = 256;
 constexpr int kCorrThreads = 128;
-constexpr int kWarpSoft0 = 3, kWarpCorr0 = 11;
-constexpr int kThreads = 32 * 3 + kSoftThreads + kCorrThreads;  // 480
+constexpr int kWarpSoft0 = 4, kWarpCorr0 = 12;
+constexpr int kThreads = 32 * 4 + kSoftThreads + kCorrThreads;  // 512
 constexpr int kVSlot = kTile + 1024;  // 8 KB V^T tile + 16 rows of ones (1 KB)
 constexpr uint32_t kOnesE4M3 = 0x38383838u;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -161,22 +164,30 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
 
-  if (warp == 0) {
-    // ------------------------------ producer ------------------------------
+  if (warp == 0 || warp == 3) {
+    // ------------------------- K and V producers --------------------------
+    // warp 0 copies Q^ and the K^ tiles of each step, warp 3 the V^T tiles.
+    // The list entries of step s+1 are read before the wait for stage s, so
+    // their latency hides behind it.
     if (lane == 0) {
+      const bool is_k = warp == 0;
       const size_t head_tiles = (size_t)bh * p.nq;
-      mbar_expect_tx(&bars->q_full, C::kQBytes);
-      if (MODE == 0) {
-        bulk_g2s(smem + C::kOffQ, p.q8t + (head_tiles + iA) * kTile, kTile, &bars->q_full);
-        const int ib = hasB ? iB : iA;  // keep the transaction count fixed
-        bulk_g2s(smem + C::kOffQ + kTile, p.q8t + (head_tiles + ib) * kTile, kTile, &bars->q_full);
-      } else {
-        bulk_g2s(smem + C::kOffQ, p.q8t + (head_tiles + 2 * iA) * kTile, 2 * kTile, &bars->q_full);
+      if (is_k) {
+        mbar_expect_tx(&bars->q_full, C::kQBytes);
+        if (MODE == 0) {
+          bulk_g2s(smem + C::kOffQ, p.q8t + (head_tiles + iA) * kTile, kTile, &bars->q_full);
+          const int ib = hasB ? iB : iA;  // keep the transaction count fixed
+          bulk_g2s(smem + C::kOffQ + kTile, p.q8t + (head_tiles + ib) * kTile, kTile, &bars->q_full);
+        } else {
+          bulk_g2s(smem + C::kOffQ, p.q8t + (head_tiles + 2 * iA) * kTile, 2 * kTile, &bars->q_full);
+        }
       }
-      int k_issued = 0, v_issued = 0;  // steps whose copies were issued
-      for (int s = 0; s < nsteps && !*abort; ++s) {
-        const int st = s % kStages;
-        int jj[2][2] = {{-1, -1}, {-1, -1}};
+      uint64_t* full = is_k ? bars->k_full : bars->v_full;
+      uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
+      const uint8_t* src = is_k ? p.k8t : p.v8t;
+      auto entries = [&](int s, int (&jj)[2][2]) {
+        jj[0][0] = jj[0][1] = jj[1][0] = jj[1][1] = -1;
+        if (s >= nsteps) return;
         if (MODE == 0) {
           const int nsub = min(2, p.kc - 2 * s);
           for (int x = 0; x < 2; ++x) {
@@ -186,40 +197,43 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         } else {
           jj[0][0] = list_at(p, bh, iA, s);
         }
-        if (s >= kStages && !mbar_wait(&bars->k_empty[st], ((s / kStages) - 1) & 1, abort, p.wd)) break;
-        uint8_t* kd = smem + C::kOffK + st * C::kKStage;
-        uint8_t* vd = smem + C::kOffV + st * C::kVStage;
+      };
+      int jn[2][2];
+      entries(0, jn);
+      int issued = 0;  // steps whose copies were issued
+      for (int s = 0; s < nsteps && !*abort; ++s) {
+        const int st = s % kStages;
+        int jj[2][2];
+        for (int x = 0; x < 2; ++x)
+          for (int u = 0; u < 2; ++u) jj[x][u] = jn[x][u];
+        entries(s + 1, jn);
+        if (s >= kStages && !mbar_wait(&empty[st], ((s / kStages) - 1) & 1, abort, p.wd)) break;
         if (MODE == 0) {
           const int nsub = min(2, p.kc - 2 * s);
-          mbar_expect_tx(&bars->k_full[st], 2 * nsub * kTile);
+          mbar_expect_tx(&full[st], 2 * nsub * kTile);
           for (int x = 0; x < 2; ++x)
-            for (int u = 0; u < nsub; ++u)
-              bulk_g2s(kd + (2 * x + u) * kTile, p.k8t + (head_tiles + jj[x][u]) * kTile, kTile, &bars->k_full[st]);
-          k_issued = s + 1;
-          if (s >= kStages && !mbar_wait(&bars->v_empty[st], ((s / kStages) - 1) & 1, abort, p.wd)) break;
-          mbar_expect_tx(&bars->v_full[st], 2 * nsub * kTile);
-          for (int x = 0; x < 2; ++x)
-            for (int u = 0; u < nsub; ++u)
-              bulk_g2s(vd + (2 * x + u) * kVSlot, p.v8t + (head_tiles + jj[x][u]) * kTile, kTile, &bars->v_full[st]);
-          v_issued = s + 1;
+            for (int u = 0; u < nsub; ++u) {
+              uint8_t* dst = is_k ? smem + C::kOffK + st * C::kKStage + (2 * x + u) * kTile
+                                  : smem + C::kOffV + st * C::kVStage + (2 * x + u) * kVSlot;
+              bulk_g2s(dst, src + (head_tiles + jj[x][u]) * kTile, kTile, &full[st]);
+            }
         } else {
           const int j = jj[0][0];
-          mbar_expect_tx(&bars->k_full[st], 2 * kTile);
-          bulk_g2s(kd, p.k8t + (head_tiles + 2 * j) * kTile, 2 * kTile, &bars->k_full[st]);
-          k_issued = s + 1;
-          if (s >= kStages && !mbar_wait(&bars->v_empty[st], ((s / kStages) - 1) & 1, abort, p.wd)) break;
-          mbar_expect_tx(&bars->v_full[st], 2 * kTile);
-          bulk_g2s(vd, p.v8t + (head_tiles + 2 * j) * kTile, kTile, &bars->v_full[st]);
-          bulk_g2s(vd + kVSlot, p.v8t + (head_tiles + 2 * j + 1) * kTile, kTile, &bars->v_full[st]);
-          v_issued = s + 1;
+          mbar_expect_tx(&full[st], 2 * kTile);
+          if (is_k) {
+            bulk_g2s(smem + C::kOffK + st * C::kKStage, src + (head_tiles + 2 * j) * kTile, 2 * kTile, &full[st]);
+          } else {
+            uint8_t* vd = smem + C::kOffV + st * C::kVStage;
+            bulk_g2s(vd, src + (head_tiles + 2 * j) * kTile, kTile, &full[st]);
+            bulk_g2s(vd + kVSlot, src + (head_tiles + 2 * j + 1) * kTile, kTile, &full[st]);
+          }
         }
+        issued = s + 1;
       }
       // Drain: every copy issued must land before the CTA may exit.
-      mbar_wait_drain(&bars->q_full, 0, p.wd);
-      for (int s = max(0, k_issued - kStages); s < k_issued; ++s)
-        mbar_wait_drain(&bars->k_full[s % kStages], (s / kStages) & 1, p.wd);
-      for (int s = max(0, v_issued - kStages); s < v_issued; ++s)
-        mbar_wait_drain(&bars->v_full[s % kStages], (s / kStages) & 1, p.wd);
+      if (is_k) mbar_wait_drain(&bars->q_full, 0, p.wd);
+      for (int s = max(0, issued - kStages); s < issued; ++s)
+        mbar_wait_drain(&full[s % kStages], (s / kStages) & 1, p.wd);
     }
   } else if (warp == 1) {
     // ------------------------------ QK^T issuer ---------------------------
@@ -351,9 +365,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         SAGESLA_TMEM_LD16(sbase + 48, acc + 48);
         tmem_ld_wait();
       }
-      // Prefetch the key scale of the next step (its list entry arrived).
-      const float sk_next = kt_next >= 0 ? __ldg(p.sk + tb + kt_next) : 0.f;
-      const int kt_after = (s + 2 < nsteps) ? tile_of(s + 2) : -1;
       int mx = INT_MIN;
       if (nvalid == 64) {
 #pragma unroll
@@ -366,6 +377,11 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       const float mu = nvalid > 0 ? __int2float_rn(mx) * cu : -INFINITY;
       xch[((s & 1) * 2 + g) * 128 + xrow] = mu;
       mbar_arrive(&bars->xbar[q][s & 1]);
+      // Prefetch the key scale of the next step (its list entry arrived) only
+      // now: an mbarrier arrive has release semantics and would wait for
+      // these global loads to complete.
+      const float sk_next = kt_next >= 0 ? __ldg(p.sk + tb + kt_next) : 0.f;
+      const int kt_after = (s + 2 < nsteps) ? tile_of(s + 2) : -1;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->xbar[q][s & 1], (s >> 1) & 1, abort, p.wd));
       if (!ok) break;
       const float mo = xch[((s & 1) * 2 + (g ^ 1)) * 128 + xrow];
