@@ -167,6 +167,7 @@ struct Buffers {
   float* z;           // z_j [BH][nb][128]
   uint32_t* selbits;  // [BH][nb][2*nbt]
   float* zl;          // Z_i [BH][nb][128]
+  float* ztot;        // sum of z_j over all j [BH][128]
   uint16_t* himg;     // H_i^T images [BH][nb][128*128]
   uint16_t* wimg;     // proj_w image
   size_t total;
@@ -202,11 +203,12 @@ Buffers carve(uint8_t* base, const Geom& g, bool linear = false) {
     b.z = reinterpret_cast<float*>(take(BH * g.nb * kD * sizeof(float)));
     b.selbits = reinterpret_cast<uint32_t*>(take(BH * g.nb * 2 * nbt * sizeof(uint32_t)));
     b.zl = reinterpret_cast<float*>(take(BH * g.nb * kD * sizeof(float)));
+    b.ztot = reinterpret_cast<float*>(take(BH * kD * sizeof(float)));
     b.himg = reinterpret_cast<uint16_t*>(take(BH * g.nb * 16384 * sizeof(uint16_t)));
     b.wimg = reinterpret_cast<uint16_t*>(take(16384 * sizeof(uint16_t)));
   } else {
     b.hs = nullptr;
-    b.z = b.zl = nullptr;
+    b.z = b.zl = b.ztot = nullptr;
     b.selbits = nullptr;
     b.himg = b.wimg = nullptr;
   }
@@ -267,7 +269,7 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
   if (!dense) {
     ProfScope ps(3, st);
     SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, b.idx, b.qbar, b.kbar, linear ? b.z : nullptr,
-                                           b.selbits, b.zl, st)));
+                                           b.ztot, b.selbits, b.zl, st)));
   }
   if (linear) {
     {
@@ -405,7 +407,7 @@ int sagesla_get_mask(const void* q, const void* k, int B, int H, int N, int d, i
   // (its quantised codes are discarded).
   SAGESLA_TRY(run_front(q, k, k, g, b, st));
   SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, idx_out, qbar ? qbar : b.qbar, kbar ? kbar : b.kbar,
-                                         nullptr, nullptr, nullptr, st)));
+                                         nullptr, nullptr, nullptr, nullptr, st)));
   if (k_out) *k_out = g.kc;
   return SAGESLA_OK;
 }

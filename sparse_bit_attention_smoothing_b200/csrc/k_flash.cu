@@ -367,8 +367,13 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       }
       int mx = INT_MIN;
       if (nvalid == 64) {
+        int m2[2] = {INT_MIN, INT_MIN};  // two chains of three-input maxima
 #pragma unroll
-        for (int c = 0; c < 64; ++c) mx = max(mx, (int)acc[c]);
+        for (int c = 0; c < 64; c += 4) {
+          m2[0] = __vimax3_s32(m2[0], (int)acc[c], (int)acc[c + 1]);
+          m2[1] = __vimax3_s32(m2[1], (int)acc[c + 2], (int)acc[c + 3]);
+        }
+        mx = max(m2[0], m2[1]);
       } else {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
@@ -390,13 +395,14 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       // exponent of 448*P: (acc - max_u) * c_u + (m_u - m_new) + log2(448); the
       // integer difference is exact, so values near the running max keep full
       // precision however large the scores are.
-      const float off = nvalid > 0 ? (mu - m_new) + kLog2_448 : 0.f;
+      // Exponent of 448*P~: S*log2(e) - m_new + log2(448), one fused
+      // multiply-add per key on the integer score (exact in fp32: |acc| <
+      // 2^24), two keys per f32x2 instruction; keys past the sequence end
+      // (last key block) get P~ = 0.
       uint8_t* pbuf = prow_base + (s % kPBufs) * C::kPBuf;
-      // acc - max is an integer in [-2^22, 0]; adding it to the bit pattern of
-      // 1.5*2^23 and subtracting 1.5*2^23 converts it to float exactly on the
-      // ALU/FMA pipes (the integer-to-float instruction would share the pipe
-      // that evaluates ex2).
-      const int bias_i = 0x4B400000 - mx;
+      const float kk = kLog2_448 - m_new;
+      const uint64_t cc = f32x2_pack(cu, cu), ko = f32x2_pack(kk, kk);
+      // (two copies of the loop: the masked one only for a ragged last block)
       if (g < nsub && nvalid == 64) {
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {  // 16-key chunks
@@ -405,9 +411,14 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
           for (int e = 0; e < 4; ++e) {
             float x[4];
 #pragma unroll
-            for (int z = 0; z < 4; ++z) {
-              const float dif = __int_as_float((int)acc[16 * ch + 4 * e + z] + bias_i) - 12582912.0f;
-              x[z] = ex2(fmaf(dif, cu, off));
+            for (int z = 0; z < 4; z += 2) {
+              const int c = 16 * ch + 4 * e + z;
+              const uint64_t d =
+                  f32x2_fma(f32x2_pack(__int2float_rn((int)acc[c]), __int2float_rn((int)acc[c + 1])), cc, ko);
+              float a, b;
+              f32x2_unpack(d, a, b);
+              x[z] = ex2(a);
+              x[z + 1] = ex2(b);
             }
             w[e] = __byte_perm(e4m3x2(x[0], x[1]), e4m3x2(x[2], x[3]), 0x5410);
           }
@@ -416,17 +427,24 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         }
       } else if (g < nsub) {
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 4; ++ch) {  // 16-key chunks
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int c = 16 * ch + 4 * e;
             float x[4];
 #pragma unroll
-            for (int z = 0; z < 4; ++z) {
-              const float dif = __int_as_float((int)acc[c + z] + bias_i) - 12582912.0f;
-              x[z] = c + z < nvalid ? ex2(fmaf(dif, cu, off)) : 0.f;
+            for (int z = 0; z < 4; z += 2) {
+              const int c = 16 * ch + 4 * e + z;
+              const uint64_t d =
+                  f32x2_fma(f32x2_pack(__int2float_rn((int)acc[c]), __int2float_rn((int)acc[c + 1])), cc, ko);
+              float a, b;
+              f32x2_unpack(d, a, b);
+              x[z] = ex2(a);
+              x[z + 1] = ex2(b);
             }
+#pragma unroll
+            for (int z = 0; z < 4; ++z)
+              if (16 * ch + 4 * e + z >= nvalid) x[z] = 0.f;
             w[e] = __byte_perm(e4m3x2(x[0], x[1]), e4m3x2(x[2], x[3]), 0x5410);
           }
           *reinterpret_cast<uint4*>(pbuf + kmajor_off(row, 64 * g + 16 * ch, kQK_LBO, kQK_SBO)) =

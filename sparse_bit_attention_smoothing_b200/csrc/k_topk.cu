@@ -17,7 +17,6 @@
 
 namespace sagesla {
 
-constexpr int kTQ = 8;       // query blocks per CTA (one warp each in phase 2)
 constexpr int kKC = 64;      // key blocks per staged chunk
 constexpr int kPad = 132;    // padded row length of the kbar chunk (floats)
 
@@ -44,34 +43,65 @@ __global__ void pool_means_kernel(const float* __restrict__ qsum, const float* _
   kbar[((size_t)bh * nb + i) * kD + c] = pooled(ksum + (size_t)bh * nq * kD, i, block, N, c);
 }
 
+// Sum of z_j over all key blocks of each head, once: grid (BH), 1024
+// threads.  Eight slices of 128 channels add every eighth block, then the
+// slices are added in a fixed order (deterministic).
+__global__ void __launch_bounds__(1024) z_total_kernel(const float* __restrict__ zin, int nb,
+                                                       float* __restrict__ ztot) {
+  __shared__ float part[8][kD];
+  const int bh = blockIdx.x, c = threadIdx.x & (kD - 1), sl = threadIdx.x >> 7;
+  const float* zh = zin + (size_t)bh * nb * kD + c;
+  float a0 = 0.f, a1 = 0.f;
+  int j = sl;
+  for (; j + 8 < nb; j += 16) {
+    a0 += zh[(size_t)j * kD];
+    a1 += zh[(size_t)(j + 8) * kD];
+  }
+  if (j < nb) a0 += zh[(size_t)j * kD];
+  part[sl][c] = a0 + a1;
+  __syncthreads();
+  if (sl == 0)
+    ztot[(size_t)bh * kD + c] =
+        ((part[0][c] + part[1][c]) + (part[2][c] + part[3][c])) + ((part[4][c] + part[5][c]) + (part[6][c] + part[7][c]));
+}
+
 // Linear-branch outputs (when zin != NULL): selbits [nb][nbw] words with
 // bit j set when key block j is selected; zout [nb][128] the fp32 sums
-// Z_i = sum_{j not in S_i} z_j, formed as (sum over all j) - (sum over S_i).
-__global__ void __launch_bounds__(256) pool_topk_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
-                                                        int nb, int kc, int32_t* __restrict__ idx,
-                                                        const float* __restrict__ zin,
-                                                        uint32_t* __restrict__ selbits, int nbw,
-                                                        float* __restrict__ zout) {
+// Z_i = sum_{j not in S_i} z_j, formed as (sum over all j, ztot) - (sum over
+// S_i).
+//
+// TQ query blocks per CTA, 32*TQ threads.  Phase 1: thread -> key block
+// t % 64 of each staged chunk and query rows 2*(t/64), 2*(t/64)+1.  Phase 2:
+// one warp per query row; with PER > 0 each lane keeps the order keys of
+// blocks lane, lane+32, ... (PER of them, nb <= 32*PER) in registers for the
+// 32-step threshold search, else it rereads them from shared memory.
+template <int TQ, int PER>
+__global__ void __launch_bounds__(32 * TQ) pool_topk_kernel(const float* __restrict__ qbar,
+                                                           const float* __restrict__ kbar, int nb, int kc,
+                                                           int32_t* __restrict__ idx, const float* __restrict__ zin,
+                                                           const float* __restrict__ ztot,
+                                                           uint32_t* __restrict__ selbits, int nbw,
+                                                           float* __restrict__ zout) {
+  constexpr int kThr = 32 * TQ;
   extern __shared__ __align__(16) float sm[];
-  float* qb = sm;                            // [kTQ][128]
-  float* kb = qb + kTQ * kD;                 // [kKC][kPad]
-  float* sc = kb + kKC * kPad;               // [kTQ][nb]
+  float* qb = sm;                            // [TQ][128]
+  float* kb = qb + TQ * kD;                  // [kKC][kPad]
+  float* sc = kb + kKC * kPad;               // [TQ][nb]
   const int bh = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int i0 = blockIdx.x * kTQ;
+  const int i0 = blockIdx.x * TQ;
   const float* qh = qbar + (size_t)bh * nb * kD;
   const float* kh = kbar + (size_t)bh * nb * kD;
   const float rs = 1.0f / sqrtf((float)kD);
 
-  for (int e = t; e < kTQ * kD; e += 256) {
+  for (int e = t; e < TQ * kD; e += kThr) {
     const int r = e / kD;
     qb[e] = i0 + r < nb ? qh[(size_t)i0 * kD + e] : 0.f;
   }
-  // Phase 1: scores.  Thread -> key block jj = t % 64 of the chunk, query
-  // rows 2*(t/64) and 2*(t/64)+1.
+  // Phase 1: scores, fp32 FMA in channel order.
   const int jj = t & 63, qg = t >> 6;
   for (int j0 = 0; j0 < nb; j0 += kKC) {
     __syncthreads();
-    for (int e = t; e < kKC * kD / 4; e += 256) {
+    for (int e = t; e < kKC * kD / 4; e += kThr) {
       const int r = e / (kD / 4), c4 = e % (kD / 4);
       const int j = j0 + r;
       const float4 val = j < nb ? *reinterpret_cast<const float4*>(kh + (size_t)j * kD + 4 * c4)
@@ -103,78 +133,134 @@ __global__ void __launch_bounds__(256) pool_topk_kernel(const float* __restrict_
       sc[(2 * qg + 1) * nb + j] = a1 * rs;
     }
   }
-  // Total of z over all key blocks of the head (fixed order), for Z_i.
-  __shared__ float ztot[kD];
-  if (zin && t < kD) {
-    float a = 0.f;
-    for (int j = 0; j < nb; ++j) a += zin[((size_t)bh * nb + j) * kD + t];
-    ztot[t] = a;
-  }
   __syncthreads();
   // Phase 2: one warp per query row.
   const int i = i0 + warp;
   if (i >= nb) return;
   const float* row = sc + warp * nb;
+  // The selected indices are also kept in this row's score slots: entry
+  // pos <= j is written only after every lane has read score j.
+  int* lst = reinterpret_cast<int*>(sc + warp * nb);
+  uint32_t keys[PER > 0 ? PER : 1];
+  if (PER > 0) {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int j = 32 * u + lane;
+      keys[u] = j < nb ? order_key(row[j]) : 0u;  // 0 is never counted: every candidate is >= 1
+    }
+  }
   // Largest T with #{key >= T} >= kc: built bit by bit from the top.
   uint32_t T = 0;
   for (int b = 31; b >= 0; --b) {
     const uint32_t cand = T | (1u << b);
     int cnt = 0;
-    for (int j = lane; j < nb; j += 32) cnt += order_key(row[j]) >= cand ? 1 : 0;
+    if (PER > 0) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+      for (int u = 0; u < PER; ++u) cnt += keys[u] >= cand ? 1 : 0;
+    } else {
+      for (int j = lane; j < nb; j += 32) cnt += order_key(row[j]) >= cand ? 1 : 0;
+    }
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
     if (cnt >= kc) T = cand;
   }
   int gt = 0;
-  for (int j = lane; j < nb; j += 32) gt += order_key(row[j]) > T ? 1 : 0;
+  if (PER > 0) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) gt += __shfl_xor_sync(0xffffffffu, gt, o);
+    for (int u = 0; u < PER; ++u) gt += (32 * u + lane < nb && keys[u] > T) ? 1 : 0;
+  } else {
+    for (int j = lane; j < nb; j += 32) gt += order_key(row[j]) > T ? 1 : 0;
+  }
+  gt = __reduce_add_sync(0xffffffffu, gt);
   const int need_eq = kc - gt;  // >= 1 by construction of T
   int32_t* out = idx + ((size_t)bh * nb + i) * kc;
   int pos = 0, eq_seen = 0;
-  for (int j0 = 0; j0 < nb; j0 += 32) {
-    const int j = j0 + lane;
-    const uint32_t key = j < nb ? order_key(row[j]) : 0u;
-    const bool is_eq = j < nb && key == T;
-    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
-    const int eq_rank = eq_seen + __popc(eqm & ((1u << lane) - 1u));
-    const bool sel = j < nb && (key > T || (is_eq && eq_rank < need_eq));
-    const unsigned sm_ = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[pos + __popc(sm_ & ((1u << lane) - 1u))] = j;
-    if (selbits && lane == 0) selbits[((size_t)bh * nb + i) * nbw + (j0 >> 5)] = sm_;
-    pos += __popc(sm_);
-    eq_seen += __popc(eqm);
+  const int nch = (nb + 31) >> 5;
+#pragma unroll
+  for (int u = 0; u < (PER > 0 ? PER : 1); ++u) {
+    for (int uu = u; uu < (PER > 0 ? u + 1 : nch); ++uu) {
+      if (uu >= nch) break;
+      const int j = 32 * uu + lane;
+      const uint32_t key = j < nb ? (PER > 0 ? keys[u] : order_key(row[j])) : 0u;
+      const bool is_eq = j < nb && key == T;
+      const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+      const int eq_rank = eq_seen + __popc(eqm & ((1u << lane) - 1u));
+      const bool sel = j < nb && (key > T || (is_eq && eq_rank < need_eq));
+      const unsigned sm_ = __ballot_sync(0xffffffffu, sel);
+      if (sel) {
+        const int at = pos + __popc(sm_ & ((1u << lane) - 1u));
+        out[at] = j;
+        lst[at] = j;
+      }
+      if (selbits && lane == 0) selbits[((size_t)bh * nb + i) * nbw + uu] = sm_;
+      pos += __popc(sm_);
+      eq_seen += __popc(eqm);
+    }
   }
   if (selbits)
-    for (int w = ((nb + 31) >> 5) + lane; w < nbw; w += 32) selbits[((size_t)bh * nb + i) * nbw + w] = 0u;
+    for (int w = nch + lane; w < nbw; w += 32) selbits[((size_t)bh * nb + i) * nbw + w] = 0u;
   if (zin) {
     __syncwarp();
     float zs[4];
 #pragma unroll
     for (int m = 0; m < 4; ++m) zs[m] = 0.f;
-    for (int tt = 0; tt < kc; ++tt) {
-      const int j = out[tt];
+    const float* zh = zin + (size_t)bh * nb * kD + lane;
+    // Eight rows of z in flight per lane; added in list order.
+    for (int t0 = 0; t0 < kc; t0 += 8) {
+      float v[8][4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) zs[m] += zin[((size_t)bh * nb + j) * kD + lane + 32 * m];
+      for (int u = 0; u < 8; ++u) {
+        const int j = t0 + u < kc ? lst[t0 + u] : -1;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) v[u][m] = j >= 0 ? __ldg(zh + (size_t)j * kD + 32 * m) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) zs[m] += v[u][m];
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) zout[((size_t)bh * nb + i) * kD + lane + 32 * m] = ztot[lane + 32 * m] - zs[m];
+    for (int m = 0; m < 4; ++m)
+      zout[((size_t)bh * nb + i) * kD + lane + 32 * m] = ztot[(size_t)bh * kD + lane + 32 * m] - zs[m];
   }
 }
 
-size_t pool_topk_smem(int nb) { return sizeof(float) * ((size_t)kTQ * kD + (size_t)kKC * kPad + (size_t)kTQ * nb); }
+namespace {
+
+size_t topk_smem(int tq, int nb) { return sizeof(float) * ((size_t)tq * kD + (size_t)kKC * kPad + (size_t)tq * nb); }
+
+template <int TQ, int PER>
+cudaError_t launch_topk_cfg(const float* qbar, const float* kbar, const Geom& g, int32_t* idx, const float* zin,
+                            const float* ztot, uint32_t* selbits, float* zout, cudaStream_t st) {
+  const size_t smem = topk_smem(TQ, g.nb);
+  cudaError_t e = cudaFuncSetAttribute(pool_topk_kernel<TQ, PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  pool_topk_kernel<TQ, PER><<<dim3((g.nb + TQ - 1) / TQ, g.BH), 32 * TQ, smem, st>>>(
+      qbar, kbar, g.nb, g.kc, idx, zin, ztot, selbits, 2 * ((g.nb + 63) / 64), zout);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t pool_topk_smem(int nb) { return topk_smem(4, nb); }
 
 cudaError_t launch_pool_topk(const float* qsum, const float* ksum, const Geom& g, int32_t* idx, float* qbar,
-                             float* kbar, const float* zin, uint32_t* selbits, float* zout, cudaStream_t st) {
+                             float* kbar, const float* zin, float* ztot, uint32_t* selbits, float* zout,
+                             cudaStream_t st) {
   pool_means_kernel<<<dim3(g.nb, g.BH), kD, 0, st>>>(qsum, ksum, g.N, g.block, g.nb, g.nq, qbar, kbar);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = pool_topk_smem(g.nb);
-  e = cudaFuncSetAttribute(pool_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  pool_topk_kernel<<<dim3((g.nb + kTQ - 1) / kTQ, g.BH), 256, smem, st>>>(qbar, kbar, g.nb, g.kc, idx, zin, selbits,
-                                                                           2 * ((g.nb + 63) / 64), zout);
-  return cudaGetLastError();
+  if (zin) {
+    z_total_kernel<<<g.BH, 1024, 0, st>>>(zin, g.nb, ztot);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // Eight query blocks per CTA where the scores fit in shared memory (three
+  // CTAs per SM at 720p), and the order keys in registers up to nb = 1280.
+  constexpr size_t kSmemMax = 227 * 1024;
+  if (topk_smem(8, g.nb) <= kSmemMax)
+    return g.nb <= 32 * 40 ? launch_topk_cfg<8, 40>(qbar, kbar, g, idx, zin, ztot, selbits, zout, st)
+                           : launch_topk_cfg<8, 0>(qbar, kbar, g, idx, zin, ztot, selbits, zout, st);
+  return launch_topk_cfg<4, 0>(qbar, kbar, g, idx, zin, ztot, selbits, zout, st);
 }
 
 }  // namespace sagesla

@@ -36,7 +36,8 @@ cudaError_t launch_untile(const uint8_t* q8t, const uint8_t* k8t, const uint8_t*
 // With zin != NULL also writes the selection bitmask (2*ceil(nb/64) words
 // per query block) and Z_i = sum of z_j over the unselected key blocks.
 cudaError_t launch_pool_topk(const float* qsum, const float* ksum, const Geom& g, int32_t* idx, float* qbar,
-                             float* kbar, const float* zin, uint32_t* selbits, float* zout, cudaStream_t st);
+                             float* kbar, const float* zin, float* ztot, uint32_t* selbits, float* zout,
+                             cudaStream_t st);
 // K4a: per key block h_j = phi(K_j)^T V_j (bf16 mask-GEMM tiles) and z_j.
 cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_t* hs, float* z, int* wd,
                              cudaStream_t st);

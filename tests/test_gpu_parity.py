@@ -67,6 +67,24 @@ def test_mask_bit_exact_up_to_near_ties(sg, orc, B, H, N, outl, block, topk):
     assert eq + near == B * H * nb
 
 
+@pytest.mark.parametrize("N,block,topk", [(75600, 64, 0.1), (90000, 64, 0.1), (75600, 128, 0.1)])
+def test_mask_full_length_sequences(sg, orc, N, block, topk):
+    """Full-length rows (1182 and 1407 key blocks): both selection paths of the
+    top-k kernel (order keys held in registers up to 1280 blocks, re-read from
+    shared memory beyond)."""
+    q, k, _, _ = _inputs(1, 1, N, True, seed=3)
+    r = sg.sagesla_get_mask(*_dev(q, k), block=block, topk=topk)
+    torch.cuda.synchronize()
+    qf, kf = q.reshape(1, N, 128), k.reshape(1, N, 128)
+    o = orc.mask(qf, kf, block, topk)
+    assert r["k"] == o["k"]
+    nb = o["idx"].shape[1]
+    s64 = orc.block_scores_f64(qf, kf, block)
+    gi = r["idx"].cpu().numpy().reshape(nb, -1)
+    eq, near = compare_masks(gi, o["idx"].reshape(nb, -1), s64.reshape(nb, nb), r["k"])
+    assert eq + near == nb
+
+
 def _check_out(got, ref):
     got = got.float().cpu().numpy().astype(np.float64)
     err = max_abs_excess(got, ref)
