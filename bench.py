@@ -199,7 +199,9 @@ def main():
     import torch
     import torch.distributed as dist
 
-    rank, world, local = _env_int("RANK", 0), _env_int("WORLD_SIZE", 1), _env_int("LOCAL_RANK", 0)
+    from sparse_bit_attention_smoothing_b200.replicas import job_throughput, max_over_ranks, rank_env
+
+    rank, world, local = rank_env()
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
@@ -244,14 +246,10 @@ def main():
     prof = sg.profile_read()
     sg.profile(False)
     status = sg.sync_status()
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], device="cuda")[0]
 
     f = flops(w)
-    value = world * f["dense"] / (ms * 1e-3) / 1e12
+    value = job_throughput(f["dense"], world, ms) / 1e12
     pk = peaks()
     peak8 = 2.0 * pk["bf16"]  # 8-bit dense = 2 x bf16 (nominal 4.5 / 2.25 PFLOP/s)
     fl_ms, fl_n = prof.get("flash", (0.0, 0))
@@ -270,11 +268,7 @@ def main():
     t0 = time.perf_counter()
     for _ in range(args.e2e_steps):
         sg.sagesla_attn_host(hq, hk, hv, hw, out=hout, block=w.block, topk=w.topk, stream=st)
-    e2e_ms = (time.perf_counter() - t0) * 1e3 / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks([(time.perf_counter() - t0) * 1e3 / args.e2e_steps], device="cuda")[0]
     E = q.numel() * 2
     h2d = 3 * E + (pw.numel() * 2 if pw is not None else 0)
 
@@ -291,7 +285,7 @@ def main():
                          "kernel": "flash", "peak_note": f"8-bit = 2 x {pk['src']} bf16 burst {pk['bf16']}",
                          "path_t_roof_ms": t_roof * 1e3, "path_frac": t_roof * 1e3 / ms},
             "clocks": clocks,
-            "e2e": {"value": world * f["dense"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+            "e2e": {"value": job_throughput(f["dense"], world, e2e_ms) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": E}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(w, q, k, v, pw)
