@@ -51,22 +51,27 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }  // namespace
 
 // ---------------------------------------------------------------- K4a ----
-// grid (nbt*32, BH): CTA x handles key blocks j = 2x, 2x+1 (zeros past nb).
-// 128 threads; thread 0 issues the MMAs.  Dynamic smem: per block, A (phi(K)
-// rows) and B (V rows) MN-major, BLK x 128 bf16 each; plus the 32 KB image.
+// grid (nbt*32, BH): CTA x handles key blocks j = 2x, 2x+1 (zeros past nb),
+// so both 16-byte halves of every 32-byte sector of the h tiles come from one
+// CTA.  256 threads; thread t owns channels 8*(t%16).. and token rows t/16 +
+// 16r of 64-row rounds: all its K and V loads of a round are issued before
+// any is used (64 KB in flight per CTA, two CTAs per SM).  Thread 0 issues
+// the MMAs.  Dynamic smem: per block, A (phi(K) rows) and B (V rows)
+// MN-major, BLK x 128 bf16 each; after the MMAs the same bytes stage the two
+// bf16 h images.
 template <int BLK>
-__global__ void __launch_bounds__(128) linear_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int N,
+__global__ void __launch_bounds__(256) linear_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int N,
                                                         int nb, int nbt, uint8_t* __restrict__ hs,
                                                         float* __restrict__ z, int* wd) {
   constexpr int kOpBytes = BLK * 128 * 2;  // one operand tile
   constexpr uint32_t kSBO = (BLK / 8) * 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* img = smem + 4 * kOpBytes;          // 32 KB staging of one h image
+  uint8_t* img = smem;  // 2 x 32 KB h images, after the MMAs are done with the operands
   __shared__ uint64_t bar;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
-  __shared__ float zred[4][128];
+  __shared__ float zred[16][2 * kD];
   const int bh = blockIdx.y, t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int j0 = 2 * blockIdx.x;
   const size_t base = (size_t)bh * N * 16;
@@ -76,7 +81,6 @@ __global__ void __launch_bounds__(128) linear_kv_kernel(const uint4* __restrict_
     mbar_fence_init();
   }
   if (warp == 0) tmem_alloc(&tmem_s, 256);
-  // Operands: thread t -> channel group cg = t%16 (8 channels), rows t/16 + 8r.
   const int cg = t & 15, r0 = t >> 4;
   float zacc[2][8];
 #pragma unroll
@@ -84,33 +88,38 @@ __global__ void __launch_bounds__(128) linear_kv_kernel(const uint4* __restrict_
 #pragma unroll
     for (int c = 0; c < 8; ++c) zacc[b][c] = 0.f;
 #pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    const int j = j0 + b;
-    uint8_t* A = smem + (2 * b) * kOpBytes;
-    uint8_t* B = smem + (2 * b + 1) * kOpBytes;
-    for (int r = r0; r < BLK; r += 8) {
-      const int n = j * BLK + r;
-      uint4 kk = make_uint4(0, 0, 0, 0), vv = kk;
-      const bool valid = j < nb && n < N;
-      if (valid) {
-        kk = __ldg(k + base + (size_t)n * 16 + cg);
-        vv = __ldg(v + base + (size_t)n * 16 + cg);
-      }
-      const uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};
-      uint32_t pw[4];
+  for (int rd = 0; rd < BLK / 64; ++rd) {
+    uint4 kk[2][4], vv[2][4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float f0 = valid ? phi(bf16_lo(kw[e])) : 0.f;
-        const float f1 = valid ? phi(bf16_hi(kw[e])) : 0.f;
-        zacc[b][2 * e] += f0;
-        zacc[b][2 * e + 1] += f1;
-        pw[e] = pack_bf16(f0, f1);
+    for (int b = 0; b < 2; ++b)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int row = 64 * rd + r0 + 16 * r, n = (j0 + b) * BLK + row;
+        const bool valid = j0 + b < nb && n < N;
+        kk[b][r] = valid ? __ldg(k + base + (size_t)n * 16 + cg) : make_uint4(0, 0, 0, 0);
+        vv[b][r] = valid ? __ldg(v + base + (size_t)n * 16 + cg) : make_uint4(0, 0, 0, 0);
       }
-      // MN-major core matrix: (m/8)*SBO + (tok/8)*128 + (tok%8)*16 + (m%8)*2
-      const uint32_t off = cg * kSBO + (r >> 3) * 128 + (r & 7) * 16;
-      *reinterpret_cast<uint4*>(A + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-      *reinterpret_cast<uint4*>(B + off) = vv;
-    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int row = 64 * rd + r0 + 16 * r, n = (j0 + b) * BLK + row;
+        const bool valid = j0 + b < nb && n < N;
+        const uint32_t kw[4] = {kk[b][r].x, kk[b][r].y, kk[b][r].z, kk[b][r].w};
+        uint32_t pw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float f0 = valid ? phi(bf16_lo(kw[e])) : 0.f;
+          const float f1 = valid ? phi(bf16_hi(kw[e])) : 0.f;
+          zacc[b][2 * e] += f0;
+          zacc[b][2 * e + 1] += f1;
+          pw[e] = pack_bf16(f0, f1);
+        }
+        // MN-major core matrix: (m/8)*SBO + (tok/8)*128 + (tok%8)*16 + (m%8)*2
+        const uint32_t off = cg * kSBO + (row >> 3) * 128 + (row & 7) * 16;
+        *reinterpret_cast<uint4*>(smem + (2 * b) * kOpBytes + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        *reinterpret_cast<uint4*>(smem + (2 * b + 1) * kOpBytes + off) = vv[b][r];
+      }
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -129,50 +138,45 @@ __global__ void __launch_bounds__(128) linear_kv_kernel(const uint4* __restrict_
     }
     mma_commit(&bar);
   }
-  // z_j: reduce the per-thread channel sums over the 8 row groups.
+  // z_j: the 16 row slots' channel sums, added in slot order.
 #pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    const int j = j0 + b;
-    __syncthreads();
-    if (r0 < 4) {
+  for (int b = 0; b < 2; ++b)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) zred[r0][cg * 8 + c] = zacc[b][c];
-    }
-    __syncthreads();
-    if (r0 >= 4) {
+    for (int c = 0; c < 8; ++c) zred[r0][b * kD + cg * 8 + c] = zacc[b][c];
+  __syncthreads();
+  {
+    const int b = t >> 7, c = t & 127;
+    float a = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) zred[r0 - 4][cg * 8 + c] += zacc[b][c];
-    }
-    __syncthreads();
-    if (j < nb) z[((size_t)bh * nb + j) * kD + t] = (zred[0][t] + zred[1][t]) + (zred[2][t] + zred[3][t]);
+    for (int r = 0; r < 16; ++r) a += zred[r][b * kD + c];
+    if (j0 + b < nb) z[((size_t)bh * nb + j0 + b) * kD + c] = a;
   }
   const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar, 0, &abort_s, wd));
   tc_fence_after();
-  // h_j rows: warp w holds ck = 32w + lane; columns cv.  Stage as the bf16
-  // image, then copy 16-byte chunks (8 image columns) to the mask-GEMM tiles.
-  uint4* out0 = nullptr;
-  (void)out0;
-#pragma unroll 1
-  for (int b = 0; b < 2; ++b) {
-    const int j = j0 + b;
-    const int ck = 32 * warp + lane;
+  // h_j rows: warp w holds ck = 32(w%4) + lane of block w/4; columns cv.
+  // Stage both bf16 images (the operands are dead once the MMAs completed).
+  {
+    const int b = warp >> 2, ck = 32 * (warp & 3) + lane;
+    uint8_t* im = img + b * 32768;
 #pragma unroll 1
     for (int c0 = 0; c0 < 128; c0 += 16) {
       uint32_t r[16];
-      SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * warp) << 16) + b * 128 + c0, r);
+      SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + b * 128 + c0, r);
       tmem_ld_wait();
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         const float val = ok ? __uint_as_float(r[e]) : 0.f;
-        *reinterpret_cast<__nv_bfloat16*>(img + himg_off(c0 + e, ck)) = __float2bfloat16_rn(val);
+        *reinterpret_cast<__nv_bfloat16*>(im + himg_off(c0 + e, ck)) = __float2bfloat16_rn(val);
       }
     }
-    __syncthreads();
-    // 2048 chunks of 16 bytes; block j's chunk goes next to block j^1's.
-    for (int c = t; c < 2048; c += 128)
-      *reinterpret_cast<uint4*>(hs + (size_t)bh * nbt * 64 * 16384 * 2 + hs_chunk(nbt, j, c)) =
-          *reinterpret_cast<const uint4*>(img + c * 16);
-    __syncthreads();
+  }
+  __syncthreads();
+  // 2048 chunk positions of 16 bytes; block 2x's chunk and block 2x+1's are
+  // adjacent in hs, so each thread writes 32 contiguous bytes per position.
+  for (int c = t; c < 2048; c += 256) {
+    uint8_t* dst = hs + (size_t)bh * nbt * 64 * 16384 * 2 + hs_chunk(nbt, j0, c);
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(img + c * 16);
+    *reinterpret_cast<uint4*>(dst + 16) = *reinterpret_cast<const uint4*>(img + 32768 + c * 16);
   }
   tc_fence_before();
   __syncthreads();
@@ -327,7 +331,8 @@ __global__ void __launch_bounds__(192, 1) linear_sum_kernel(const uint8_t* __res
 // Block 64: two query blocks per CTA whose M=64 accumulators share TMEM at
 // lane offsets 0 / 16 (all 128 threads hold a row); block 128: M = 128.
 // 128 threads; thread 0 issues the copies and MMAs.  TMEM: num (128 cols) and
-// y (128 cols).  Shared: H images, W image, phi(Q) (reused for O_l).
+// y (128 cols).  Shared: H images (the W image replaces them once num is
+// done, so two CTAs fit on an SM), phi(Q) (reused for O_l).
 template <int MODE>
 __global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __restrict__ q,
                                                            const uint8_t* __restrict__ himg,
@@ -338,10 +343,10 @@ __global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __res
   constexpr int nH = MODE == 0 ? 2 : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sH = smem;                       // nH x 32 KB
-  uint8_t* sW = smem + nH * kImg;           // 32 KB
-  uint8_t* sA = sW + kImg;                  // 32 KB: phi(Q), then O_l
-  __shared__ uint64_t bar_in, bar_n, bar_y;
+  uint8_t* sH = smem;                       // nH x 32 KB: H images, then the W image
+  uint8_t* sW = smem;                       // (W lands where H was once num is done)
+  uint8_t* sA = smem + nH * kImg;           // 32 KB: phi(Q), then O_l
+  __shared__ uint64_t bar_in, bar_n, bar_y, bar_w;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -353,6 +358,7 @@ __global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __res
     mbar_init(&bar_in, 1);
     mbar_init(&bar_n, 1);
     mbar_init(&bar_y, 1);
+    mbar_init(&bar_w, 1);
     abort_s = 0;
     mbar_fence_init();
   }
@@ -362,12 +368,11 @@ __global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __res
   tc_fence_after();
   const uint32_t tmem = tmem_s;
   if (t == 0) {
-    mbar_expect_tx(&bar_in, (nH + 1) * kImg);
+    mbar_expect_tx(&bar_in, nH * kImg);
     for (int x = 0; x < nH; ++x) {
       const int i = (x == 0 || !hasB) ? iA : iB;
       bulk_g2s(sH + x * kImg, himg + ((size_t)bh * nb + i) * kImg, kImg, &bar_in);
     }
-    bulk_g2s(sW, wimg, kImg, &bar_in);
   }
   // Row of this thread (same TMEM lane mapping as the flash kernel).
   int row, i;
@@ -427,6 +432,12 @@ __global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __res
   }
   bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_n, 0, &abort_s, wd));
   tc_fence_after();
+  // The MMAs are done reading H: bring the W image (L2-resident) into its
+  // place while num becomes O_l.
+  if (t == 0) {
+    mbar_expect_tx(&bar_w, kImg);
+    bulk_g2s(sW, wimg, kImg, &bar_w);
+  }
   const uint32_t lb = (uint32_t)(32 * warp) << 16;
   {
     const float inv_den = (store && den > 0.f) ? 1.f / den : 0.f;
@@ -449,7 +460,7 @@ __global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __res
   __syncthreads();
   if (t == 0) {
     tc_fence_after();
-    if (ok) {
+    if (ok && mbar_wait(&bar_w, 0, &abort_s, wd)) {
       for (int x = 0; x < nx; ++x) {
         const uint32_t d = tmem + 128 + ((uint32_t)(x * 16) << 16);
 #pragma unroll
@@ -478,13 +489,16 @@ __global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __res
     }
   }
   // The inputs' bulk copies must have landed before the CTA exits.
-  if (t == 0) mbar_wait_drain(&bar_in, 0, wd);
+  if (t == 0) {
+    mbar_wait_drain(&bar_in, 0, wd);
+    mbar_wait_drain(&bar_w, 0, wd);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
-int linear_apply_smem(int block) { return (block == 64 ? 4 : 3) * 32768 + 1024; }
+int linear_apply_smem(int block) { return (block == 64 ? 3 : 2) * 32768 + 1024; }
 
 cudaError_t launch_linear_apply(const void* q, const uint16_t* himg, const float* zl, const uint16_t* wimg,
                                 const Geom& g, void* out, int* wd, cudaStream_t st) {
@@ -511,7 +525,7 @@ __global__ void w_tile_kernel(const uint16_t* __restrict__ w, uint16_t* __restri
   wt[himg_off(co, ci) / 2] = w[co * kD + ci];
 }
 
-int linear_kv_smem(int block) { return 4 * block * 128 * 2 + 32768 + 1024; }
+int linear_kv_smem(int block) { return 4 * block * 128 * 2 + 1024; }
 int linear_sum_smem() { return kLStages * (kHsTile + kATile) + (int)sizeof(LBars) + 1024; }
 
 cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_t* hs, float* z, int* wd,
@@ -522,12 +536,12 @@ cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_
   if (g.block == 64) {
     e = cudaFuncSetAttribute(linear_kv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    linear_kv_kernel<64><<<dim3(nbt * 32, g.BH), 128, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt, hs,
+    linear_kv_kernel<64><<<dim3(nbt * 32, g.BH), 256, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt, hs,
                                                                   z, wd);
   } else {
     e = cudaFuncSetAttribute(linear_kv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    linear_kv_kernel<128><<<dim3(nbt * 32, g.BH), 128, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt,
+    linear_kv_kernel<128><<<dim3(nbt * 32, g.BH), 256, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt,
                                                                    hs, z, wd);
   }
   return cudaGetLastError();
