@@ -84,7 +84,10 @@ __global__ void stats_final_kernel(const double* __restrict__ psum, const float*
 
 // ---------------------------------------------------------------- K2 ----
 // grid (nq, BH), 128 threads: one 64-token tile of Q, K and V.
-// Thread t handles channel group cg = t%16 (8 channels) of rows t/16 + 8*i.
+// Thread t handles channel group cg = t/8 (8 channels) of rows t%8 + 8*i:
+// the lanes of a warp span 8 rows and 4 channel groups, which keeps the
+// stores into the tile images (whose channel groups lie 512 or 1024 bytes
+// apart, one bank) at most 4-way conflicted.
 __device__ __forceinline__ float block_max128(float x, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
@@ -95,11 +98,12 @@ __device__ __forceinline__ float block_max128(float x, float* red) {
   return r;
 }
 
-__device__ __forceinline__ int8_t i8code(float x, float mult) {
-  float p = __fmul_rn(x, mult);
-  int r = __float2int_rn(p);
-  r = max(-127, min(127, r));
-  return (int8_t)r;
+// rne(fl32(x * mult)) as a byte.  |x| <= amax and mult = fl32(127/amax), so
+// the product lies within 127 * (1 + 2^-23) and no clamp is needed; adding
+// 1.5 * 2^23 rounds it to the nearest integer (ties to even) in the low
+// mantissa bits, on the FMA pipe rather than the conversion unit.
+__device__ __forceinline__ uint32_t i8code(float x, float mult) {
+  return (uint32_t)__float_as_int(__fadd_rn(__fmul_rn(x, mult), 12582912.0f)) & 0xFFu;
 }
 
 __global__ void __launch_bounds__(128) quant_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
@@ -110,7 +114,7 @@ __global__ void __launch_bounds__(128) quant_kernel(const uint4* __restrict__ q,
                                                     float* __restrict__ sk, float* __restrict__ qsum,
                                                     float* __restrict__ ksum) {
   const int bh = blockIdx.y, tile = blockIdx.x, t = threadIdx.x;
-  const int cg = t & 15, rr = t >> 4;
+  const int cg = t >> 3, rr = t & 7;
   const int n0 = tile * kQB;
   __shared__ __align__(16) uint8_t sq8[kTile];
   __shared__ __align__(16) uint8_t sk8[kTile];
@@ -183,10 +187,10 @@ __global__ void __launch_bounds__(128) quant_kernel(const uint4* __restrict__ q,
     uint32_t qa = 0, qb = 0, ka = 0, kb = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      qa |= (uint32_t)(uint8_t)i8code(xq[i][j], mq) << (8 * j);
-      qb |= (uint32_t)(uint8_t)i8code(xq[i][j + 4], mq) << (8 * j);
-      ka |= (uint32_t)(uint8_t)i8code(xk[i][j], mk) << (8 * j);
-      kb |= (uint32_t)(uint8_t)i8code(xk[i][j + 4], mk) << (8 * j);
+      qa |= i8code(xq[i][j], mq) << (8 * j);
+      qb |= i8code(xq[i][j + 4], mq) << (8 * j);
+      ka |= i8code(xk[i][j], mk) << (8 * j);
+      kb |= i8code(xk[i][j + 4], mk) << (8 * j);
     }
     const uint32_t off = kmajor_off(r, cg * 8, kQK_LBO, kQK_SBO);
     *reinterpret_cast<uint2*>(sq8 + off) = make_uint2(qa, qb);
