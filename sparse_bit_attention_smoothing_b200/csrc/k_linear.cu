@@ -270,28 +270,22 @@ __global__ void __launch_bounds__(192, 1) linear_sum_kernel(const uint8_t* __res
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->empty[st], ((kt / kLStages) - 1) & 1, abort, wd));
         if (!ok) break;
       }
-      uint32_t w0 = 0, w1 = 0;
+      // ones = NOT selected and j < nb (and i < nb), as 64 bits
+      uint64_t ones = 0;
       if (i < nb) {
-        w0 = selbits[((size_t)bh * nb + i) * nbw + 2 * kt];
-        w1 = selbits[((size_t)bh * nb + i) * nbw + 2 * kt + 1];
+        const uint64_t w = (uint64_t)selbits[((size_t)bh * nb + i) * nbw + 2 * kt] |
+                           ((uint64_t)selbits[((size_t)bh * nb + i) * nbw + 2 * kt + 1] << 32);
+        const int left = nb - kt * 64;  // key blocks of this tile that exist
+        ones = ~w & (left >= 64 ? ~0ull : ((1ull << left) - 1ull));
       }
       uint8_t* A = sA + st * kATile;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {  // 8 keys per 16-byte chunk
+        const uint32_t b8 = (uint32_t)(ones >> (8 * ch)) & 0xFFu;
         uint32_t pk[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint32_t h2 = 0;
-#pragma unroll
-          for (int z2 = 0; z2 < 2; ++z2) {
-            const int jj = ch * 8 + e * 2 + z2;  // key block within the tile
-            const int j = kt * 64 + jj;
-            const uint32_t bit = jj < 32 ? (w0 >> jj) & 1u : (w1 >> (jj - 32)) & 1u;
-            const bool one = i < nb && j < nb && !bit;
-            h2 |= (one ? 0x3F80u : 0u) << (16 * z2);
-          }
-          pk[e] = h2;
-        }
+        for (int e = 0; e < 4; ++e)  // bf16 1.0 = 0x3F80 in each half whose bit is set
+          pk[e] = (((b8 >> (2 * e)) & 1u) * 0x3F80u) | (((b8 >> (2 * e + 1)) & 1u) * 0x3F800000u);
         *reinterpret_cast<uint4*>(A + kmajor_off(r, ch * 16, kQK_LBO, kQK_SBO)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       fence_proxy_async_smem();
