@@ -97,7 +97,12 @@ __global__ void __launch_bounds__(32 * TQ) pool_topk_kernel(const float* __restr
     const int r = e / kD;
     qb[e] = i0 + r < nb ? qh[(size_t)i0 * kD + e] : 0.f;
   }
-  // Phase 1: scores, fp32 FMA in channel order.
+  // Phase 1: scores, fp32 FMA.  With TQ = 8, thread t takes key t % 64 of the
+  // chunk and channel quarter t / 64 for all eight rows (a warp shares its
+  // quarter, so the query reads are broadcasts and each key value feeds
+  // eight FMAs); the four quarter sums are added in quarter order.  Other
+  // TQ: key t % 64, rows 2*(t/64) and 2*(t/64)+1, channels in order.
+  float* psc = sc + TQ * nb;  // [4][TQ][kKC] quarter sums (TQ == 8 only)
   const int jj = t & 63, qg = t >> 6;
   for (int j0 = 0; j0 < nb; j0 += kKC) {
     __syncthreads();
@@ -110,7 +115,33 @@ __global__ void __launch_bounds__(32 * TQ) pool_topk_kernel(const float* __restr
     }
     __syncthreads();
     const int j = j0 + jj;
-    if (j < nb) {
+    if (TQ == 8) {
+      float a[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) a[r] = 0.f;
+      const float* kr = kb + jj * kPad + 32 * qg;
+#pragma unroll
+      for (int c = 0; c < 32; c += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(kr + c);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const float4 x = *reinterpret_cast<const float4*>(qb + r * kD + 32 * qg + c);
+          a[r] = fmaf(x.x, k4.x, a[r]);
+          a[r] = fmaf(x.y, k4.y, a[r]);
+          a[r] = fmaf(x.z, k4.z, a[r]);
+          a[r] = fmaf(x.w, k4.w, a[r]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r) psc[(qg * 8 + r) * kKC + jj] = a[r];
+      __syncthreads();
+      for (int e = t; e < 8 * kKC; e += kThr) {
+        const int r = e / kKC, k = e % kKC, jk = j0 + k;
+        if (jk < nb)
+          sc[r * nb + jk] = ((psc[(0 * 8 + r) * kKC + k] + psc[(1 * 8 + r) * kKC + k]) +
+                             (psc[(2 * 8 + r) * kKC + k] + psc[(3 * 8 + r) * kKC + k])) * rs;
+      }
+    } else if (j < nb) {
       float a0 = 0.f, a1 = 0.f;
       const float* kr = kb + jj * kPad;
       const float* q0 = qb + (2 * qg) * kD;
@@ -226,7 +257,9 @@ __global__ void __launch_bounds__(32 * TQ) pool_topk_kernel(const float* __restr
 
 namespace {
 
-size_t topk_smem(int tq, int nb) { return sizeof(float) * ((size_t)tq * kD + (size_t)kKC * kPad + (size_t)tq * nb); }
+size_t topk_smem(int tq, int nb) {
+  return sizeof(float) * ((size_t)tq * kD + (size_t)kKC * kPad + (size_t)tq * nb + (tq == 8 ? 4 * 8 * kKC : 0));
+}
 
 template <int TQ, int PER>
 cudaError_t launch_topk_cfg(const float* qbar, const float* kbar, const Geom& g, int32_t* idx, const float* zin,
