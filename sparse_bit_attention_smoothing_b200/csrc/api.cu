@@ -320,12 +320,40 @@ int dense_int8_attn(const void* q, const void* k, const void* v, void* out, int 
   return run_attn(q, k, v, nullptr, out, B, H, N, d, 64, 1.0f, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Copy streams of the host-buffer entry point, one pair per device (created
+// once, never destroyed: they live as long as the process).
+struct CopyStreams {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+};
+
+int copy_streams(int dev, CopyStreams* out) {
+  static std::mutex cmu;
+  static std::map<int, CopyStreams> cs;
+  std::lock_guard<std::mutex> lk(cmu);
+  CopyStreams& c = cs[dev];
+  if (!c.h2d) {
+    if (cudaStreamCreateWithFlags(&c.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&c.d2h, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaGetLastError();
+      return SAGESLA_ERR_LAUNCH;
+    }
+  }
+  *out = c;
+  return SAGESLA_OK;
+}
+
+// The heads are independent problems, so the host-buffer call runs in chunks
+// of heads as a three-stage pipeline: host->device copies of chunk c+1 (copy
+// stream), the path on chunk c (the caller's stream) and device->host copies
+// of chunk c-1 (a second copy stream) overlap.
 int sagesla_attn_host(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B, int H,
                       int N, int d, int block, float topk, sagesla_stream_t stream) {
   SAGESLA_TRY(validate(q, k, v, out, B, H, N, d, block, topk));
   int dev = 0;
   SAGESLA_TRY(check_device(&dev));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  CopyStreams cs;
+  SAGESLA_TRY(copy_streams(dev, &cs));
   const size_t E = (size_t)B * H * N * d * 2;  // bytes of one bf16 tensor
   const size_t W = (size_t)d * d * 2;
   // Device staging lives in its own cached region, keyed by a distinct stream tag.
@@ -353,14 +381,57 @@ int sagesla_attn_host(const void* q, const void* k, const void* v, const void* p
   uint8_t* dv = dk + up(E);
   uint8_t* dout = dv + up(E);
   uint8_t* dw = dout + up(E);
-  if (cudaMemcpyAsync(dq, q, E, cudaMemcpyHostToDevice, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
-  if (cudaMemcpyAsync(dk, k, E, cudaMemcpyHostToDevice, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
-  if (cudaMemcpyAsync(dv, v, E, cudaMemcpyHostToDevice, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
-  if (proj_w && cudaMemcpyAsync(dw, proj_w, W, cudaMemcpyHostToDevice, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
-  SAGESLA_TRY(run_attn(dq, dk, dv, proj_w ? dw : nullptr, dout, B, H, N, d, block, topk, st));
-  if (cudaMemcpyAsync(out, dout, E, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
-  return SAGESLA_OK;
+  const uint8_t* hq = static_cast<const uint8_t*>(q);
+  const uint8_t* hk = static_cast<const uint8_t*>(k);
+  const uint8_t* hv = static_cast<const uint8_t*>(v);
+  uint8_t* hout = static_cast<uint8_t*>(out);
+  const int BH = B * H;
+  const int nchunk = BH < 20 ? BH : 20;
+  const int per = (BH + nchunk - 1) / nchunk;  // heads per chunk (the last may have fewer)
+  const size_t head_bytes = (size_t)N * d * 2;
+  std::vector<cudaEvent_t> ev(2 * nchunk + 1, nullptr);
+  auto cleanup = [&]() {
+    for (cudaEvent_t e : ev)
+      if (e) cudaEventDestroy(e);
+  };
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      cleanup();
+      return SAGESLA_ERR_LAUNCH;
+    }
+  int rc = SAGESLA_OK;
+  // The staging buffers may still be read by work queued earlier on `st`.
+  if (cudaEventRecord(ev[2 * nchunk], st) != cudaSuccess || cudaStreamWaitEvent(cs.h2d, ev[2 * nchunk], 0) != cudaSuccess)
+    rc = SAGESLA_ERR_LAUNCH;
+  if (rc == SAGESLA_OK && proj_w && cudaMemcpyAsync(dw, proj_w, W, cudaMemcpyHostToDevice, cs.h2d) != cudaSuccess)
+    rc = SAGESLA_ERR_LAUNCH;
+  for (int c = 0; rc == SAGESLA_OK && c < nchunk; ++c) {
+    const int h0 = c * per, hn = (h0 + per <= BH ? per : BH - h0);
+    if (hn <= 0) break;
+    const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)hn * head_bytes;
+    if (cudaMemcpyAsync(dq + off, hq + off, bytes, cudaMemcpyHostToDevice, cs.h2d) != cudaSuccess ||
+        cudaMemcpyAsync(dk + off, hk + off, bytes, cudaMemcpyHostToDevice, cs.h2d) != cudaSuccess ||
+        cudaMemcpyAsync(dv + off, hv + off, bytes, cudaMemcpyHostToDevice, cs.h2d) != cudaSuccess ||
+        cudaEventRecord(ev[c], cs.h2d) != cudaSuccess || cudaStreamWaitEvent(st, ev[c], 0) != cudaSuccess) {
+      rc = SAGESLA_ERR_LAUNCH;
+      break;
+    }
+    rc = run_attn(dq + off, dk + off, dv + off, proj_w ? dw : nullptr, dout + off, 1, hn, N, d, block, topk, st);
+    if (rc != SAGESLA_OK) break;
+    if (cudaEventRecord(ev[nchunk + c], st) != cudaSuccess || cudaStreamWaitEvent(cs.d2h, ev[nchunk + c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(hout + off, dout + off, bytes, cudaMemcpyDeviceToHost, cs.d2h) != cudaSuccess) {
+      rc = SAGESLA_ERR_LAUNCH;
+      break;
+    }
+  }
+  // Every queued copy and kernel must be finished before the caller's host
+  // buffers are released (also on an error path).
+  if (cudaStreamSynchronize(cs.h2d) != cudaSuccess) rc = SAGESLA_ERR_LAUNCH;
+  if (cudaStreamSynchronize(st) != cudaSuccess) rc = SAGESLA_ERR_LAUNCH;
+  if (cudaStreamSynchronize(cs.d2h) != cudaSuccess) rc = SAGESLA_ERR_LAUNCH;
+  cleanup();
+  return rc;
 }
 
 int sagesla_get_quant(const void* q, const void* k, const void* v, int B, int H, int N, int d, int8_t* q8,

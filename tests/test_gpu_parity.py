@@ -167,3 +167,20 @@ def test_linear_branch_topk_one_contributes_nothing(sg):
     b = sg.dense_int8_attn(dq, dk, dv)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_host_entry_point_matches_device_path(sg):
+    """sagesla_attn_host runs in chunks of heads on three streams (copies in,
+    path, copies out overlapped); heads are independent, so the result is the
+    device entry point's, bit for bit (9 heads: one per chunk, and 23 heads:
+    chunks of 2 with a ragged last one)."""
+    for H in (9, 23):
+        q, k, v, w = _inputs(1, H, 777, True, seed=5)
+        dq, dk, dv, dw = _dev(q, k, v, w)
+        ref = sg.sagesla_attn(dq, dk, dv, dw, block=64, topk=0.2)
+        torch.cuda.synchronize()
+        hq, hk, hv, hw = (t.pin_memory() for t in (q, k, v, w))
+        hout = torch.empty_like(hq).pin_memory()
+        sg.sagesla_attn_host(hq, hk, hv, hw, out=hout, block=64, topk=0.2)
+        assert sg.sync_status() == 0
+        assert torch.equal(hout, ref.cpu())
