@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of the SageSLA attention path on B200.
 
-python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME|all]
 
 One step = one sagesla_attn call over the whole workload (every kernel of the
 path: statistics, quantisation, pooled top-k mask, linear branch, sparse
@@ -9,7 +9,11 @@ flash).  Default workload: Wan2.1-14B-720P-shaped self-attention, B=1, H=40,
 N=75600, d=128, block 64, topk 0.1, seeded synthetic bf16 inputs (2.3 GB, far
 larger than L2, so no flush is needed between steps).  Prints one JSON line.
 Under torchrun every rank runs its own replica of the workload (independent
-problems, no collective on the data path): weak scaling.
+problems, no collective on the data path): weak scaling.  `--workload all`
+(one GPU) prints one shorter line per benchmark configuration instead: the
+five configurations (tiny, 1.3B-480P, 14B-480P, 14B-720P at topk 0.1 and
+0.05) and the sparsity sweep at 720p (block 64 and 128, topk 0.05 / 0.1 /
+0.15, dense with the linear branch off).
 """
 from __future__ import annotations
 
@@ -156,6 +160,57 @@ def cpu_baseline(w, q, k, v, pw, heads: int = 8, qblocks: int = 4) -> dict:
                 sample_seconds=t_fixed + t_sample)
 
 
+def run_all(args):
+    """One line per benchmark configuration (kernel-only timing, one GPU)."""
+    import torch
+    from sparse_bit_attention_smoothing_b200 import build as sbuild
+    sbuild.build()
+    import sparse_bit_attention_smoothing_b200 as sg
+    from sparse_bit_attention_smoothing_b200.inputs import make_inputs
+    st = torch.cuda.current_stream()
+    pk = peaks()
+    peak8 = 2.0 * pk["bf16"]
+    cache = {}
+    for w in workloads().values():
+        key = (w.B, w.H, w.N, w.d, w.outliers)
+        if key not in cache:
+            cache.clear()
+            q, k, v, pw = make_inputs(w.B, w.H, w.N, w.d, seed=0, outliers=w.outliers)
+            cache[key] = (q.cuda(), k.cuda(), v.cuda(), pw.cuda())
+        dq, dk, dv, dw = cache[key]
+        dw = dw if w.linear else None
+        out = torch.empty_like(dq)
+        for _ in range(max(3, args.warmup)):
+            sg.sagesla_attn(dq, dk, dv, dw, out=out, block=w.block, topk=w.topk, stream=st)
+        torch.cuda.synchronize()
+        sg.profile(True)
+        sg.profile_read()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(args.steps):
+            sg.sagesla_attn(dq, dk, dv, dw, out=out, block=w.block, topk=w.topk, stream=st)
+        e1.record(st)
+        torch.cuda.synchronize()
+        prof = sg.profile_read()
+        sg.profile(False)
+        ms = e0.elapsed_time(e1) / args.steps
+        f = flops(w)
+        fl_ms, fl_n = prof.get("flash", (0.0, 0))
+        flash_ms = fl_ms / max(1, fl_n)
+        achieved = f["computed"] / (flash_ms * 1e-3) / 1e12 if flash_ms > 0 else None
+        t_roof = max(f["computed"] / (peak8 * 1e12), f["hbm_bytes"] / (pk["hbm"] * 1e9))
+        line = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "block": w.block, "topk": w.topk,
+                "linear": w.linear, "k_blocks": f["kc"], "ms_per_call": ms,
+                "dense_equiv_tflops": f["dense"] / (ms * 1e-3) / 1e12,
+                "flash_ms": flash_ms, "flash_tflops": achieved,
+                "flash_frac_of_8bit_peak": (achieved / peak8) if achieved else None,
+                "path_frac_of_roofline": t_roof * 1e3 / ms, "device_status": sg.sync_status(),
+                "kernels_ms": {kname: round(t / max(1, n), 4) for kname, (t, n) in prof.items()}}
+        print(json.dumps(line), flush=True)
+        del out
+    return 0
+
+
 def run_reference(args):
     rank = _env_int("RANK", 0)
     if rank != 0:
@@ -195,6 +250,8 @@ def main():
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "all":
+        return run_all(args)
 
     import torch
     import torch.distributed as dist
