@@ -91,8 +91,14 @@ int dense_int8_attn(const void* q, const void* k, const void* v, void* out, int 
 /*
  * sagesla_attn_host: sagesla_attn on HOST buffers (pinned memory gives
  * asynchronous copies).  Copies q, k, v (and proj_w) to the device, runs the
- * path, copies out back and synchronises `stream` before returning.  Same
- * shapes and codes as sagesla_attn; proj_w may be NULL.
+ * path, copies out back and synchronises before returning.  The B*H heads are
+ * independent problems, so the call runs in up to 20 chunks of heads as a
+ * pipeline: host->device copies of the next chunk and device->host copies of
+ * the previous one (on two copy streams the library creates once per device)
+ * overlap the path on the current chunk (on `stream`).  The result is
+ * bit-identical to sagesla_attn.  Same shapes and codes as sagesla_attn;
+ * proj_w may be NULL.  The device staging (4 x B*H*N*d bf16 + d*d) is cached
+ * per (device, stream) until sagesla_release.
  */
 int sagesla_attn_host(const void* q, const void* k, const void* v, const void* proj_w, void* out,
                       int B, int H, int N, int d, int block, float topk, sagesla_stream_t stream);

@@ -28,7 +28,8 @@ struct Workspace {
   size_t bytes = 0;
 };
 std::mutex g_mu;
-std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;     // path workspace
+std::map<std::pair<int, cudaStream_t>, Workspace> g_stage;  // host entry point's device staging
 std::map<int, int*> g_wd;        // per-device watchdog word
 std::map<int, int> g_dev_ok;     // per-device: 1 = sm_100, 0 = not
 
@@ -356,13 +357,11 @@ int sagesla_attn_host(const void* q, const void* k, const void* v, const void* p
   SAGESLA_TRY(copy_streams(dev, &cs));
   const size_t E = (size_t)B * H * N * d * 2;  // bytes of one bf16 tensor
   const size_t W = (size_t)d * d * 2;
-  // Device staging lives in its own cached region, keyed by a distinct stream tag.
-  static std::mutex smu;
-  static std::map<std::pair<int, cudaStream_t>, Workspace> stage;
+  // Device staging lives in its own cached region per (device, stream).
   uint8_t* base = nullptr;
   {
-    std::lock_guard<std::mutex> lk(smu);
-    Workspace& w = stage[std::make_pair(dev, st)];
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace& w = g_stage[std::make_pair(dev, st)];
     const size_t need = 4 * up(E) + up(W);
     if (w.bytes < need) {
       if (w.ptr) cudaFreeAsync(w.ptr, st);
@@ -543,6 +542,9 @@ void sagesla_release(void) {
   for (auto& kv : g_ws)
     if (kv.second.ptr) cudaFree(kv.second.ptr);
   g_ws.clear();
+  for (auto& kv : g_stage)
+    if (kv.second.ptr) cudaFree(kv.second.ptr);
+  g_stage.clear();
 }
 
 }  // extern "C"
