@@ -34,7 +34,8 @@ __global__ void __launch_bounds__(128) stats_partial_kernel(const uint4* __restr
     m[i] = 0.f;
   }
   const size_t base = (size_t)bh * N * 16;  // in uint4 (8 bf16) units
-  for (int n = n_begin + r0; n < n_end; n += 8) {
+#pragma unroll 4
+  for (int n = n_begin + r0; n < n_end; n += 8) {  // unrolled: four row pairs of loads in flight
     uint4 kk = __ldg(k + base + (size_t)n * 16 + cg);
     uint4 vv = __ldg(v + base + (size_t)n * 16 + cg);
     uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};

@@ -186,8 +186,10 @@ __global__ void __launch_bounds__(32 * TQ) pool_topk_kernel(const float* __restr
     const uint32_t cand = T | (1u << b);
     int cnt = 0;
     if (PER > 0) {
+      int c4[4] = {0, 0, 0, 0};  // four independent counters: short dependency chains
 #pragma unroll
-      for (int u = 0; u < PER; ++u) cnt += keys[u] >= cand ? 1 : 0;
+      for (int u = 0; u < PER; ++u) c4[u & 3] += keys[u] >= cand ? 1 : 0;
+      cnt = (c4[0] + c4[1]) + (c4[2] + c4[3]);
     } else {
       for (int j = lane; j < nb; j += 32) cnt += order_key(row[j]) >= cand ? 1 : 0;
     }
