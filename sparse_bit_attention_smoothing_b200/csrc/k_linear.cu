@@ -51,75 +51,69 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }  // namespace
 
 // ---------------------------------------------------------------- K4a ----
-// grid (nbt*32, BH): CTA x handles key blocks j = 2x, 2x+1 (zeros past nb),
-// so both 16-byte halves of every 32-byte sector of the h tiles come from one
-// CTA.  256 threads; thread t owns channels 8*(t%16).. and token rows t/16 +
-// 16r of 64-row rounds: all its K and V loads of a round are issued before
-// any is used (64 KB in flight per CTA, two CTAs per SM).  Thread 0 issues
-// the MMAs.  Dynamic smem: per block, A (phi(K) rows) and B (V rows)
-// MN-major, BLK x 128 bf16 each; after the MMAs the same bytes stage the two
-// bf16 h images.
+// grid (nbt*64, BH): CTA x handles key block j = x (zeros past nb, so the
+// mask-GEMM tiles hold no garbage).  256 threads; thread t owns channels
+// 8*(t%16).. and token rows t/16 + 16r of 64-row rounds: all its K and V
+// loads of a round are issued before any is used.  Small CTAs (128 TMEM
+// columns, ~40 KB of shared memory) so that four share an SM and their load
+// phases overlap each other's compute.  Thread 0 issues the MMAs.  Dynamic
+// smem: A (phi(K) rows) and B (V rows) MN-major, BLK x 128 bf16 each; after
+// the MMAs the same bytes stage the bf16 h image.
 template <int BLK>
-__global__ void __launch_bounds__(256) linear_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int N,
-                                                        int nb, int nbt, uint8_t* __restrict__ hs,
-                                                        float* __restrict__ z, int* wd) {
+__global__ void __launch_bounds__(256, 4) linear_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                                           int N, int nb, int nbt, uint8_t* __restrict__ hs,
+                                                           float* __restrict__ z, int* wd) {
   constexpr int kOpBytes = BLK * 128 * 2;  // one operand tile
   constexpr uint32_t kSBO = (BLK / 8) * 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* img = smem;  // 2 x 32 KB h images, after the MMAs are done with the operands
+  uint8_t* img = smem;  // 32 KB h image, after the MMAs are done with the operands
   __shared__ uint64_t bar;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
-  __shared__ float zred[16][2 * kD];
+  __shared__ float zred[16][kD];
   const int bh = blockIdx.y, t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int j0 = 2 * blockIdx.x;
+  const int j = blockIdx.x;
   const size_t base = (size_t)bh * N * 16;
   if (t == 0) {
     mbar_init(&bar, 1);
     abort_s = 0;
     mbar_fence_init();
   }
-  if (warp == 0) tmem_alloc(&tmem_s, 256);
+  if (warp == 0) tmem_alloc(&tmem_s, 128);
   const int cg = t & 15, r0 = t >> 4;
-  float zacc[2][8];
+  float zacc[8];
 #pragma unroll
-  for (int b = 0; b < 2; ++b)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) zacc[b][c] = 0.f;
+  for (int c = 0; c < 8; ++c) zacc[c] = 0.f;
 #pragma unroll
   for (int rd = 0; rd < BLK / 64; ++rd) {
-    uint4 kk[2][4], vv[2][4];
+    uint4 kk[4], vv[4];
 #pragma unroll
-    for (int b = 0; b < 2; ++b)
+    for (int r = 0; r < 4; ++r) {
+      const int row = 64 * rd + r0 + 16 * r, n = j * BLK + row;
+      const bool valid = j < nb && n < N;
+      kk[r] = valid ? __ldg(k + base + (size_t)n * 16 + cg) : make_uint4(0, 0, 0, 0);
+      vv[r] = valid ? __ldg(v + base + (size_t)n * 16 + cg) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int row = 64 * rd + r0 + 16 * r, n = (j0 + b) * BLK + row;
-        const bool valid = j0 + b < nb && n < N;
-        kk[b][r] = valid ? __ldg(k + base + (size_t)n * 16 + cg) : make_uint4(0, 0, 0, 0);
-        vv[b][r] = valid ? __ldg(v + base + (size_t)n * 16 + cg) : make_uint4(0, 0, 0, 0);
+    for (int r = 0; r < 4; ++r) {
+      const int row = 64 * rd + r0 + 16 * r, n = j * BLK + row;
+      const bool valid = j < nb && n < N;
+      const uint32_t kw[4] = {kk[r].x, kk[r].y, kk[r].z, kk[r].w};
+      uint32_t pw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float f0 = valid ? phi(bf16_lo(kw[e])) : 0.f;
+        const float f1 = valid ? phi(bf16_hi(kw[e])) : 0.f;
+        zacc[2 * e] += f0;
+        zacc[2 * e + 1] += f1;
+        pw[e] = pack_bf16(f0, f1);
       }
-#pragma unroll
-    for (int b = 0; b < 2; ++b)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int row = 64 * rd + r0 + 16 * r, n = (j0 + b) * BLK + row;
-        const bool valid = j0 + b < nb && n < N;
-        const uint32_t kw[4] = {kk[b][r].x, kk[b][r].y, kk[b][r].z, kk[b][r].w};
-        uint32_t pw[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float f0 = valid ? phi(bf16_lo(kw[e])) : 0.f;
-          const float f1 = valid ? phi(bf16_hi(kw[e])) : 0.f;
-          zacc[b][2 * e] += f0;
-          zacc[b][2 * e + 1] += f1;
-          pw[e] = pack_bf16(f0, f1);
-        }
-        // MN-major core matrix: (m/8)*SBO + (tok/8)*128 + (tok%8)*16 + (m%8)*2
-        const uint32_t off = cg * kSBO + (row >> 3) * 128 + (row & 7) * 16;
-        *reinterpret_cast<uint4*>(smem + (2 * b) * kOpBytes + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-        *reinterpret_cast<uint4*>(smem + (2 * b + 1) * kOpBytes + off) = vv[b][r];
-      }
+      // MN-major core matrix: (m/8)*SBO + (tok/8)*128 + (tok%8)*16 + (m%8)*2
+      const uint32_t off = cg * kSBO + (row >> 3) * 128 + (row & 7) * 16;
+      *reinterpret_cast<uint4*>(smem + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+      *reinterpret_cast<uint4*>(smem + kOpBytes + off) = vv[r];
+    }
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -129,58 +123,47 @@ __global__ void __launch_bounds__(256) linear_kv_kernel(const uint4* __restrict_
   if (t == 0) {
     const uint32_t id = idesc_bf16(128, 128, 1) | (1u << 15);  // A and B MN-major
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      const uint8_t* A = smem + (2 * b) * kOpBytes;
-      const uint8_t* B = smem + (2 * b + 1) * kOpBytes;
-#pragma unroll
-      for (int ks = 0; ks < BLK / 16; ++ks)
-        mma_bf16(tmem + b * 128, smem_desc(A + ks * 256, 128, kSBO), smem_desc(B + ks * 256, 128, kSBO), id, ks > 0);
-    }
+    for (int ks = 0; ks < BLK / 16; ++ks)
+      mma_bf16(tmem, smem_desc(smem + ks * 256, 128, kSBO), smem_desc(smem + kOpBytes + ks * 256, 128, kSBO), id,
+               ks > 0);
     mma_commit(&bar);
   }
   // z_j: the 16 row slots' channel sums, added in slot order.
 #pragma unroll
-  for (int b = 0; b < 2; ++b)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) zred[r0][b * kD + cg * 8 + c] = zacc[b][c];
+  for (int c = 0; c < 8; ++c) zred[r0][cg * 8 + c] = zacc[c];
   __syncthreads();
-  {
-    const int b = t >> 7, c = t & 127;
+  if (t < kD) {
     float a = 0.f;
 #pragma unroll
-    for (int r = 0; r < 16; ++r) a += zred[r][b * kD + c];
-    if (j0 + b < nb) z[((size_t)bh * nb + j0 + b) * kD + c] = a;
+    for (int r = 0; r < 16; ++r) a += zred[r][t];
+    if (j < nb) z[((size_t)bh * nb + j) * kD + t] = a;
   }
   const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar, 0, &abort_s, wd));
   tc_fence_after();
-  // h_j rows: warp w holds ck = 32(w%4) + lane of block w/4; columns cv.
-  // Stage both bf16 images (the operands are dead once the MMAs completed).
+  // h_j rows: warp w holds ck = 32(w%4) + lane, columns cv in [64(w/4), +64).
+  // Stage the bf16 image (the operands are dead once the MMAs completed).
   {
-    const int b = warp >> 2, ck = 32 * (warp & 3) + lane;
-    uint8_t* im = img + b * 32768;
+    const int ck = 32 * (warp & 3) + lane, cb = 64 * (warp >> 2);
 #pragma unroll 1
-    for (int c0 = 0; c0 < 128; c0 += 16) {
+    for (int c0 = cb; c0 < cb + 64; c0 += 16) {
       uint32_t r[16];
-      SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + b * 128 + c0, r);
+      SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0, r);
       tmem_ld_wait();
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         const float val = ok ? __uint_as_float(r[e]) : 0.f;
-        *reinterpret_cast<__nv_bfloat16*>(im + himg_off(c0 + e, ck)) = __float2bfloat16_rn(val);
+        *reinterpret_cast<__nv_bfloat16*>(img + himg_off(c0 + e, ck)) = __float2bfloat16_rn(val);
       }
     }
   }
   __syncthreads();
-  // 2048 chunk positions of 16 bytes; block 2x's chunk and block 2x+1's are
-  // adjacent in hs, so each thread writes 32 contiguous bytes per position.
-  for (int c = t; c < 2048; c += 256) {
-    uint8_t* dst = hs + (size_t)bh * nbt * 64 * 16384 * 2 + hs_chunk(nbt, j0, c);
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(img + c * 16);
-    *reinterpret_cast<uint4*>(dst + 16) = *reinterpret_cast<const uint4*>(img + 32768 + c * 16);
-  }
+  // 2048 chunks of 16 bytes into the mask-GEMM tiles.
+  for (int c = t; c < 2048; c += 256)
+    *reinterpret_cast<uint4*>(hs + (size_t)bh * nbt * 64 * 16384 * 2 + hs_chunk(nbt, j, c)) =
+        *reinterpret_cast<const uint4*>(img + c * 16);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
 // ---------------------------------------------------------------- K4b ----
@@ -519,7 +502,7 @@ __global__ void w_tile_kernel(const uint16_t* __restrict__ w, uint16_t* __restri
   wt[himg_off(co, ci) / 2] = w[co * kD + ci];
 }
 
-int linear_kv_smem(int block) { return 4 * block * 128 * 2 + 1024; }
+int linear_kv_smem(int block) { return 2 * block * 128 * 2 + 1024; }
 int linear_sum_smem() { return kLStages * (kHsTile + kATile) + (int)sizeof(LBars) + 1024; }
 
 cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_t* hs, float* z, int* wd,
@@ -530,12 +513,12 @@ cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_
   if (g.block == 64) {
     e = cudaFuncSetAttribute(linear_kv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    linear_kv_kernel<64><<<dim3(nbt * 32, g.BH), 256, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt, hs,
+    linear_kv_kernel<64><<<dim3(nbt * 64, g.BH), 256, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt, hs,
                                                                   z, wd);
   } else {
     e = cudaFuncSetAttribute(linear_kv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    linear_kv_kernel<128><<<dim3(nbt * 32, g.BH), 256, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt,
+    linear_kv_kernel<128><<<dim3(nbt * 64, g.BH), 256, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt,
                                                                    hs, z, wd);
   }
   return cudaGetLastError();
