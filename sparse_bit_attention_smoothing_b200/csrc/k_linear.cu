@@ -1,4 +1,4 @@
-// k_linear.cu -- the SLA linear-attention branch, part 1 and 2.
+// k_linear.cu -- the SLA linear-attention branch.
 //
 // "揭秘TurboDiffusion：如何让视频生成实现百倍加速？" 支柱二 SLA and
 // "TurboDiffusion跨模态" 2.2: besides the exactly computed blocks, a light
@@ -8,14 +8,16 @@
 //   h_j = phi(K_j)^T V_j  (d x d),  z_j = sum of the rows of phi(K_j)
 //   H_i = sum_{j not in S_i} h_j   (a 0/1 complement-mask GEMM per head)
 //
-// K4a linear_kv:  per pair of key blocks, h_j on tcgen05 (kind::f16, both
-//   operands MN-major straight from the token-major rows), fp32 accumulate,
-//   stored in bf16 as the B tiles of the mask GEMM; z_j in fp32.
+// K4a linear_kv:  per key block, h_j on tcgen05 (kind::f16, both operands
+//   MN-major, staged from the token-major rows), fp32 accumulate, stored in
+//   bf16 as the B tiles of the mask GEMM; z_j in fp32.
 // K4b linear_sum: per head, H = (1 - M) . Hstack with tcgen05 (M=128 query
 //   blocks x N=256 columns of the d*d matrices, K = key blocks); the 0/1 A
 //   tiles are expanded in shared memory from the selection bitmask.  Each
-//   output row is the bf16 image of H_i^T in the operand layout the flash
-//   kernel's epilogue MMA reads (so it is one bulk copy there).
+//   output row is the bf16 image of H_i^T in the operand layout the
+//   linear_apply kernel's MMA reads (one bulk copy there).
+// K4c linear_apply: y = (phi(Q) H_i / phi(Q) Z_i) W^T into `out`, to which
+//   the flash kernel adds the sparse output.
 #include "common.cuh"
 #include "kernels.h"
 
