@@ -148,10 +148,11 @@ Geom make_geom(int B, int H, int N, int block, float topk) {
   g.nb = (N + block - 1) / block;
   g.nq = 2 * ((N + 127) / 128);
   g.kc = sagesla_topk_count(g.nb, topk);
-  // Row splits for the statistics pass: about 4 CTAs per SM over the grid.
-  int split = (592 + g.BH - 1) / g.BH;
-  const int max_split = (N + 63) / 64;
-  g.split = split < 1 ? 1 : (split > max_split ? max_split : split);
+  // Row splits of the statistics pass: one per 1024 tokens.  The split
+  // depends on N alone, so the fp64 partial sums of the K mean are added in
+  // the same order whatever B*H a call covers (the host entry point's chunks
+  // of heads give the same bits as one call over all heads).
+  g.split = (N + 1023) / 1024;
   return g;
 }
 

@@ -61,14 +61,12 @@ extern "C" int sagesla_smooth_stats_noalloc(const void* k, const void* v, int B,
   if (B < 1 || H < 1 || N < 1 || d != sagesla::kD) return SAGESLA_ERR_INVALID;
   const long long BH = (long long)B * H;
   if (BH > 65535 || (double)BH * N * d >= 1099511627776.0) return SAGESLA_ERR_INVALID;
-  // Same row split as the regular path (about 4 CTAs per SM), reduced if the
-  // partial sums would not fit the scratch; one split per head at minimum.
+  // Same row split as the regular path (one per 1024 tokens, so the same
+  // fp64 summation order and the same bits), reduced only if the partial sums
+  // would not fit the scratch; one split per head at minimum.
   const size_t room = kNoAllocScratchBytes - (size_t)BH * kPerHeadBytes;
   if ((size_t)BH * kPerHeadBytes + (size_t)BH * kPerSplitBytes > kNoAllocScratchBytes) return SAGESLA_ERR_INVALID;
-  int split = (int)((592 + BH - 1) / BH);
-  const int max_split = (N + 63) / 64;
-  if (split > max_split) split = max_split;
-  if (split < 1) split = 1;
+  int split = (N + 1023) / 1024;
   const int fit = (int)(room / ((size_t)BH * kPerSplitBytes));
   if (split > fit) split = fit;
   if ((reinterpret_cast<uintptr_t>(k) & 15u) || (reinterpret_cast<uintptr_t>(v) & 15u) ||
