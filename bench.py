@@ -312,7 +312,10 @@ def main():
     fl_ms, fl_n = prof.get("flash", (0.0, 0))
     flash_ms = fl_ms / max(1, fl_n)
     achieved = f["computed"] / (flash_ms * 1e-3) / 1e12 if flash_ms > 0 else None
-    launches = sum(n for _, n in prof.values())
+    # profiler scopes -> kernels: the top-k scope launches pool_means, z_total
+    # (linear branch on) and pool_topk; every other scope one kernel
+    per_scope = {"pool_topk": 3 if (w.linear and pw is not None) else 2}
+    launches = sum(n * per_scope.get(kname, 1) for kname, (_, n) in prof.items())
     t_roof = max(f["computed"] / (peak8 * 1e12), f["hbm_bytes"] / (pk["hbm"] * 1e9))
 
     # end to end through the host-buffer entry point (pinned memory)
