@@ -169,13 +169,17 @@ __global__ void __launch_bounds__(256, 4) linear_kv_kernel(const uint4* __restri
 }
 
 // ---------------------------------------------------------------- K4b ----
-// grid (64 n-tiles, ceil(nb/128) i-tiles, BH).  192 threads: warp 0 bulk
-// loads the B tiles, warp 1 issues MMAs, warps 2-5 expand the 0/1 A tiles
-// from the selection bitmask and run the epilogue.  K tiles of 64 key
-// blocks, 2-stage ring; D = 128 x 256 fp32 in TMEM.
+// grid (ceil(nb/256), 64 n-tiles, BH): the CTAs that read the same B tiles
+// are neighbours in launch order.  A CTA covers two M=128 tiles of query
+// blocks, so each B tile it loads feeds two MMA chains.  320 threads: warp 0
+// bulk-loads the B tiles, warp 1 issues MMAs, warps 2-9 expand the 0/1 A
+// tiles from the selection bitmask and run the epilogue.  K tiles of 64 key
+// blocks, 3-stage ring; D = 2 x (128 x 256) fp32 in TMEM.
 namespace {
-constexpr int kLStages = 2;
-constexpr int kATile = 128 * 64 * 2;  // 16 KB
+constexpr int kLStages = 3;
+constexpr int kSumTiles = 2;          // M=128 query-block tiles per CTA
+constexpr int kATile = 128 * 64 * 2;  // 16 KB per M tile
+constexpr int kAThreads = 128 * kSumTiles;
 struct LBars {
   uint64_t b_full[kLStages], a_full[kLStages], empty[kLStages], done;
   uint32_t tmem;
@@ -183,30 +187,30 @@ struct LBars {
 };
 }  // namespace
 
-__global__ void __launch_bounds__(192, 1) linear_sum_kernel(const uint8_t* __restrict__ hs,
+__global__ void __launch_bounds__(64 + kAThreads, 1) linear_sum_kernel(const uint8_t* __restrict__ hs,
                                                              const uint32_t* __restrict__ selbits, int nb, int nbt,
                                                              int nbw, uint16_t* __restrict__ hout, int* wd) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sB = smem;                               // kLStages x 32 KB
-  uint8_t* sA = smem + kLStages * kHsTile;          // kLStages x 16 KB
-  LBars* bars = reinterpret_cast<LBars*>(sA + kLStages * kATile);
+  uint8_t* sA = smem + kLStages * kHsTile;          // kLStages x kSumTiles x 16 KB
+  LBars* bars = reinterpret_cast<LBars*>(sA + kLStages * kSumTiles * kATile);
   volatile int* abort = &bars->abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nt = blockIdx.x, it = blockIdx.y, bh = blockIdx.z;
-  const int i0 = it * 128;
+  const int it = blockIdx.x, nt = blockIdx.y, bh = blockIdx.z;
+  const int i0 = it * 128 * kSumTiles;
   const uint8_t* hs_head = hs + (size_t)bh * nbt * 64 * 16384 * 2;
   if (tid == 0) {
     for (int s = 0; s < kLStages; ++s) {
       mbar_init(&bars->b_full[s], 1);
-      mbar_init(&bars->a_full[s], 128);
+      mbar_init(&bars->a_full[s], kAThreads);
       mbar_init(&bars->empty[s], 1);
     }
     mbar_init(&bars->done, 1);
     bars->abort = 0;
     mbar_fence_init();
   }
-  if (warp == 1) tmem_alloc(&bars->tmem, 256);
+  if (warp == 1) tmem_alloc(&bars->tmem, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -235,9 +239,11 @@ __global__ void __launch_bounds__(192, 1) linear_sum_kernel(const uint8_t* __res
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_bf16(tmem, smem_desc(sA + st * kATile + ks * 256, kQK_LBO, kQK_SBO),
-                   smem_desc(sB + st * kHsTile + ks * 2 * kHs_LBO, kHs_LBO, kHs_SBO), id, (kt > 0 || ks > 0));
+        for (int u = 0; u < kSumTiles; ++u)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(tmem + u * 256, smem_desc(sA + (st * kSumTiles + u) * kATile + ks * 256, kQK_LBO, kQK_SBO),
+                     smem_desc(sB + st * kHsTile + ks * 2 * kHs_LBO, kHs_LBO, kHs_SBO), id, (kt > 0 || ks > 0));
         mma_commit(&bars->empty[st]);
       }
       mma_commit(&bars->done);
@@ -246,8 +252,8 @@ __global__ void __launch_bounds__(192, 1) linear_sum_kernel(const uint8_t* __res
   } else {
     // A producer: thread -> query block row i = i0 + (tid - 64); 64 key
     // blocks per K tile from two bitmask words; 1 = NOT selected, j < nb.
-    const int r = tid - 64;
-    const int i = i0 + r;
+    const int u = (tid - 64) >> 7, r = (tid - 64) & 127;
+    const int i = i0 + 128 * u + r;
     bool ok = true;
     for (int kt = 0; kt < nbt; ++kt) {
       const int st = kt % kLStages;
@@ -263,7 +269,7 @@ __global__ void __launch_bounds__(192, 1) linear_sum_kernel(const uint8_t* __res
         const int left = nb - kt * 64;  // key blocks of this tile that exist
         ones = ~w & (left >= 64 ? ~0ull : ((1ull << left) - 1ull));
       }
-      uint8_t* A = sA + st * kATile;
+      uint8_t* A = sA + (st * kSumTiles + u) * kATile;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {  // 8 keys per 16-byte chunk
         const uint32_t b8 = (uint32_t)(ones >> (8 * ch)) & 0xFFu;
@@ -280,14 +286,14 @@ __global__ void __launch_bounds__(192, 1) linear_sum_kernel(const uint8_t* __res
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, abort, wd));
     if (ok) {
       tc_fence_after();
-      const int q = warp & 3;
+      const int q = warp & 3, ue = (warp - 2) >> 2;  // TMEM quadrant, M tile
       const int row = 32 * q + lane;  // TMEM lane == row of the M=128 tile
-      const int ir = i0 + row;
+      const int ir = i0 + 128 * ue + row;
       uint16_t* dst = hout + ((size_t)bh * nb + (ir < nb ? ir : 0)) * 16384 + (size_t)nt * 256;
 #pragma unroll 1
       for (int c0 = 0; c0 < 256; c0 += 16) {
         uint32_t v16[16];
-        SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * q) << 16) + c0, v16);
+        SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * q) << 16) + ue * 256 + c0, v16);
         tmem_ld_wait();
         if (ir < nb) {
           uint32_t pk[8];
@@ -301,7 +307,7 @@ __global__ void __launch_bounds__(192, 1) linear_sum_kernel(const uint8_t* __res
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- K4c ----
@@ -505,7 +511,7 @@ __global__ void w_tile_kernel(const uint16_t* __restrict__ w, uint16_t* __restri
 }
 
 int linear_kv_smem(int block) { return 2 * block * 128 * 2 + 1024; }
-int linear_sum_smem() { return kLStages * (kHsTile + kATile) + (int)sizeof(LBars) + 1024; }
+int linear_sum_smem() { return kLStages * (kHsTile + kSumTiles * kATile) + (int)sizeof(LBars) + 1024; }
 
 cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_t* hs, float* z, int* wd,
                              cudaStream_t st) {
@@ -532,7 +538,8 @@ cudaError_t launch_linear_sum(const uint8_t* hs, const uint32_t* selbits, const 
   const int smem = linear_sum_smem();
   cudaError_t e = cudaFuncSetAttribute(linear_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  linear_sum_kernel<<<dim3(64, (g.nb + 127) / 128, g.BH), 192, smem, st>>>(hs, selbits, g.nb, nbt, 2 * nbt, hout, wd);
+  linear_sum_kernel<<<dim3((g.nb + 128 * kSumTiles - 1) / (128 * kSumTiles), 64, g.BH), 64 + kAThreads, smem, st>>>(
+      hs, selbits, g.nb, nbt, 2 * nbt, hout, wd);
   return cudaGetLastError();
 }
 
