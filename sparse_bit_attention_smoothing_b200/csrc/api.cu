@@ -227,7 +227,8 @@ inline int launch_rc(cudaError_t e) { return e == cudaSuccess ? SAGESLA_OK : SAG
   } while (0)
 
 // Stats + quantisation (the front shared by every entry point).
-int run_front(const void* q, const void* k, const void* v, const Geom& g, const Buffers& b, cudaStream_t st) {
+int run_front(const void* q, const void* k, const void* v, const Geom& g, const Buffers& b, int dev,
+              cudaStream_t st) {
   {
     ProfScope ps(0, st);
     SAGESLA_TRY(launch_rc(launch_stats_partial(k, v, g, b.psum, b.pmax, st)));
@@ -239,7 +240,7 @@ int run_front(const void* q, const void* k, const void* v, const Geom& g, const 
   {
     ProfScope ps(2, st);
     SAGESLA_TRY(launch_rc(
-        launch_quant(q, k, v, b.mu, b.mv, g, b.q8t, b.k8t, b.v8t, b.sq, b.sk, b.qsum, b.ksum, st)));
+        launch_quant(q, k, v, b.mu, b.mv, g, b.q8t, b.k8t, b.v8t, b.sq, b.sk, b.qsum, b.ksum, watchdog(dev), st)));
   }
   return SAGESLA_OK;
 }
@@ -258,7 +259,7 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
   uint8_t* base = nullptr;
   SAGESLA_TRY(get_workspace(dev, st, sizes.total, &base));
   const Buffers b = carve(base, g, linear);
-  SAGESLA_TRY(run_front(q, k, v, g, b, st));
+  SAGESLA_TRY(run_front(q, k, v, g, b, dev, st));
   int* wd = watchdog(dev);
   if (linear) {
     {
@@ -446,7 +447,7 @@ int sagesla_get_quant(const void* q, const void* k, const void* v, int B, int H,
   uint8_t* base = nullptr;
   SAGESLA_TRY(get_workspace(dev, st, sizes.total, &base));
   const Buffers b = carve(base, g);
-  SAGESLA_TRY(run_front(q, k, v, g, b, st));
+  SAGESLA_TRY(run_front(q, k, v, g, b, dev, st));
   SAGESLA_TRY(launch_rc(launch_untile(b.q8t, b.k8t, b.v8t, g, q8, k8, v8, st)));
   const int nq64 = (N + 63) / 64;
   const size_t pitch = (size_t)g.nq * sizeof(float);
@@ -476,7 +477,7 @@ int sagesla_get_mask(const void* q, const void* k, int B, int H, int N, int d, i
   const Buffers b = carve(base, g);
   // The mask needs only K's mean and the pooled sums; V is read as K here
   // (its quantised codes are discarded).
-  SAGESLA_TRY(run_front(q, k, k, g, b, st));
+  SAGESLA_TRY(run_front(q, k, k, g, b, dev, st));
   SAGESLA_TRY(launch_rc(launch_pool_topk(b.qsum, b.ksum, g, idx_out, qbar ? qbar : b.qbar, kbar ? kbar : b.kbar,
                                          nullptr, nullptr, nullptr, nullptr, st)));
   if (k_out) *k_out = g.kc;

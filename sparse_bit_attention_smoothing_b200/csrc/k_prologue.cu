@@ -84,20 +84,32 @@ __global__ void stats_final_kernel(const double* __restrict__ psum, const float*
 }
 
 // ---------------------------------------------------------------- K2 ----
-// grid (nq, BH), 128 threads: one 64-token tile of Q, K and V.
-// Thread t handles channel group cg = t/8 (8 channels) of rows t%8 + 8*i:
-// the lanes of a warp span 8 rows and 4 channel groups, which keeps the
-// stores into the tile images (whose channel groups lie 512 or 1024 bytes
-// apart, one bank) at most 4-way conflicted.
-__device__ __forceinline__ float block_max128(float x, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = x;
-  __syncthreads();
-  float r = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  __syncthreads();
-  return r;
-}
+// Persistent: one CTA per SM walks the list of (head, 64-token tile) pairs
+// with a stride of gridDim.x.  Thread 0 stages the Q, K and V rows of the
+// next kQStages tiles in shared memory with bulk copies (one per tensor,
+// nvalid x 256 bytes, completing on the stage's mbarrier), so that the HBM
+// reads of later tiles overlap the quantisation of this one.
+//   Q/K: thread t holds channels 8*cg..+7 (cg = (t/8) % 16) of the rows
+//        t%8 + 32*(t/128) + 8*i, i < 4.  A warp spans 8 rows and 4 channel
+//        groups, so its 8-byte stores into the K-major tile images cover
+//        all 32 banks twice (no conflict).
+//   V:   warp w converts keys 16*(w/2)..+15 of channels 64*(w%2)..+63; lane
+//        l the channel pair c0 = 64*(w%2) + 2l, c0 + 1.  Each channel gives
+//        one 16-byte chunk (16 consecutive keys) of the V^T image; lanes
+//        whose bit 2 is set store the odd channel first, which spreads the
+//        chunks of a quarter warp over all 32 banks.
+constexpr int kQStages = 3;
+constexpr int kQThreads = 256;
+constexpr int kRowBytes = kD * 2;  // one bf16 row of Q, K or V
+constexpr int kSumPitch = kD + 1;  // pooled partial sums: padded rows (bank spread)
+struct QuantSmem {
+  uint8_t stage[kQStages][3][kQB * kRowBytes];  // Q, K, V rows of a tile (48 KB per stage)
+  uint8_t img[3][kTile];                        // Q^, K^ and V^T tile images
+  float psum[2][16][kSumPitch];                 // per-thread column sums of Q and K - mu
+  float red[2][8];
+  uint64_t full[kQStages];
+  int abort;
+};
 
 // rne(fl32(x * mult)) as a byte.  |x| <= amax and mult = fl32(127/amax), so
 // the product lies within 127 * (1 + 2^-23) and no clamp is needed; adding
@@ -107,132 +119,193 @@ __device__ __forceinline__ uint32_t i8code(float x, float mult) {
   return (uint32_t)__float_as_int(__fadd_rn(__fmul_rn(x, mult), 12582912.0f)) & 0xFFu;
 }
 
-__global__ void __launch_bounds__(128) quant_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
-                                                    const uint4* __restrict__ v, const float* __restrict__ mu,
-                                                    const float* __restrict__ mv, int N, int nq,
-                                                    uint8_t* __restrict__ q8t, uint8_t* __restrict__ k8t,
-                                                    uint8_t* __restrict__ v8t, float* __restrict__ sq,
-                                                    float* __restrict__ sk, float* __restrict__ qsum,
-                                                    float* __restrict__ ksum) {
-  const int bh = blockIdx.y, tile = blockIdx.x, t = threadIdx.x;
-  const int cg = t >> 3, rr = t & 7;
-  const int n0 = tile * kQB;
-  __shared__ __align__(16) uint8_t sq8[kTile];
-  __shared__ __align__(16) uint8_t sk8[kTile];
-  __shared__ __align__(16) uint8_t sv8[kTile];
-  __shared__ float red[4];
-  __shared__ float psq[8][kD];
-  __shared__ float psk[8][kD];
-
-  float muc[8], mvc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    muc[i] = mu[(size_t)bh * kD + cg * 8 + i];
-    mvc[i] = mv[(size_t)bh * kD + cg * 8 + i];
-  }
-  // Load this thread's 8 rows x 8 channels of Q, K, V (zeros past N).
-  float xq[8][8], xk[8][8];
-  uint32_t vw[8][4];
-  const size_t base = (size_t)bh * N * 16;
-  float aq = 0.f, ak = 0.f;
-  float sumq[8], sumk[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    sumq[i] = 0.f;
-    sumk[i] = 0.f;
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = rr + 8 * i;
-    const int n = n0 + r;
-    uint4 qq = make_uint4(0, 0, 0, 0), kk = qq, vv = qq;
-    const bool valid = n < N;
-    if (valid) {
-      qq = __ldg(q + base + (size_t)n * 16 + cg);
-      kk = __ldg(k + base + (size_t)n * 16 + cg);
-      vv = __ldg(v + base + (size_t)n * 16 + cg);
-    }
-    uint32_t qw[4] = {qq.x, qq.y, qq.z, qq.w};
-    uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};
-    vw[i][0] = vv.x;
-    vw[i][1] = vv.y;
-    vw[i][2] = vv.z;
-    vw[i][3] = vv.w;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      xq[i][2 * j] = bf16_lo(qw[j]);
-      xq[i][2 * j + 1] = bf16_hi(qw[j]);
-      xk[i][2 * j] = valid ? __fsub_rn(bf16_lo(kw[j]), muc[2 * j]) : 0.f;
-      xk[i][2 * j + 1] = valid ? __fsub_rn(bf16_hi(kw[j]), muc[2 * j + 1]) : 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      aq = fmaxf(aq, fabsf(xq[i][j]));
-      ak = fmaxf(ak, fabsf(xk[i][j]));
-      sumq[j] += xq[i][j];
-      sumk[j] += xk[i][j];
-    }
-  }
-  aq = block_max128(aq, red);
-  ak = block_max128(ak, red);
-  const float mq = aq > 0.f ? __fdiv_rn(127.f, aq) : 0.f;
-  const float mk = ak > 0.f ? __fdiv_rn(127.f, ak) : 0.f;
+__global__ void __launch_bounds__(kQThreads, 1)
+    quant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ k, const uint8_t* __restrict__ v,
+                 const float* __restrict__ mu, const float* __restrict__ mv, int N, int nq, int ntiles,
+                 uint8_t* __restrict__ q8t, uint8_t* __restrict__ k8t, uint8_t* __restrict__ v8t,
+                 float* __restrict__ sq, float* __restrict__ sk, float* __restrict__ qsum, float* __restrict__ ksum,
+                 int* wd) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  QuantSmem& S = *reinterpret_cast<QuantSmem*>(smem_raw);
+  volatile int* abort = &S.abort;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int cg = (t >> 3) & 15, rr = t & 7, h = t >> 7;
+  const int nmine = (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
   if (t == 0) {
-    sq[(size_t)bh * nq + tile] = aq > 0.f ? __fdiv_rn(aq, 127.f) : 1.f;
-    sk[(size_t)bh * nq + tile] = ak > 0.f ? __fdiv_rn(ak, 127.f) : 1.f;
-  }
-  // Codes into the smem tile images.
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = rr + 8 * i;
-    uint32_t qa = 0, qb = 0, ka = 0, kb = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      qa |= i8code(xq[i][j], mq) << (8 * j);
-      qb |= i8code(xq[i][j + 4], mq) << (8 * j);
-      ka |= i8code(xk[i][j], mk) << (8 * j);
-      kb |= i8code(xk[i][j + 4], mk) << (8 * j);
-    }
-    const uint32_t off = kmajor_off(r, cg * 8, kQK_LBO, kQK_SBO);
-    *reinterpret_cast<uint2*>(sq8 + off) = make_uint2(qa, qb);
-    *reinterpret_cast<uint2*>(sk8 + off) = make_uint2(ka, kb);
-    // V^T tile: element (channel c, key r).
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c0 = cg * 8 + 2 * j;
-      const float v0 = __fmul_rn(bf16_lo(vw[i][j]), mvc[2 * j]);
-      const float v1 = __fmul_rn(bf16_hi(vw[i][j]), mvc[2 * j + 1]);
-      const uint32_t pr = e4m3x2(v0, v1);
-      sv8[kmajor_off(c0, r, kV_LBO, kV_SBO)] = (uint8_t)(pr & 0xFF);
-      sv8[kmajor_off(c0 + 1, r, kV_LBO, kV_SBO)] = (uint8_t)(pr >> 8);
-    }
-  }
-  // Pooled column sums over this tile's valid rows.
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    psq[rr][cg * 8 + j] = sumq[j];
-    psk[rr][cg * 8 + j] = sumk[j];
+    for (int s = 0; s < kQStages; ++s) mbar_init(&S.full[s], 1);
+    S.abort = 0;
+    mbar_fence_init();
   }
   __syncthreads();
-  {
-    float a = 0.f, b = 0.f;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      a += psq[r][t];
-      b += psk[r][t];
+  // Thread 0: stage the rows of this CTA's j-th tile.
+  auto issue = [&](int j) {
+    const int gt = (int)blockIdx.x + j * (int)gridDim.x;
+    const int bh = gt / nq, n0 = (gt - bh * nq) * kQB;
+    uint64_t* bar = &S.full[j % kQStages];
+    if (n0 >= N) {  // the padding tile of an odd tile count: nothing to load
+      mbar_arrive(bar);
+      return;
     }
-    qsum[((size_t)bh * nq + tile) * kD + t] = a;
-    ksum[((size_t)bh * nq + tile) * kD + t] = b;
-  }
-  // Coalesced 16-byte copies of the three 8 KB tiles.
-  const size_t tb = ((size_t)bh * nq + tile) * kTile;
+    const uint32_t bytes = (uint32_t)min(kQB, N - n0) * kRowBytes;
+    const size_t off = ((size_t)bh * N + n0) * kRowBytes;
+    mbar_expect_tx(bar, 3 * bytes);
+    bulk_g2s(S.stage[j % kQStages][0], q + off, bytes, bar);
+    bulk_g2s(S.stage[j % kQStages][1], k + off, bytes, bar);
+    bulk_g2s(S.stage[j % kQStages][2], v + off, bytes, bar);
+  };
+  int issued = 0;
+  if (t == 0)
+    for (; issued < min(kQStages, nmine); ++issued) issue(issued);
+
+  int j = 0;
+  for (; j < nmine; ++j) {
+    const int st = j % kQStages;
+    const bool ok = mbar_wait(&S.full[st], (uint32_t)(j / kQStages) & 1u, abort, wd);
+    // Uniform exit; also orders the previous tile's reads of img/psum/red
+    // before this tile's writes.
+    if (__syncthreads_or(!ok)) break;
+    const int gt = (int)blockIdx.x + j * (int)gridDim.x;
+    const int bh = gt / nq, n0 = (gt - bh * nq) * kQB;
+    const int nvalid = max(0, min(kQB, N - n0));  // rows past N read as 0
+    const uint8_t* sQ = S.stage[st][0];
+    const uint8_t* sK = S.stage[st][1];
+    const uint8_t* sV = S.stage[st][2];
+
+    // ---- Q, K rows: absmax and column sums (rows past N read as 0) ----
+    const float4 mu0 = *reinterpret_cast<const float4*>(mu + (size_t)bh * kD + cg * 8);
+    const float4 mu1 = *reinterpret_cast<const float4*>(mu + (size_t)bh * kD + cg * 8 + 4);
+    const float muc[8] = {mu0.x, mu0.y, mu0.z, mu0.w, mu1.x, mu1.y, mu1.z, mu1.w};
+    uint32_t rq[4][4], rk[4][4];
+    float aq = 0.f, ak = 0.f, sumq[8], sumk[8];
 #pragma unroll
-  for (int i = 0; i < kTile / 16 / 128; ++i) {
-    const int o = (t + i * 128) * 16;
-    *reinterpret_cast<uint4*>(q8t + tb + o) = *reinterpret_cast<const uint4*>(sq8 + o);
-    *reinterpret_cast<uint4*>(k8t + tb + o) = *reinterpret_cast<const uint4*>(sk8 + o);
-    *reinterpret_cast<uint4*>(v8t + tb + o) = *reinterpret_cast<const uint4*>(sv8 + o);
+    for (int c = 0; c < 8; ++c) {
+      sumq[c] = 0.f;
+      sumk[c] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = rr + 32 * h + 8 * i;
+      uint4 qq = make_uint4(0, 0, 0, 0), kk = qq;
+      if (r < nvalid) {
+        qq = *reinterpret_cast<const uint4*>(sQ + r * kRowBytes + cg * 16);
+        kk = *reinterpret_cast<const uint4*>(sK + r * kRowBytes + cg * 16);
+      }
+      rq[i][0] = qq.x; rq[i][1] = qq.y; rq[i][2] = qq.z; rq[i][3] = qq.w;
+      rk[i][0] = kk.x; rk[i][1] = kk.y; rk[i][2] = kk.z; rk[i][3] = kk.w;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float xq = (c & 1) ? bf16_hi(rq[i][c >> 1]) : bf16_lo(rq[i][c >> 1]);
+        const float xk =
+            r < nvalid ? __fsub_rn((c & 1) ? bf16_hi(rk[i][c >> 1]) : bf16_lo(rk[i][c >> 1]), muc[c]) : 0.f;
+        aq = fmaxf(aq, fabsf(xq));
+        ak = fmaxf(ak, fabsf(xk));
+        sumq[c] += xq;
+        sumk[c] += xk;
+      }
+    }
+
+    // ---- V -> FP8 codes, two 16-key chunks of the V^T image ----
+    {
+      const int c0 = 64 * (warp & 1) + 2 * lane, r0 = 16 * (warp >> 1);
+      const float m0 = mv[(size_t)bh * kD + c0], m1 = mv[(size_t)bh * kD + c0 + 1];
+      uint32_t e0[4] = {0u, 0u, 0u, 0u}, e1[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int m = 0; m < 16; m += 2) {
+        const int r = r0 + m;
+        const uint32_t w0 = r < nvalid ? *reinterpret_cast<const uint32_t*>(sV + r * kRowBytes + c0 * 2) : 0u;
+        const uint32_t w1 = r + 1 < nvalid ? *reinterpret_cast<const uint32_t*>(sV + (r + 1) * kRowBytes + c0 * 2) : 0u;
+        const uint32_t p0 = e4m3x2(__fmul_rn(bf16_lo(w0), m0), __fmul_rn(bf16_lo(w1), m0));
+        const uint32_t p1 = e4m3x2(__fmul_rn(bf16_hi(w0), m1), __fmul_rn(bf16_hi(w1), m1));
+        e0[m >> 2] |= p0 << (8 * (m & 2));
+        e1[m >> 2] |= p1 << (8 * (m & 2));
+      }
+      const bool odd_first = (lane >> 2) & 1;
+      const uint4 ev = make_uint4(e0[0], e0[1], e0[2], e0[3]), od = make_uint4(e1[0], e1[1], e1[2], e1[3]);
+      *reinterpret_cast<uint4*>(S.img[2] + kmajor_off(odd_first ? c0 + 1 : c0, r0, kV_LBO, kV_SBO)) =
+          odd_first ? od : ev;
+      *reinterpret_cast<uint4*>(S.img[2] + kmajor_off(odd_first ? c0 : c0 + 1, r0, kV_LBO, kV_SBO)) =
+          odd_first ? ev : od;
+    }
+
+    // ---- tile absmax of Q and K - mu ----
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      aq = fmaxf(aq, __shfl_xor_sync(0xffffffffu, aq, o));
+      ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, o));
+    }
+    if (lane == 0) {
+      S.red[0][warp] = aq;
+      S.red[1][warp] = ak;
+    }
+    __syncthreads();  // every read of this stage is done: refill it
+    if (t == 0 && issued < nmine) {
+      fence_proxy_async_smem();
+      issue(issued++);
+    }
+    aq = S.red[0][0];
+    ak = S.red[1][0];
+#pragma unroll
+    for (int w = 1; w < kQThreads / 32; ++w) {
+      aq = fmaxf(aq, S.red[0][w]);
+      ak = fmaxf(ak, S.red[1][w]);
+    }
+    const float mq = aq > 0.f ? __fdiv_rn(127.f, aq) : 0.f;
+    const float mk = ak > 0.f ? __fdiv_rn(127.f, ak) : 0.f;
+    if (t == 0) {
+      sq[gt] = aq > 0.f ? __fdiv_rn(aq, 127.f) : 1.f;
+      sk[gt] = ak > 0.f ? __fdiv_rn(ak, 127.f) : 1.f;
+    }
+
+    // ---- Q, K codes into the tile images; partial column sums ----
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = rr + 32 * h + 8 * i;
+      uint32_t qa = 0, qb = 0, ka = 0, kb = 0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float xq0 = (c & 1) ? bf16_hi(rq[i][c >> 1]) : bf16_lo(rq[i][c >> 1]);
+        const float xq1 = (c & 1) ? bf16_hi(rq[i][2 + (c >> 1)]) : bf16_lo(rq[i][2 + (c >> 1)]);
+        const float xk0 =
+            r < nvalid ? __fsub_rn((c & 1) ? bf16_hi(rk[i][c >> 1]) : bf16_lo(rk[i][c >> 1]), muc[c]) : 0.f;
+        const float xk1 =
+            r < nvalid ? __fsub_rn((c & 1) ? bf16_hi(rk[i][2 + (c >> 1)]) : bf16_lo(rk[i][2 + (c >> 1)]), muc[c + 4])
+                       : 0.f;
+        qa |= i8code(xq0, mq) << (8 * c);
+        qb |= i8code(xq1, mq) << (8 * c);
+        ka |= i8code(xk0, mk) << (8 * c);
+        kb |= i8code(xk1, mk) << (8 * c);
+      }
+      const uint32_t off = kmajor_off(r, cg * 8, kQK_LBO, kQK_SBO);
+      *reinterpret_cast<uint2*>(S.img[0] + off) = make_uint2(qa, qb);
+      *reinterpret_cast<uint2*>(S.img[1] + off) = make_uint2(ka, kb);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      S.psum[0][8 * h + rr][cg * 8 + c] = sumq[c];
+      S.psum[1][8 * h + rr][cg * 8 + c] = sumk[c];
+    }
+    __syncthreads();
+
+    // ---- pooled column sums (fixed order) and the tile images to HBM ----
+    {
+      const int which = t >> 7, col = t & 127;
+      float a = 0.f;
+#pragma unroll
+      for (int p = 0; p < 16; ++p) a += S.psum[which][p][col];
+      (which ? ksum : qsum)[(size_t)gt * kD + col] = a;
+    }
+    const size_t tb = (size_t)gt * kTile;
+#pragma unroll
+    for (int m = 0; m < 3 * kTile / 16 / kQThreads; ++m) {
+      const int idx = t + m * kQThreads;  // 16-byte unit over the three images
+      const int which = idx / (kTile / 16), o = (idx % (kTile / 16)) * 16;
+      uint8_t* dst = which == 0 ? q8t : (which == 1 ? k8t : v8t);
+      *reinterpret_cast<uint4*>(dst + tb + o) = *reinterpret_cast<const uint4*>(S.img[which] + o);
+    }
   }
+  // After an abort, wait for the copies still in flight before exiting.
+  if (t == 0)
+    for (int jj = j; jj < issued; ++jj) mbar_wait_drain(&S.full[jj % kQStages], (uint32_t)(jj / kQStages) & 1u, wd);
 }
 
 // Row-major codes from the tiles (parity entry point only).
@@ -266,9 +339,16 @@ cudaError_t launch_stats_final(const double* psum, const float* pmax, const Geom
 
 cudaError_t launch_quant(const void* q, const void* k, const void* v, const float* mu, const float* mv, const Geom& g,
                          uint8_t* q8t, uint8_t* k8t, uint8_t* v8t, float* sq, float* sk, float* qsum, float* ksum,
-                         cudaStream_t st) {
-  quant_kernel<<<dim3(g.nq, g.BH), 128, 0, st>>>((const uint4*)q, (const uint4*)k, (const uint4*)v, mu, mv, g.N, g.nq,
-                                                 q8t, k8t, v8t, sq, sk, qsum, ksum);
+                         int* wd, cudaStream_t st) {
+  const int smem = (int)sizeof(QuantSmem);
+  cudaError_t e = cudaFuncSetAttribute(quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int ntiles = g.BH * g.nq;
+  quant_kernel<<<min(ntiles, sms), kQThreads, smem, st>>>((const uint8_t*)q, (const uint8_t*)k, (const uint8_t*)v, mu,
+                                                          mv, g.N, g.nq, ntiles, q8t, k8t, v8t, sq, sk, qsum, ksum, wd);
   return cudaGetLastError();
 }
 

@@ -27,7 +27,7 @@ cudaError_t launch_stats_final(const double* psum, const float* pmax, const Geom
 // K2: smoothing + INT8 Q/K tiles + FP8 V^T tiles + per-64-row pooled sums.
 cudaError_t launch_quant(const void* q, const void* k, const void* v, const float* mu, const float* mv,
                          const Geom& g, uint8_t* q8t, uint8_t* k8t, uint8_t* v8t, float* sq, float* sk,
-                         float* qsum, float* ksum, cudaStream_t st);
+                         float* qsum, float* ksum, int* wd, cudaStream_t st);
 // Untile the quantised tiles back to row-major codes (parity entry only).
 cudaError_t launch_untile(const uint8_t* q8t, const uint8_t* k8t, const uint8_t* v8t, const Geom& g, int8_t* q8,
                           int8_t* k8, uint8_t* v8, cudaStream_t st);
