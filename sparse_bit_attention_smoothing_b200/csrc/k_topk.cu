@@ -289,8 +289,9 @@ cudaError_t launch_pool_topk(const float* qsum, const float* ksum, const Geom& g
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  // Eight query blocks per CTA where the scores fit in shared memory (three
-  // CTAs per SM at 720p), and the order keys in registers up to nb = 1280.
+  // Eight query blocks per CTA where the scores fit in shared memory (82 KB
+  // and 256 threads at nb = 1182: two CTAs per SM), and the order keys in
+  // registers up to nb = 1280.
   constexpr size_t kSmemMax = 227 * 1024;
   if (topk_smem(8, g.nb) <= kSmemMax)
     return g.nb <= 32 * 40 ? launch_topk_cfg<8, 40>(qbar, kbar, g, idx, zin, ztot, selbits, zout, st)
