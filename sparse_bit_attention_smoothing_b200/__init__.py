@@ -28,8 +28,8 @@ class SageSLAError(RuntimeError):
 
 
 EXPORTS = ["sagesla_attn", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
-           "sagesla_topk_count", "sagesla_sync_status", "sagesla_strerror", "sagesla_release", "sagesla_profile",
-           "sagesla_profile_read"]
+           "sagesla_smooth_stats_noalloc", "sagesla_topk_count", "sagesla_sync_status", "sagesla_strerror",
+           "sagesla_release", "sagesla_profile", "sagesla_profile_read"]
 KERNELS = ["stats", "stats_final", "quant", "pool_topk", "linear_kv", "linear_sum", "flash", "w_tile",
            "linear_apply"]
 
@@ -47,6 +47,7 @@ def lib():
         L.sagesla_attn_host.argtypes = [P, P, P, P, P, i, i, i, i, i, f, P]
         L.sagesla_get_quant.argtypes = [P, P, P, i, i, i, i, P, P, P, P, P, P, P, P]
         L.sagesla_get_mask.argtypes = [P, P, i, i, i, i, i, f, P, P, P, P, P]
+        L.sagesla_smooth_stats_noalloc.argtypes = [P, P, i, i, i, i, P, P, P]
         L.sagesla_topk_count.argtypes = [i, f]
         L.sagesla_sync_status.argtypes = [P]
         L.sagesla_strerror.restype = ctypes.c_char_p
@@ -152,6 +153,20 @@ def sagesla_get_mask(q, k, block: int = 64, topk: float = 0.1, pooled: bool = Fa
     return r
 
 
+def sagesla_smooth_stats_noalloc(k, v, mu=None, sv=None, stream=None):
+    """Per-channel mean of K and FP8 scale of V, [B, H, d] fp32 each, without any device allocation by the
+    library (mu / sv are allocated here by torch unless given).  Returns (mu, sv)."""
+    import torch
+    B, H, N, d = _shape(k)
+    if mu is None:
+        mu = torch.empty(B, H, d, dtype=torch.float32, device=k.device)
+    if sv is None:
+        sv = torch.empty(B, H, d, dtype=torch.float32, device=k.device)
+    _check(lib().sagesla_smooth_stats_noalloc(_ptr(k), _ptr(v), B, H, N, d, _ptr(mu), _ptr(sv), _stream(stream)),
+           "sagesla_smooth_stats_noalloc")
+    return mu, sv
+
+
 def sync_status(stream=None) -> int:
     return lib().sagesla_sync_status(_stream(stream))
 
@@ -172,3 +187,16 @@ def profile_read() -> dict:
 
 def release():
     lib().sagesla_release()
+
+
+def strerror(code: int) -> str:
+    return lib().sagesla_strerror(code).decode()
+
+
+# The C names of the utility calls, for callers that follow the header.
+sagesla_topk_count = topk_count
+sagesla_sync_status = sync_status
+sagesla_strerror = strerror
+sagesla_release = release
+sagesla_profile = profile
+sagesla_profile_read = profile_read

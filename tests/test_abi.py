@@ -31,6 +31,14 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, n), n
 
 
+def test_binding_covers_every_declared_symbol():
+    import sparse_bit_attention_smoothing_b200 as sg
+    names = declared_functions()
+    assert set(sg.EXPORTS) == set(names)
+    for n in names:
+        assert callable(getattr(sg, n, None)), n
+
+
 def test_topk_count_matches_oracle(L, orc):
     for nb in (1, 7, 10, 16, 512, 591, 1182, 5000):
         for t in (0.01, 0.05, 0.1, 0.15, 0.25, 0.3, 0.5, 0.99, 1.0):
