@@ -3,6 +3,7 @@ host-side argument checks reject bad calls before any CUDA work (no GPU needed).
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -73,3 +74,39 @@ def test_rejects_bad_arguments_without_launch(L):
     assert L.sagesla_attn(a, m, a, None, a, 1, 1, 64, 128, 64, F(0.1), None) == -2
     assert L.sagesla_attn(a, a, a, m, a, 1, 1, 64, 128, 64, F(0.1), None) == -2
     assert L.dense_int8_attn(a, a, None, a, 1, 1, 64, 128, None) == -1
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "sagesla.h"
+int main(void) {
+  /* every call below is answered by the host-side checks: no CUDA work */
+  if (sagesla_topk_count(1182, 0.1f) != 119) return 1;
+  if (sagesla_topk_count(16, 0.25f) != 4) return 2;
+  if (sagesla_attn(NULL, NULL, NULL, NULL, NULL, 1, 1, 64, 128, 64, 0.1f, NULL) != SAGESLA_ERR_INVALID) return 3;
+  if (dense_int8_attn(NULL, NULL, NULL, NULL, 1, 1, 64, 128, NULL) != SAGESLA_ERR_INVALID) return 4;
+  if (strlen(sagesla_strerror(SAGESLA_ERR_MISALIGNED)) == 0) return 5;
+  puts("c client ok");
+  return 0;
+}
+"""
+
+
+def test_header_is_c99_and_the_library_links_from_c(L, tmp_path):
+    """A plain C99 program includes the header, links against the library and
+    gets the documented answers from calls that fail their argument checks."""
+    import shutil
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    pkg = os.path.join(ROOT, "sparse_bit_attention_smoothing_b200")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-L", pkg, "-lsagesla", f"-Wl,-rpath,{pkg}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and "c client ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
