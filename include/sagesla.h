@@ -158,6 +158,19 @@ int sagesla_topk_count(int nb, float topk);
  */
 int sagesla_sync_status(sagesla_stream_t stream);
 
+/*
+ * sagesla_watchdog_selftest: exercises the failure-detection path on the GPU
+ * without faulting it.  Launches (on `stream`) one thread that waits on an
+ * mbarrier nothing ever arrives on, `probes` times (1 .. 1048576; each probe
+ * may suspend the thread briefly), and then records the expiry in the
+ * device's watchdog word the way every bounded wait of the library does.
+ * The next sagesla_sync_status() on the stream returns
+ * SAGESLA_ERR_DEVICE_TIMEOUT and clears the word; the context stays usable.
+ * Returns SAGESLA_ERR_INVALID for `probes` out of range (no launch),
+ * SAGESLA_ERR_NO_DEVICE / SAGESLA_ERR_LAUNCH as the other entry points.
+ */
+int sagesla_watchdog_selftest(int probes, sagesla_stream_t stream);
+
 /* Human-readable text for a return code (static storage). */
 const char* sagesla_strerror(int code);
 

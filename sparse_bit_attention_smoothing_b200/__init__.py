@@ -29,7 +29,7 @@ class SageSLAError(RuntimeError):
 
 EXPORTS = ["sagesla_attn", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
            "sagesla_smooth_stats_noalloc", "sagesla_topk_count", "sagesla_sync_status", "sagesla_strerror",
-           "sagesla_release", "sagesla_profile", "sagesla_profile_read"]
+           "sagesla_release", "sagesla_profile", "sagesla_profile_read", "sagesla_watchdog_selftest"]
 KERNELS = ["stats", "stats_final", "quant", "pool_topk", "linear_kv", "linear_sum", "flash", "w_tile",
            "linear_apply"]
 
@@ -50,6 +50,7 @@ def lib():
         L.sagesla_smooth_stats_noalloc.argtypes = [P, P, i, i, i, i, P, P, P]
         L.sagesla_topk_count.argtypes = [i, f]
         L.sagesla_sync_status.argtypes = [P]
+        L.sagesla_watchdog_selftest.argtypes = [i, P]
         L.sagesla_strerror.restype = ctypes.c_char_p
         L.sagesla_strerror.argtypes = [i]
         L.sagesla_release.restype = None
@@ -165,6 +166,12 @@ def sagesla_smooth_stats_noalloc(k, v, mu=None, sv=None, stream=None):
     _check(lib().sagesla_smooth_stats_noalloc(_ptr(k), _ptr(v), B, H, N, d, _ptr(mu), _ptr(sv), _stream(stream)),
            "sagesla_smooth_stats_noalloc")
     return mu, sv
+
+
+def sagesla_watchdog_selftest(probes: int = 1000, stream=None):
+    """Make one bounded device-side wait expire on purpose (nothing faults); the next sync_status() on the stream
+    then returns -5 (device watchdog timeout) and clears the flag."""
+    _check(lib().sagesla_watchdog_selftest(probes, _stream(stream)), "sagesla_watchdog_selftest")
 
 
 def sync_status(stream=None) -> int:

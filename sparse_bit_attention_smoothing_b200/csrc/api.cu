@@ -484,6 +484,13 @@ int sagesla_get_mask(const void* q, const void* k, int B, int H, int N, int d, i
   return SAGESLA_OK;
 }
 
+int sagesla_watchdog_selftest(int probes, sagesla_stream_t stream) {
+  if (probes < 1 || probes > (1 << 20)) return SAGESLA_ERR_INVALID;
+  int dev = 0;
+  SAGESLA_TRY(check_device(&dev));
+  return launch_rc(launch_watchdog_selftest(probes, watchdog(dev), reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int sagesla_sync_status(sagesla_stream_t stream) {
   int dev = 0;
   SAGESLA_TRY(check_device(&dev));

@@ -62,5 +62,7 @@ struct FlashArgs {
   int add_out;          // 1: out already holds the linear branch y (bf16); add O_s to it
 };
 cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int* wd);
+// Waits `probes` times on an mbarrier that never completes, then sets *wd.
+cudaError_t launch_watchdog_selftest(int probes, int* wd, cudaStream_t st);
 
 }  // namespace sagesla

@@ -74,6 +74,8 @@ def test_rejects_bad_arguments_without_launch(L):
     assert L.sagesla_attn(a, m, a, None, a, 1, 1, 64, 128, 64, F(0.1), None) == -2
     assert L.sagesla_attn(a, a, a, m, a, 1, 1, 64, 128, 64, F(0.1), None) == -2
     assert L.dense_int8_attn(a, a, None, a, 1, 1, 64, 128, None) == -1
+    assert L.sagesla_watchdog_selftest(0, None) == -1
+    assert L.sagesla_watchdog_selftest((1 << 20) + 1, None) == -1
 
 
 C_CLIENT = r"""
@@ -87,6 +89,7 @@ int main(void) {
   if (sagesla_attn(NULL, NULL, NULL, NULL, NULL, 1, 1, 64, 128, 64, 0.1f, NULL) != SAGESLA_ERR_INVALID) return 3;
   if (dense_int8_attn(NULL, NULL, NULL, NULL, 1, 1, 64, 128, NULL) != SAGESLA_ERR_INVALID) return 4;
   if (strlen(sagesla_strerror(SAGESLA_ERR_MISALIGNED)) == 0) return 5;
+  if (sagesla_watchdog_selftest(0, NULL) != SAGESLA_ERR_INVALID) return 6;
   puts("c client ok");
   return 0;
 }
