@@ -96,7 +96,7 @@ int main(void) {
 """
 
 
-def test_header_is_c99_and_the_library_links_from_c(L, tmp_path):
+def test_header_is_c99_and_the_library_links_from_c(L):
     """A plain C99 program includes the header, links against the library and
     gets the documented answers from calls that fail their argument checks."""
     import shutil
@@ -104,9 +104,12 @@ def test_header_is_c99_and_the_library_links_from_c(L, tmp_path):
     if cc is None:
         pytest.skip("no C compiler")
     pkg = os.path.join(ROOT, "sparse_bit_attention_smoothing_b200")
-    src = tmp_path / "client.c"
-    src.write_text(C_CLIENT)
-    exe = tmp_path / "client"
+    work = os.path.join(ROOT, "_build")  # the build directory (not tracked)
+    os.makedirs(work, exist_ok=True)
+    src = os.path.join(work, "c_client.c")
+    with open(src, "w") as f:
+        f.write(C_CLIENT)
+    exe = os.path.join(work, "c_client")
     r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
                         str(src), "-L", pkg, "-lsagesla", f"-Wl,-rpath,{pkg}", "-o", str(exe)],
                        capture_output=True, text=True)
