@@ -38,8 +38,10 @@
  *     first call needing a larger workspace on a (device, stream) allocates it
  *     stream-ordered.
  *   - Supported: d == 128, block in {64, 128}, 0 < topk <= 1, B, H, N >= 1,
- *     B*H*N*d < 2^40.  Anything else returns SAGESLA_ERR_INVALID without
- *     launching.  There is no CPU fallback and no alternative backend.
+ *     B*H <= 65535, ceil(N / block) <= 12288 (N <= 786432 at block 64,
+ *     1572864 at block 128), B*H*N*d < 2^40.  Anything else returns
+ *     SAGESLA_ERR_INVALID without launching.  There is no CPU fallback and no
+ *     alternative backend.
  *   - The library owns a workspace cache keyed by (device, stream);
  *     sagesla_release() frees it.
  */

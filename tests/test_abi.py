@@ -75,6 +75,11 @@ def test_rejects_bad_arguments_without_launch(L):
     assert L.sagesla_attn(a, a, a, m, a, 1, 1, 64, 128, 64, F(0.1), None) == -2
     assert L.dense_int8_attn(a, a, None, a, 1, 1, 64, 128, None) == -1
     assert L.sagesla_watchdog_selftest(0, None) == -1
+    # the longest sequence: Nb <= 12288 (four score rows of the top-k kernel in 227 KB of shared memory);
+    # one token more is refused before any CUDA call, the limit itself passes the argument checks
+    for n_max, blk in ((786432, 64), (1572864, 128)):
+        assert L.sagesla_attn(a, a, a, None, a, 1, 1, n_max + 1, 128, blk, F(0.1), None) == -1
+        assert L.sagesla_attn(a, a, a, None, a, 1, 1, n_max, 128, blk, F(0.1), None) != -1
     assert L.sagesla_watchdog_selftest((1 << 20) + 1, None) == -1
 
 
