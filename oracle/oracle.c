@@ -40,7 +40,7 @@
 
 #define ORC_QBLK 64 /* quantisation block of Q and K: 64 tokens */
 
-int orc_version(void) { return 1; }
+int orc_version(void) { return 2; }
 
 int orc_threads(void) {
 #ifdef _OPENMP
@@ -391,8 +391,12 @@ void orc_block_scores_f64(const uint16_t* q, const uint16_t* k, int BH, int N, i
 /* ------------------------------------------------------------------------ */
 /* Steps 6-8: the sparse softmax branch, the linear branch, the projection. */
 /* ------------------------------------------------------------------------ */
-#define ORC_NOQUANT 1 /* test switch: no quantisation anywhere (T3)       */
-#define ORC_WALK 128  /* keys per online-softmax tile of the walk          */
+#define ORC_NOQUANT 1 /* test switch: no quantisation anywhere (reduction to dense) */
+/* Alternative readings, kept only so that a test can measure how far the
+ * result moves between readings the pages leave open; the method's reading
+ * is flags = 0. */
+#define ORC_ALT_WALK128 2 /* update the running max once per 128 keys of the list */
+#define ORC_ALT_LSUM_P 4  /* row sum over the unquantised P instead of P~        */
 
 typedef struct {
   int N, d, block, nb, kc;
@@ -410,7 +414,11 @@ static void emul_qblock(const orc_head* H, int i, const int32_t* sel, double* ou
   const double rsd = 1.0 / sqrt((double)d);
   int n0 = i * block, n1 = n0 + block < N ? n0 + block : N;
   double* o = (double*)malloc(sizeof(double) * d);
-  double* sc = (double*)malloc(sizeof(double) * (ORC_WALK > block ? ORC_WALK : block));
+  /* The walk visits the selected key blocks of the list in ascending order,
+   * one block at a time: the running max is updated once per block and that
+   * block's P is quantised against it (ORC_ALT_WALK128: 128 keys at a time). */
+  const int per_tile = (H->flags & ORC_ALT_WALK128) && 128 / block > 1 ? 128 / block : 1;
+  double* sc = (double*)malloc(sizeof(double) * (size_t)per_tile * block);
   double* Hc = NULL;
   double* Zc = NULL;
   uint8_t* in_s = (uint8_t*)calloc(H->nb, 1);
@@ -431,55 +439,53 @@ static void emul_qblock(const orc_head* H, int i, const int32_t* sel, double* ou
     /* --- sparse softmax branch: online over the selected blocks, ascending --- */
     double m = -INFINITY, l = 0.0;
     for (int c = 0; c < d; ++c) o[c] = 0.0;
-    /* The walk takes the selected keys 128 at a time (ORC_WALK / block
-     * consecutive entries of the list): the running max is updated once per
-     * such tile and the tile's P is quantised against it. */
-    const int per_tile = ORC_WALK / block > 0 ? ORC_WALK / block : 1;
     for (int t0 = 0; t0 < kc; t0 += per_tile) {
       const int t1 = t0 + per_tile < kc ? t0 + per_tile : kc;
+      /* scores of the walk unit (one key block; keys past N are not scored) */
       double mj = -INFINITY;
       for (int t = t0; t < t1; ++t) {
-      int j = sel[t];
-      int k0 = j * block, k1 = k0 + block < N ? k0 + block : N;
-      for (int kk = k0; kk < k1; ++kk) {
-        double s;
-        if (H->flags & ORC_NOQUANT) {
-          double acc = 0.0;
-          for (int c = 0; c < d; ++c)
-            acc += (double)bf16_f32(H->q[(int64_t)n * d + c]) *
-                   ((double)bf16_f32(H->k[(int64_t)kk * d + c]) - (double)H->mu[c]);
-          s = acc * rsd;
-        } else {
-          int64_t acc = 0;
-          for (int c = 0; c < d; ++c)
-            acc += (int64_t)H->q8[(int64_t)n * d + c] * (int64_t)H->k8[(int64_t)kk * d + c];
-          s = (double)acc * (double)H->sq[n / ORC_QBLK] * (double)H->sk[kk / ORC_QBLK] * rsd;
+        const int j = sel[t];
+        const int k0 = j * block, k1 = k0 + block < N ? k0 + block : N;
+        for (int kk = k0; kk < k1; ++kk) {
+          double s;
+          if (H->flags & ORC_NOQUANT) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+              acc += (double)bf16_f32(H->q[(int64_t)n * d + c]) *
+                     ((double)bf16_f32(H->k[(int64_t)kk * d + c]) - (double)H->mu[c]);
+            s = acc * rsd;
+          } else {
+            int64_t acc = 0;
+            for (int c = 0; c < d; ++c)
+              acc += (int64_t)H->q8[(int64_t)n * d + c] * (int64_t)H->k8[(int64_t)kk * d + c];
+            s = (double)acc * (double)H->sq[n / ORC_QBLK] * (double)H->sk[kk / ORC_QBLK] * rsd;
+          }
+          sc[(t - t0) * block + (kk - k0)] = s;
+          if (s > mj) mj = s;
         }
-        sc[(t - t0) * block + (kk - k0)] = s;
-        if (s > mj) mj = s;
       }
-      }
-      double mnew = mj > m ? mj : m;
-      double alpha = exp(m - mnew); /* m = -inf on the first tile -> 0 */
+      /* new running max; O and l move to it (alpha = 0 on the first unit) */
+      const double mnew = mj > m ? mj : m;
+      const double alpha = exp(m - mnew);
       l *= alpha;
       for (int c = 0; c < d; ++c) o[c] *= alpha;
       for (int t = t0; t < t1; ++t) {
-      int j = sel[t];
-      int k0 = j * block, k1 = k0 + block < N ? k0 + block : N;
-      for (int kk = k0; kk < k1; ++kk) {
-        double p = exp(sc[(t - t0) * block + (kk - k0)] - mnew);
-        if (H->flags & ORC_NOQUANT) {
-          l += p;
-          for (int c = 0; c < d; ++c) o[c] += p * (double)bf16_f32(H->v[(int64_t)kk * d + c]);
-        } else {
-          /* P~ = e4m3(P*448): the FP8 probabilities; the row sum l is taken
-           * over the same quantised values that weight V. */
-          double pq = orc_e4m3_decode(orc_e4m3_encode((float)(p * 448.0)));
-          l += pq;
-          for (int c = 0; c < d; ++c)
-            o[c] += pq * orc_e4m3_decode(H->v8[(int64_t)kk * d + c]);
+        const int j = sel[t];
+        const int k0 = j * block, k1 = k0 + block < N ? k0 + block : N;
+        for (int kk = k0; kk < k1; ++kk) {
+          const double p = exp(sc[(t - t0) * block + (kk - k0)] - mnew);
+          if (H->flags & ORC_NOQUANT) {
+            l += p;
+            for (int c = 0; c < d; ++c) o[c] += p * (double)bf16_f32(H->v[(int64_t)kk * d + c]);
+          } else {
+            /* P~ = e4m3(P*448): the FP8 probabilities; the row sum l is taken
+             * over the same quantised values that weight V, so a constant V
+             * passes through unchanged. */
+            const double pq = orc_e4m3_decode(orc_e4m3_encode((float)(p * 448.0)));
+            l += (H->flags & ORC_ALT_LSUM_P) ? p * 448.0 : pq;
+            for (int c = 0; c < d; ++c) o[c] += pq * orc_e4m3_decode(H->v8[(int64_t)kk * d + c]);
+          }
         }
-      }
       }
       m = mnew;
     }

@@ -18,6 +18,10 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 NOQUANT = 1  # test switch: no quantisation anywhere (reduction to dense)
+# Alternative readings, only for measuring how far the result moves between
+# readings the pages leave open (the method's reading is flags = 0).
+ALT_WALK128 = 2  # running max updated once per 128 keys of the list
+ALT_LSUM_P = 4  # row sum over the unquantised P instead of P~
 
 
 def build(force: bool = False) -> str:

@@ -176,8 +176,9 @@ def test_external_mask_and_query_selection(orc):
         assert np.abs(out4[0, :64] - out[0, :64]).max() > 1e-4
 
 
-@pytest.mark.parametrize("block", [64, 128])
-def test_worked_walk_tile(orc, block):
+@pytest.mark.parametrize("block,flags", [(64, 0), (128, 0), (64, 2), (128, 2)])
+def test_worked_walk(orc, block, flags):
+    """The walk updates the running max after every selected key block (hand-derived, golden file)."""
     with open(os.path.join(GOLDEN, "worked_walk_tiles.json")) as f:
         g = json.load(f)
     N, d = g["N"], g["d"]
@@ -188,6 +189,18 @@ def test_worked_walk_tile(orc, block):
     v = torch.zeros(1, N, d)
     v[0, :64, :2] = torch.tensor(g["v_block0"])
     v[0, 64:, :2] = torch.tensor(g["v_block1"])
-    out, _ = orc.sagesla(q.bfloat16(), k.bfloat16(), v.bfloat16(), None, block, 1.0)
-    for (c, num, den) in g["expect"]:
-        np.testing.assert_allclose(out[0, :, c], num / den, rtol=0, atol=1e-12)
+    assert flags in (0, orc.ALT_WALK128)
+    out, _ = orc.sagesla(q.bfloat16(), k.bfloat16(), v.bfloat16(), None, block, 1.0, flags=flags)
+    if block == 64 and flags == 0:
+        # the key scale is fl32(delta/127) (scales are fp32), so c is taken with it
+        c = 127 * 127 * float(np.float32(g["delta"] / 127)) / (128 * np.sqrt(d))
+        assert abs(c - g["c"]) < 1e-7
+        alpha = np.exp(-2 * c)
+        v0, v1 = g["v_block0"], g["v_block1"]
+        for ch in range(2):
+            np.testing.assert_allclose(out[0, :, ch], (alpha * v0[ch] + v1[ch]) / (alpha + 1), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(out[0, :, 0], -0.695986, rtol=0, atol=1e-6)
+        assert np.all(out[0, :, 2:] == 0)
+    else:
+        for (c, num, den) in g["expect_128_keys"]:
+            np.testing.assert_allclose(out[0, :, c], num / den, rtol=0, atol=1e-12)
