@@ -1,43 +1,50 @@
 // k_flash.cu -- K5: block-sparse SageAttention-style flash kernel on tcgen05.
 //
-// For each query block i and each key block j of its top-k list (ascending),
-//   S = (q^ . k^) * s_q,i * s_k,j / sqrt(d)     INT8 x INT8 -> INT32 in TMEM
-//   online softmax, P~ = e4m3(448 * exp(S - running max))
-//   O += P~ . v^                                 FP8 x FP8 -> FP32 in TMEM
-// and finally O_s = (O / rowsum(P~)) * s_v (per channel).  Sources:
+// For each query block i, the key blocks of its top-k list are walked in
+// ascending order, one key block at a time:
+//   S = (q^ . k^) * s_q,i * s_k,j / sqrt(d)       INT8 x INT8 -> INT32 in TMEM
+//   running max m updated after the block; P~ = e4m3(448 * exp(S - m))
+//   O = O * exp(m_old - m) + P~ . v^               FP8 x FP8 -> FP32 in TMEM
+// and finally O_s = (O / rowsum(P~)) * s_v per channel.  Sources:
 // "揭秘TurboDiffusion：如何让视频生成实现百倍加速？" 支柱一 (INT8 attention with
 // smoothing on integer tensor cores) and 支柱二 (only the selected blocks are
 // computed exactly); 量子位 news 技术解密 1 (SageAttention2++).
 //
-// Roles on the SM (16 warps, 1 CTA/SM):
-//   warp 0     K producer: bulk copies of the Q^ and K^ tiles (pre-tiled in
-//              HBM by the quantiser, so one cp.async.bulk moves a whole tile);
-//   warp 1     QK^T issuer (one thread) and TMEM owner;
-//   warp 2     PV issuer (one thread) -- two issuers keep the tensor pipe fed
-//              while either of them waits;
-//   warp 3     V producer: bulk copies of the V^T tiles.  K and V have their
-//              own producers so a K copy never queues behind a V stage that
-//              the later PV step still holds;
-//   warps 4-11 softmax: two warps per TMEM lane quadrant, each owning one
-//              64-key sub-tile of the 128-key step of every row;
-//   warps 12-15 correction: one warp per quadrant; rescales O by
-//              exp(m_old - m_new) between PV steps, off the softmax path, and
-//              runs the epilogue.
-// Mode 64 (block 64): a CTA owns two query blocks A and B.  Their M=64
-//   accumulators share TMEM columns at lane offsets 0 and 16, so all 128
-//   lanes hold a row.  Each step takes two key blocks per query block (S tile
-//   N = 128); PV is M=64, N=144 (128 V channels + 16 rows of ones whose
-//   product is the row sum of P~).
-// Mode 128 (block 128): one query block of 128 rows per CTA, M = 128.
-// TMEM: S double buffer (2 x 128 cols) + O (144 cols) of 512 allocated.
+// Work unit: block 64 -- a pair of query blocks A, B (their M=64 accumulators
+// sit at TMEM lane offsets 0 and 16, so every lane holds a row); block 128 --
+// one 128-row query block (M=128).  The grid is persistent: one CTA per SM
+// walks units u = blockIdx.x, blockIdx.x + gridDim.x, ... (head-major, so the
+// SMs share the K^/V^ tiles of one or two heads in L2).
 //
-// Step hand-offs (s = step): S(s) -> s_full -> softmax(s) -> p_full(s) ->
-// correction(s) [waits PV(s-1)] -> s_free(s), o_ready(s) -> PV(s) -> o_done.
-// QK^T for step s+2 waits s_free(s) (its S buffer and alpha slot are then
-// free); P is triple-buffered, so the buffer softmax(s+3) writes was read by
-// PV(s), which correction(s+1) saw complete before s_free(s+1) released
-// QK^T(s+3).  Every parity wait below is at most one phase behind its
-// barrier (o_ready has the PV issuer as its only waiter).
+// Step: two 64-key halves g = 0, 1 -- at block 64 the list entries 2s and
+// 2s+1 (two walk blocks), at block 128 the two halves of list entry s (one
+// walk block).  QK^T of a step is one N=128 MMA chain per query block.
+// Softmax warpgroup g exponentiates half g; each thread owns one row and
+// reads the other half of its row too, so it knows both maxima without any
+// exchange.  Because the walk updates the running max after every walk
+// block, half g accumulates in its own TMEM accumulator O_g whose frame is
+// the running max after that half's block (at block 128 both frames are the
+// block's max): O_g is rescaled by exp(frame_old - frame_new) before its PV,
+// and the epilogue combines O_0 and O_1 in the final max.  PV is M=64/128,
+// N=136/144: 128 V channels plus rows of ones, so the row sum of P~ comes
+// out of the tensor core in column 128.
+//
+// Roles (16 warps, 1 CTA/SM):
+//   warp 0      K producer: Q^ tiles of each unit (double-buffered) and the
+//               K^ tiles of each step (2-stage ring), one bulk copy per tile;
+//   warp 1      QK^T issuer (one thread) and TMEM owner;
+//   warp 2      PV issuer (one thread);
+//   warp 3      V producer: V^T tiles (2-stage ring);
+//   warps 4-11  softmax: warpgroup g = 0 (warps 4-7), g = 1 (warps 8-11);
+//   warps 12-15 correction: rescales O_g between its PV steps, epilogue.
+// TMEM: S (128 columns, single buffer: QK^T of step s+1 waits until both
+// warpgroups have loaded S(s)), O_0 at column 128, O_1 at column 272.
+//
+// Barrier protocol (gs = global step of this CTA, b = gs & 1): every
+// per-step barrier a role can run ahead on is double-buffered by b, and each
+// chain of a step passes through p_empty (PV_g(gs-2) complete) before the
+// softmax publishes anything for step gs, so no parity wait is ever more
+// than one phase behind its barrier.  Every wait is bounded (watchdog).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -45,18 +52,14 @@ namespace sagesla {
 
 namespace {
 
-constexpr int kStages = 2;
-constexpr int kPBufs = 3;
-constexpr int kSoftThreads = 256;
-constexpr int kCorrThreads = 128;
-constexpr int kWarpSoft0 = 4, kWarpCorr0 = 12;
-constexpr int kThreads = 32 * 4 + kSoftThreads + kCorrThreads;  // 512
-constexpr int kVSlot = kTile + 1024;  // 8 KB V^T tile + 16 rows of ones (1 KB)
+constexpr int kThreads = 512;
+constexpr int kWarpLoadK = 0, kWarpQK = 1, kWarpPV = 2, kWarpLoadV = 3, kWarpSoft0 = 4, kWarpCorr0 = 12;
 constexpr uint32_t kOnesE4M3 = 0x38383838u;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;
-constexpr uint32_t kTmemCols = 512, kColS0 = 0, kColS1 = 128, kColO = 256;
-constexpr int kNO = 144;  // PV N: 128 channels + 16 ones
+constexpr float kRsqrtD = 0.08838834764831845f;  // 1/sqrt(128)
+constexpr uint32_t kTmemCols = 512, kColS = 0, kColO0 = 128, kColO1 = 272;
+constexpr uint32_t kP_LBO = 128, kP_SBO = 512;  // P~ tiles [rows][64 keys], K-major
 
 struct Params {
   const uint8_t* q8t;
@@ -68,42 +71,70 @@ struct Params {
   const int32_t* idx;
   __nv_bfloat16* out;
   int* wd;
-  int N, nb, nq, kc, nsteps;
-  int add_out;  // 1: out already holds the linear branch (bf16); add O_s to it
+  int N, nb, nq, kc;
+  int upb;     // units per head
+  int units;   // BH * upb
+  int nsteps;  // steps per unit
+  int add_out; // 1: out already holds the linear branch (bf16); add O_s to it
 };
 
 template <int MODE>
 struct Cfg {
-  // MODE 0: two query blocks (A,B) x two 64-key sub-tiles per step.
-  // MODE 1: one 128-row query block x one 128-key block per step.
+  static constexpr int kNO = MODE == 0 ? 136 : 144;  // PV N: 128 channels + ones (M=128 needs N % 16 == 0)
+  static constexpr int kOnes = (kNO - 128) * 64;     // bytes of ones rows under a V^T tile
+  static constexpr int kVSlot = kTile + kOnes;
+  static constexpr int kSlots = MODE == 0 ? 4 : 2;   // K^ / V^T tiles per step
   static constexpr int kQBytes = 2 * kTile;
-  static constexpr int kKStage = (MODE == 0 ? 4 : 2) * kTile;
-  static constexpr int kVStage = (MODE == 0 ? 4 : 2) * kVSlot;
-  static constexpr int kPBuf = 2 * kTile;  // 128 rows x 128 keys (two 64-row halves in mode 0)
+  static constexpr int kKStage = kSlots * kTile;
+  static constexpr int kVStage = kSlots * kVSlot;
+  static constexpr int kPTile = 8192;                // 128 rows x 64 keys
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kStages * kKStage;
-  static constexpr int kOffP = kOffV + kStages * kVStage;
-  static constexpr int kOffBar = kOffP + kPBufs * kPBuf;
-  static constexpr int kBarBytes = 512;
-  static constexpr int kOffX = kOffBar + kBarBytes;      // row-max exchange [2][2][128] f32
-  static constexpr int kOffA = kOffX + 2 * 2 * 128 * 4;  // alpha [2][128] f32
-  static constexpr int kSmem = kOffA + 2 * 128 * 4 + 1024;  // + alignment slack
+  static constexpr int kOffK = kOffQ + 2 * kQBytes;
+  static constexpr int kOffV = kOffK + 2 * kKStage;
+  static constexpr int kOffP = kOffV + 2 * kVStage;  // [parity b][half g]
+  static constexpr int kOffA = kOffP + 4 * kPTile;   // alpha [g][b][128] f32
+  static constexpr int kOffF = kOffA + 2 * 2 * 128 * 4;  // final frames [unit parity][g][128] f32
+  static constexpr int kOffBar = kOffF + 2 * 2 * 128 * 4;
+  static constexpr int kSmem = kOffBar + 512 + 1024;  // + alignment slack
 };
 
 struct Bars {
-  uint64_t q_full;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_ready, o_done;
-  uint64_t s_free[2];
-  uint64_t fin;
-  uint64_t xbar[4][2];  // row-max exchange between the two softmax warps of a quadrant
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[2], k_empty[2];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full, s_free;
+  uint64_t a_ready[2][4][2];  // [g][quadrant][b]: alpha of the quadrant's rows published
+  uint64_t p_full[2][2];      // [g][b]: P~ stored
+  uint64_t p_empty[2][2];     // [g][b]: PV that read the P~ buffer complete
+  uint64_t o_ready[2][2];     // [g][b]: O_g rescaled, PV_g may accumulate
+  uint64_t o_done[2];         // [g]: PV_g of the step complete
+  uint64_t fin;               // every MMA of both issuers complete
   uint32_t tmem;
   int abort;
 };
 static_assert(sizeof(Bars) <= 512, "barrier block");
+
+struct Unit {
+  int bh, iA, iB;
+  bool hasB;
+};
+
+template <int MODE>
+__device__ __forceinline__ Unit unit_of(const Params& p, int u) {
+  Unit x;
+  x.bh = u / p.upb;
+  const int pi = u - x.bh * p.upb;
+  if (MODE == 0) {
+    x.iA = 2 * pi;
+    x.iB = 2 * pi + 1;
+    x.hasB = x.iB < p.nb;
+  } else {
+    x.iA = pi;
+    x.iB = -1;
+    x.hasB = false;
+  }
+  return x;
+}
 
 // key block (mask block index) of list entry t for query block i
 __device__ __forceinline__ int list_at(const Params& p, int bh, int i, int t) {
@@ -118,445 +149,504 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
-  float* xch = reinterpret_cast<float*>(smem + C::kOffX);
   float* alpha_s = reinterpret_cast<float*>(smem + C::kOffA);
+  float* frame_s = reinterpret_cast<float*>(smem + C::kOffF);
   volatile int* abort = &bars->abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.y;
-  // Query blocks of this CTA (mask-block indices).
-  const int iA = MODE == 0 ? 2 * (int)blockIdx.x : (int)blockIdx.x;
-  const int iB = MODE == 0 ? 2 * (int)blockIdx.x + 1 : -1;
-  const bool hasB = MODE == 0 && iB < p.nb;
   const int nsteps = p.nsteps;
 
   if (tid == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->k_empty[s], 1);
-      mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->v_empty[s], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->q_full[x], 1);
+      mbar_init(&bars->q_empty[x], 1);
+      mbar_init(&bars->k_full[x], 1);
+      mbar_init(&bars->k_empty[x], 1);
+      mbar_init(&bars->v_full[x], 1);
+      mbar_init(&bars->v_empty[x], 1);
+      mbar_init(&bars->o_done[x], 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&bars->p_full[x][b], 4);
+        mbar_init(&bars->p_empty[x][b], 1);
+        mbar_init(&bars->o_ready[x][b], 4);
+        for (int w = 0; w < 4; ++w) mbar_init(&bars->a_ready[x][w][b], 1);
+      }
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], kSoftThreads);
-    }
-    mbar_init(&bars->o_ready, kCorrThreads);
-    mbar_init(&bars->s_free[0], kCorrThreads);
-    mbar_init(&bars->s_free[1], kCorrThreads);
-    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, 8);
     mbar_init(&bars->fin, 2);
-    for (int qq = 0; qq < 4; ++qq)
-      for (int b = 0; b < 2; ++b) mbar_init(&bars->xbar[qq][b], 64);
     bars->abort = 0;
     mbar_fence_init();
   }
-  // Rows of ones under every V slot (PV's extra 16 output columns = row sum).
-  for (int e = tid; e < kStages * (C::kVStage / kVSlot) * 64; e += kThreads) {
-    const int slot = e / 64, w = e % 64;
-    *reinterpret_cast<uint4*>(smem + C::kOffV + slot * kVSlot + kTile + w * 16) =
+  // Rows of ones under every V^T slot (PV's extra output columns = row sum of P~).
+  constexpr int kOnesWords = C::kOnes / 16;
+  for (int e = tid; e < 2 * C::kSlots * kOnesWords; e += kThreads) {
+    const int slot = e / kOnesWords, w = e % kOnesWords;
+    *reinterpret_cast<uint4*>(smem + C::kOffV + slot * C::kVSlot + kTile + w * 16) =
         make_uint4(kOnesE4M3, kOnesE4M3, kOnesE4M3, kOnesE4M3);
   }
   fence_proxy_async_smem();
-  if (warp == 1) tmem_alloc(&bars->tmem, kTmemCols);
+  if (warp == kWarpQK) tmem_alloc(&bars->tmem, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
 
-  if (warp == 0 || warp == 3) {
-    // ------------------------- K and V producers --------------------------
-    // warp 0 copies Q^ and the K^ tiles of each step, warp 3 the V^T tiles.
-    // The list entries of step s+1 are read before the wait for stage s, so
-    // their latency hides behind it.
+  if (warp == kWarpLoadK || warp == kWarpLoadV) {
+    // ---------------------------- producers -------------------------------
     if (lane == 0) {
-      const bool is_k = warp == 0;
-      const size_t head_tiles = (size_t)bh * p.nq;
-      if (is_k) {
-        mbar_expect_tx(&bars->q_full, C::kQBytes);
-        if (MODE == 0) {
-          bulk_g2s(smem + C::kOffQ, p.q8t + (head_tiles + iA) * kTile, kTile, &bars->q_full);
-          const int ib = hasB ? iB : iA;  // keep the transaction count fixed
-          bulk_g2s(smem + C::kOffQ + kTile, p.q8t + (head_tiles + ib) * kTile, kTile, &bars->q_full);
-        } else {
-          bulk_g2s(smem + C::kOffQ, p.q8t + (head_tiles + 2 * iA) * kTile, 2 * kTile, &bars->q_full);
-        }
-      }
+      const bool is_k = warp == kWarpLoadK;
       uint64_t* full = is_k ? bars->k_full : bars->v_full;
       uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
       const uint8_t* src = is_k ? p.k8t : p.v8t;
-      auto entries = [&](int s, int (&jj)[2][2]) {
-        jj[0][0] = jj[0][1] = jj[1][0] = jj[1][1] = -1;
-        if (s >= nsteps) return;
-        if (MODE == 0) {
-          const int nsub = min(2, p.kc - 2 * s);
-          for (int x = 0; x < 2; ++x) {
-            const int i = (x == 0 || !hasB) ? iA : iB;
-            for (int u = 0; u < nsub; ++u) jj[x][u] = list_at(p, bh, i, 2 * s + u);
-          }
-        } else {
-          jj[0][0] = list_at(p, bh, iA, s);
-        }
-      };
-      int jn[2][2];
-      entries(0, jn);
-      int issued = 0;  // steps whose copies were issued
-      for (int s = 0; s < nsteps && !*abort; ++s) {
-        const int st = s % kStages;
-        int jj[2][2];
-        for (int x = 0; x < 2; ++x)
-          for (int u = 0; u < 2; ++u) jj[x][u] = jn[x][u];
-        entries(s + 1, jn);
-        if (s >= kStages && !mbar_wait(&empty[st], ((s / kStages) - 1) & 1, abort, p.wd)) break;
-        if (MODE == 0) {
-          const int nsub = min(2, p.kc - 2 * s);
-          mbar_expect_tx(&full[st], 2 * nsub * kTile);
-          for (int x = 0; x < 2; ++x)
-            for (int u = 0; u < nsub; ++u) {
-              uint8_t* dst = is_k ? smem + C::kOffK + st * C::kKStage + (2 * x + u) * kTile
-                                  : smem + C::kOffV + st * C::kVStage + (2 * x + u) * kVSlot;
-              bulk_g2s(dst, src + (head_tiles + jj[x][u]) * kTile, kTile, &full[st]);
-            }
-        } else {
-          const int j = jj[0][0];
-          mbar_expect_tx(&full[st], 2 * kTile);
-          if (is_k) {
-            bulk_g2s(smem + C::kOffK + st * C::kKStage, src + (head_tiles + 2 * j) * kTile, 2 * kTile, &full[st]);
+      const int stage_bytes = is_k ? C::kKStage : C::kVStage;
+      const int slot_bytes = is_k ? kTile : C::kVSlot;
+      uint8_t* ring = smem + (is_k ? C::kOffK : C::kOffV);
+      int gs = 0, ui = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ui) {
+        const Unit un = unit_of<MODE>(p, u);
+        const size_t head_tiles = (size_t)un.bh * p.nq;
+        if (is_k) {
+          const int qb = ui & 1;
+          if (ui >= 2 && !(ok = mbar_wait(&bars->q_empty[qb], ((ui >> 1) - 1) & 1, abort, p.wd))) break;
+          uint8_t* qd = smem + C::kOffQ + qb * C::kQBytes;
+          mbar_expect_tx(&bars->q_full[qb], C::kQBytes);
+          if (MODE == 0) {
+            bulk_g2s(qd, p.q8t + (head_tiles + un.iA) * kTile, kTile, &bars->q_full[qb]);
+            bulk_g2s(qd + kTile, p.q8t + (head_tiles + (un.hasB ? un.iB : un.iA)) * kTile, kTile, &bars->q_full[qb]);
           } else {
-            uint8_t* vd = smem + C::kOffV + st * C::kVStage;
-            bulk_g2s(vd, src + (head_tiles + 2 * j) * kTile, kTile, &full[st]);
-            bulk_g2s(vd + kVSlot, src + (head_tiles + 2 * j + 1) * kTile, kTile, &full[st]);
+            bulk_g2s(qd, p.q8t + (head_tiles + 2 * un.iA) * kTile, 2 * kTile, &bars->q_full[qb]);
           }
         }
-        issued = s + 1;
+        for (int s = 0; s < nsteps; ++s, ++gs) {
+          // Tiles of this step: slot (2X + g) = list entry 2s+g of query block X (block 64);
+          // slots 0, 1 = the two 64-key tiles of list entry s (block 128).
+          int tiles[4];
+          int nt = 0;
+          if (MODE == 0) {
+            for (int x = 0; x < 2; ++x)
+              for (int g = 0; g < 2; ++g) {
+                const int t = 2 * s + g;
+                tiles[2 * x + g] = (t < p.kc && (x == 0 || un.hasB)) ? list_at(p, un.bh, x ? un.iB : un.iA, t) : -1;
+                nt += tiles[2 * x + g] >= 0;
+              }
+          } else {
+            const int j = list_at(p, un.bh, un.iA, s);
+            tiles[0] = 2 * j;
+            tiles[1] = 2 * j + 1;
+            nt = 2;
+          }
+          const int st = gs & 1;
+          if (gs >= 2 && !(ok = mbar_wait(&empty[st], ((gs >> 1) - 1) & 1, abort, p.wd))) break;
+          mbar_expect_tx(&full[st], nt * kTile);
+          for (int x = 0; x < C::kSlots; ++x)
+            if (tiles[x] >= 0)
+              bulk_g2s(ring + st * stage_bytes + x * slot_bytes, src + (head_tiles + tiles[x]) * kTile, kTile,
+                       &full[st]);
+        }
       }
       // Drain: every copy issued must land before the CTA may exit.
-      if (is_k) mbar_wait_drain(&bars->q_full, 0, p.wd);
-      for (int s = max(0, issued - kStages); s < issued; ++s)
-        mbar_wait_drain(&full[s % kStages], (s / kStages) & 1, p.wd);
+      for (int g2 = max(0, gs - 2); g2 < gs; ++g2) mbar_wait_drain(&full[g2 & 1], (g2 >> 1) & 1, p.wd);
+      if (is_k)
+        for (int u2 = max(0, ui - 2); u2 < ui; ++u2) mbar_wait_drain(&bars->q_full[u2 & 1], (u2 >> 1) & 1, p.wd);
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpQK) {
     // ------------------------------ QK^T issuer ---------------------------
     if (lane == 0) {
-      const uint64_t dqk = smem_desc(smem, kQK_LBO, kQK_SBO);
-      bool ok = mbar_wait(&bars->q_full, 0, abort, p.wd);
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int st = s % kStages;
-        if (!(ok = mbar_wait(&bars->k_full[st], (s / kStages) & 1, abort, p.wd))) break;
-        // S buffer s&1 and alpha slot s&1 are free once step s-2 is corrected.
-        if (s >= 2) {
-          if (!(ok = mbar_wait(&bars->s_free[s & 1], ((s - 2) >> 1) & 1, abort, p.wd))) break;
+      const uint64_t dq = smem_desc(smem, kQK_LBO, kQK_SBO);
+      int gs = 0, ui = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ui) {
+        const Unit un = unit_of<MODE>(p, u);
+        const int qb = ui & 1;
+        if (!(ok = mbar_wait(&bars->q_full[qb], (ui >> 1) & 1, abort, p.wd))) break;
+        const uint32_t qoff = C::kOffQ + qb * C::kQBytes;
+        for (int s = 0; s < nsteps; ++s, ++gs) {
+          const int st = gs & 1;
+          if (!(ok = mbar_wait(&bars->k_full[st], (gs >> 1) & 1, abort, p.wd))) break;
+          if (gs > 0 && !(ok = mbar_wait(&bars->s_free, (gs - 1) & 1, abort, p.wd))) break;
           tc_fence_after();
-        }
-        const uint32_t dS = tmem + ((s & 1) ? kColS1 : kColS0);
-        const uint32_t koff = C::kOffK + st * C::kKStage;
-        if (MODE == 0) {
-          const uint32_t id = p.kc - 2 * s >= 2 ? idesc_i8(64, 128) : idesc_i8(64, 64);
+          const uint32_t koff = C::kOffK + st * C::kKStage;
+          if (MODE == 0) {
+            const uint32_t id = 2 * s + 1 < p.kc ? idesc_i8(64, 128) : idesc_i8(64, 64);
 #pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (x == 1 && !hasB) break;
-            const uint32_t d = dS + ((uint32_t)(x * 16) << 16);
+            for (int x = 0; x < 2; ++x) {
+              if (x == 1 && !un.hasB) break;
+              const uint32_t d = tmem + kColS + ((uint32_t)(x * 16) << 16);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_i8(d, desc_at(dq, qoff + x * kTile + kk * 256), desc_at(dq, koff + 2 * x * kTile + kk * 256), id,
+                       kk > 0);
+            }
+          } else {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_i8(d, desc_at(dqk, C::kOffQ + x * kTile + kk * 256), desc_at(dqk, koff + 2 * x * kTile + kk * 256), id,
+              mma_i8(tmem + kColS, desc_at(dq, qoff + kk * 256), desc_at(dq, koff + kk * 256), idesc_i8(128, 128),
                      kk > 0);
           }
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_i8(dS, desc_at(dqk, C::kOffQ + kk * 256), desc_at(dqk, koff + kk * 256), idesc_i8(128, 128), kk > 0);
+          mma_commit(&bars->s_full);
+          mma_commit(&bars->k_empty[st]);
         }
-        mma_commit(&bars->s_full[s & 1]);
-        mma_commit(&bars->k_empty[st]);
+        if (ok) mma_commit(&bars->q_empty[qb]);
       }
       mma_commit(&bars->fin);
     }
-  } else if (warp == 2) {
+  } else if (warp == kWarpPV) {
     // ------------------------------ PV issuer -----------------------------
     if (lane == 0) {
-      const uint64_t dqk = smem_desc(smem, kQK_LBO, kQK_SBO);
+      const uint64_t dp = smem_desc(smem, kP_LBO, kP_SBO);
       const uint64_t dv = smem_desc(smem, kV_LBO, kV_SBO);
-      const uint32_t id_pv = idesc_e4m3(MODE == 0 ? 64 : 128, kNO);
+      const uint32_t id = idesc_e4m3(MODE == 0 ? 64 : 128, C::kNO);
+      int gs = 0;
       bool ok = true;
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int st = s % kStages;
-        if (!(ok = mbar_wait(&bars->v_full[st], (s / kStages) & 1, abort, p.wd))) break;
-        if (!(ok = mbar_wait(&bars->o_ready, s & 1, abort, p.wd))) break;
-        tc_fence_after();
-        const uint32_t voff = C::kOffV + st * C::kVStage;
-        const uint32_t poff = C::kOffP + (s % kPBufs) * C::kPBuf;
-        if (MODE == 0) {
-          const int nk = p.kc - 2 * s >= 2 ? 4 : 2;
+      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+        const Unit un = unit_of<MODE>(p, u);
+        for (int s = 0; s < nsteps; ++s, ++gs) {
+          const int st = gs & 1, b = gs & 1, ph = (gs >> 1) & 1;
+          if (!(ok = mbar_wait(&bars->v_full[st], ph, abort, p.wd))) break;
+          for (int g = 0; g < 2; ++g) {
+            if (!(ok = mbar_wait(&bars->p_full[g][b], ph, abort, p.wd))) break;
+            if (!(ok = mbar_wait(&bars->o_ready[g][b], ph, abort, p.wd))) break;
+            tc_fence_after();
+            const bool has = MODE == 0 ? 2 * s + g < p.kc : true;
+            if (has) {
+              const uint32_t o = tmem + (g ? kColO1 : kColO0);
+              const uint32_t poff = C::kOffP + (2 * b + g) * C::kPTile;
+              const uint32_t voff = C::kOffV + st * C::kVStage;
 #pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (x == 1 && !hasB) break;
-            const uint32_t d = tmem + kColO + ((uint32_t)(x * 16) << 16);
+              for (int x = 0; x < (MODE == 0 ? 2 : 1); ++x) {
+                if (x == 1 && !un.hasB) break;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              if (kk >= nk) break;
-              mma_e4m3(d, desc_at(dqk, poff + x * kTile + kk * 256),
-                       desc_at(dv, voff + (2 * x + (kk >> 1)) * kVSlot + (kk & 1) * 256), id_pv, (s > 0 || kk > 0));
+                for (int kk = 0; kk < 2; ++kk)
+                  mma_e4m3(o + ((uint32_t)(x * 16) << 16), desc_at(dp, poff + x * 4096 + kk * 256),
+                           desc_at(dv, voff + (MODE == 0 ? 2 * x + g : g) * C::kVSlot + kk * 256), id,
+                           (s > 0 || kk > 0));
+              }
             }
+            mma_commit(&bars->o_done[g]);
+            mma_commit(&bars->p_empty[g][b]);
           }
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_e4m3(tmem + kColO, desc_at(dqk, poff + kk * 256), desc_at(dv, voff + (kk >> 1) * kVSlot + (kk & 1) * 256),
-                     id_pv, (s > 0 || kk > 0));
+          if (!ok) break;
+          mma_commit(&bars->v_empty[st]);
         }
-        mma_commit(&bars->o_done);
-        mma_commit(&bars->v_empty[st]);
       }
       mma_commit(&bars->fin);
     }
   } else if (warp < kWarpCorr0) {
     // ------------------------------ softmax -------------------------------
-    // Two warps per TMEM lane quadrant: group g = 0 owns the first 64-key
-    // sub-tile of each step, group 1 the second.  The two threads of a row
-    // trade their sub-tile maxima through a double-buffered shared slot and a
-    // per-quadrant mbarrier (bounded wait).
     const int g = (warp - kWarpSoft0) >> 2;
-    const int q = warp & 3;
-    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    int row, i, qtile;
-    bool active;
-    if (MODE == 0) {
-      const bool isB = lane >= 16;
-      row = 16 * q + (lane & 15);
-      i = isB ? iB : iA;
-      active = isB ? hasB : true;
-      qtile = i;
-    } else {
-      row = 32 * q + lane;
-      i = iA;
-      active = true;
-      qtile = 2 * iA + (row >> 6);
-    }
-    const size_t tb = (size_t)bh * p.nq;
-    const float c0 = active ? __ldg(p.sq + tb + qtile) * (kLog2e * 0.08838834764831845f) : 0.f;
-    const int xrow = 32 * q + lane;  // TMEM lane of this row
-    uint8_t* prow_base = smem + C::kOffP + (MODE == 0 && lane >= 16 ? kTile : 0);
-    // Metadata of this thread's sub-tile, one step ahead of use.
-    auto tile_of = [&](int s) -> int {
+    const int w = warp & 3;  // TMEM lane quadrant
+    const uint32_t lane_base = (uint32_t)(32 * w) << 16;
+    const int L = 32 * w + lane;  // TMEM lane of this row
+    int gs = 0, ui = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ui) {
+      const Unit un = unit_of<MODE>(p, u);
+      int r, i, qtile;
+      bool active;
       if (MODE == 0) {
-        const int t = 2 * s + g;
-        return (active && t < p.kc) ? list_at(p, bh, i, t) : -1;
-      }
-      return 2 * list_at(p, bh, i, s) + g;
-    };
-    int kt_cur = tile_of(0);
-    float sk_cur = kt_cur >= 0 ? __ldg(p.sk + tb + kt_cur) : 0.f;
-    int kt_next = nsteps > 1 ? tile_of(1) : -1;
-    float m_run = -INFINITY;
-    for (int s = 0; s < nsteps; ++s) {
-      bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[s & 1], (s >> 1) & 1, abort, p.wd));
-      if (!ok) break;
-      tc_fence_after();
-      const int nsub = MODE == 0 ? min(2, p.kc - 2 * s) : 2;
-      const bool have = g < nsub && active && kt_cur >= 0;
-      const int nvalid = have ? max(0, min(64, p.N - kt_cur * 64)) : 0;
-      const float cu = c0 * sk_cur;
-      uint32_t acc[64];
-      if (g < nsub) {
-        const uint32_t sbase = tmem + lane_base + ((s & 1) ? kColS1 : kColS0) + 64 * g;
-        SAGESLA_TMEM_LD16(sbase + 0, acc + 0);
-        SAGESLA_TMEM_LD16(sbase + 16, acc + 16);
-        SAGESLA_TMEM_LD16(sbase + 32, acc + 32);
-        SAGESLA_TMEM_LD16(sbase + 48, acc + 48);
-        tmem_ld_wait();
-      }
-      int mx = INT_MIN;
-      if (nvalid == 64) {
-        int m2[2] = {INT_MIN, INT_MIN};  // two chains of three-input maxima
-#pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-          m2[0] = __vimax3_s32(m2[0], (int)acc[c], (int)acc[c + 1]);
-          m2[1] = __vimax3_s32(m2[1], (int)acc[c + 2], (int)acc[c + 3]);
-        }
-        mx = max(m2[0], m2[1]);
+        const bool isB = lane >= 16;
+        r = 16 * w + (lane & 15);
+        i = isB ? un.iB : un.iA;
+        active = isB ? un.hasB : true;
+        qtile = i;
       } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c < nvalid) mx = max(mx, (int)acc[c]);
+        r = L;
+        i = un.iA;
+        active = true;
+        qtile = 2 * un.iA + (r >> 6);
       }
-      const float mu = nvalid > 0 ? __int2float_rn(mx) * cu : -INFINITY;
-      xch[((s & 1) * 2 + g) * 128 + xrow] = mu;
-      mbar_arrive(&bars->xbar[q][s & 1]);
-      // Prefetch the key scale of the next step (its list entry arrived) only
-      // now: an mbarrier arrive has release semantics and would wait for
-      // these global loads to complete.
-      const float sk_next = kt_next >= 0 ? __ldg(p.sk + tb + kt_next) : 0.f;
-      const int kt_after = (s + 2 < nsteps) ? tile_of(s + 2) : -1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->xbar[q][s & 1], (s >> 1) & 1, abort, p.wd));
-      if (!ok) break;
-      const float mo = xch[((s & 1) * 2 + (g ^ 1)) * 128 + xrow];
-      const float m_new = fmaxf(m_run, fmaxf(mu, mo));
-      if (g == 0) alpha_s[(s & 1) * 128 + xrow] = (m_run == -INFINITY) ? 1.f : ex2(m_run - m_new);
-      // exponent of 448*P: (acc - max_u) * c_u + (m_u - m_new) + log2(448); the
-      // integer difference is exact, so values near the running max keep full
-      // precision however large the scores are.
-      // Exponent of 448*P~: S*log2(e) - m_new + log2(448), one fused
-      // multiply-add per key on the integer score (exact in fp32: |acc| <
-      // 2^24), two keys per f32x2 instruction; keys past the sequence end
-      // (last key block) get P~ = 0.
-      uint8_t* pbuf = prow_base + (s % kPBufs) * C::kPBuf;
-      const float kk = kLog2_448 - m_new;
-      const uint64_t cc = f32x2_pack(cu, cu), ko = f32x2_pack(kk, kk);
-      // (two copies of the loop: the masked one only for a ragged last block)
-      if (g < nsub && nvalid == 64) {
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {  // 16-key chunks
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float x[4];
-#pragma unroll
-            for (int z = 0; z < 4; z += 2) {
-              const int c = 16 * ch + 4 * e + z;
-              const uint64_t d =
-                  f32x2_fma(f32x2_pack(__int2float_rn((int)acc[c]), __int2float_rn((int)acc[c + 1])), cc, ko);
-              float a, b;
-              f32x2_unpack(d, a, b);
-              x[z] = ex2(a);
-              x[z + 1] = ex2(b);
-            }
-            w[e] = __byte_perm(e4m3x2(x[0], x[1]), e4m3x2(x[2], x[3]), 0x5410);
-          }
-          *reinterpret_cast<uint4*>(pbuf + kmajor_off(row, 64 * g + 16 * ch, kQK_LBO, kQK_SBO)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+      const size_t tb = (size_t)un.bh * p.nq;
+      const float c0 = active ? __ldg(p.sq + tb + qtile) * (kLog2e * kRsqrtD) : 0.f;
+      uint8_t* prow = smem + C::kOffP + g * C::kPTile + (MODE == 0 && lane >= 16 ? 4096 : 0);
+      float m_all = -INFINITY, frame = -INFINITY;
+      // Key tiles (64 keys each) of this row's own half and of the other half
+      // of step s, and their scales; fetched one step ahead of use.
+      auto tiles_of = [&](int s, int& t_own, int& t_oth) {
+        t_own = t_oth = -1;
+        if (s >= nsteps || !active) return;
+        if (MODE == 0) {
+          const int e0 = 2 * s + g, e1 = 2 * s + 1 - g;
+          if (e0 < p.kc) t_own = list_at(p, un.bh, i, e0);
+          if (e1 < p.kc) t_oth = list_at(p, un.bh, i, e1);
+        } else {
+          const int j = list_at(p, un.bh, i, s);
+          t_own = 2 * j + g;
+          t_oth = 2 * j + 1 - g;
         }
-      } else if (g < nsub) {
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {  // 16-key chunks
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float x[4];
-#pragma unroll
-            for (int z = 0; z < 4; z += 2) {
-              const int c = 16 * ch + 4 * e + z;
-              const uint64_t d =
-                  f32x2_fma(f32x2_pack(__int2float_rn((int)acc[c]), __int2float_rn((int)acc[c + 1])), cc, ko);
-              float a, b;
-              f32x2_unpack(d, a, b);
-              x[z] = ex2(a);
-              x[z + 1] = ex2(b);
-            }
-#pragma unroll
-            for (int z = 0; z < 4; ++z)
-              if (16 * ch + 4 * e + z >= nvalid) x[z] = 0.f;
-            w[e] = __byte_perm(e4m3x2(x[0], x[1]), e4m3x2(x[2], x[3]), 0x5410);
-          }
-          *reinterpret_cast<uint4*>(pbuf + kmajor_off(row, 64 * g + 16 * ch, kQK_LBO, kQK_SBO)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+      };
+      auto nvalid = [&](int t) { return t >= 0 ? max(0, min(64, p.N - 64 * t)) : 0; };
+      int t_own, t_oth;
+      tiles_of(0, t_own, t_oth);
+      float sk_own = nvalid(t_own) > 0 ? __ldg(p.sk + tb + t_own) : 0.f;
+      float sk_oth = nvalid(t_oth) > 0 ? __ldg(p.sk + tb + t_oth) : 0.f;
+      int n_own, n_oth;
+      tiles_of(1, n_own, n_oth);
+      for (int s = 0; s < nsteps; ++s, ++gs) {
+        const int b = gs & 1;
+        const int nv_own = nvalid(t_own), nv_oth = nvalid(t_oth);
+        const float cu_own = c0 * sk_own, cu_oth = c0 * sk_oth;
+        // The P~ buffer b was read by PV_g(gs-2); waiting for it first keeps
+        // every barrier this warp publishes on at most one phase ahead.
+        if (gs >= 2) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars->p_empty[g][b], ((gs >> 1) - 1) & 1, abort, p.wd));
+          if (!ok) break;
         }
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, gs & 1, abort, p.wd));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t acc[64];
+        int mx_oth = INT_MIN;
+        {
+          const uint32_t so = tmem + lane_base + kColS + 64 * g;
+          const uint32_t sx = tmem + lane_base + kColS + 64 * (1 - g);
+          uint32_t t[32];
+          SAGESLA_TMEM_LD16(so + 0, acc + 0);
+          SAGESLA_TMEM_LD16(so + 16, acc + 16);
+          SAGESLA_TMEM_LD16(so + 32, acc + 32);
+          SAGESLA_TMEM_LD16(so + 48, acc + 48);
+          SAGESLA_TMEM_LD16(sx + 0, t + 0);
+          SAGESLA_TMEM_LD16(sx + 16, t + 16);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c < nv_oth) mx_oth = max(mx_oth, (int)t[c]);
+          SAGESLA_TMEM_LD16(sx + 32, t + 0);
+          SAGESLA_TMEM_LD16(sx + 48, t + 16);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c + 32 < nv_oth) mx_oth = max(mx_oth, (int)t[c]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free);
+        // Scales of the next step (its list entries arrived during this one)
+        // and the list entries of the step after; issued only now, since an
+        // mbarrier arrive has release semantics and would wait for them.
+        const float sk_own_n = nvalid(n_own) > 0 ? __ldg(p.sk + tb + n_own) : 0.f;
+        const float sk_oth_n = nvalid(n_oth) > 0 ? __ldg(p.sk + tb + n_oth) : 0.f;
+        int a_own, a_oth;
+        tiles_of(s + 2, a_own, a_oth);
+        int mx_own = INT_MIN;
+        if (nv_own == 64) {
+          int m2[2] = {INT_MIN, INT_MIN};
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            m2[0] = __vimax3_s32(m2[0], (int)acc[c], (int)acc[c + 1]);
+            m2[1] = __vimax3_s32(m2[1], (int)acc[c + 2], (int)acc[c + 3]);
+          }
+          mx_own = max(m2[0], m2[1]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < nv_own) mx_own = max(mx_own, (int)acc[c]);
+        }
+        const float mf_own = nv_own > 0 ? __int2float_rn(mx_own) * cu_own : -INFINITY;
+        const float mf_oth = nv_oth > 0 ? __int2float_rn(mx_oth) * cu_oth : -INFINITY;
+        // Frame of O_g after this step: at block 64 half 0 is walk block 2s
+        // (max over the blocks so far and this one), half 1 is block 2s+1
+        // (which has also seen block 2s); at block 128 both are the block's max.
+        float fnew = (MODE == 0 && g == 0) ? fmaxf(m_all, mf_own) : fmaxf(m_all, fmaxf(mf_own, mf_oth));
+        m_all = fmaxf(m_all, fmaxf(mf_own, mf_oth));
+        if (nv_own == 0) fnew = frame;  // no block for this half: O_g keeps its frame
+        const float alpha = (frame == -INFINITY || fnew == -INFINITY) ? 1.f : ex2(frame - fnew);
+        frame = fnew;
+        alpha_s[(g * 2 + b) * 128 + L] = alpha;
+        if (s == nsteps - 1) frame_s[((ui & 1) * 2 + g) * 128 + L] = frame;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->a_ready[g][w][b]);
+        // P~ of the own half: exponent of 448*P = S*c - frame + log2(448), one
+        // fused multiply-add per key, two keys per f32x2 instruction; keys
+        // past the sequence end get P~ = 0.
+        uint8_t* pbuf = prow + 2 * b * C::kPTile;
+        // (block 128: a half past the sequence end still feeds the PV, with P~ = 0)
+        if (nv_own > 0 || (MODE == 1 && active)) {
+          const float kk = kLog2_448 - frame;
+          const uint64_t cc = f32x2_pack(cu_own, cu_own), ko = f32x2_pack(kk, kk);
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float x[4];
+#pragma unroll
+              for (int z = 0; z < 4; z += 2) {
+                const int c = 16 * ch + 4 * e + z;
+                const uint64_t dd =
+                    f32x2_fma(f32x2_pack(__int2float_rn((int)acc[c]), __int2float_rn((int)acc[c + 1])), cc, ko);
+                float a0, a1;
+                f32x2_unpack(dd, a0, a1);
+                x[z] = ex2(a0);
+                x[z + 1] = ex2(a1);
+              }
+              if (nv_own < 64) {
+#pragma unroll
+                for (int z = 0; z < 4; ++z)
+                  if (16 * ch + 4 * e + z >= nv_own) x[z] = 0.f;
+              }
+              wv[e] = __byte_perm(e4m3x2(x[0], x[1]), e4m3x2(x[2], x[3]), 0x5410);
+            }
+            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, 16 * ch, kP_LBO, kP_SBO)) =
+                make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[g][b]);
+        t_own = n_own;
+        t_oth = n_oth;
+        sk_own = sk_own_n;
+        sk_oth = sk_oth_n;
+        n_own = a_own;
+        n_oth = a_oth;
       }
-      m_run = m_new;
-      kt_cur = kt_next;
-      sk_cur = sk_next;
-      kt_next = kt_after;
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[s & 1]);
     }
   } else {
     // ------------------------------ correction ----------------------------
-    // One warp per quadrant; thread = TMEM lane (one row of A/B or of the
-    // 128-row block).  Between PV(s-1) and PV(s) it multiplies the row's O
-    // and row-sum columns by alpha(s) when the running max moved.
-    const int q = warp & 3;
-    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    const uint32_t obase = tmem + lane_base + kColO;
-    const int xrow = 32 * q + lane;
-    int row, i;
-    bool active;
-    if (MODE == 0) {
-      row = 16 * q + (lane & 15);
-      i = lane >= 16 ? iB : iA;
-      active = lane >= 16 ? hasB : true;
-    } else {
-      row = 32 * q + lane;
-      i = iA;
-      active = true;
-    }
-    const int block = MODE == 0 ? 64 : 128;
-    const int n = i * block + row;
-    const bool store = active && n < p.N;
+    // One warp per TMEM lane quadrant; thread = row.  Between PV_g(gs-1) and
+    // PV_g(gs) it multiplies the row's O_g (channels and row sum) by alpha
+    // when the frame moved; after a unit's last step it writes the output.
+    const int w = warp & 3;
+    const uint32_t lane_base = (uint32_t)(32 * w) << 16;
+    const int L = 32 * w + lane;
+    int gs = 0, ui = 0;
     bool ok = true;
-    for (int s = 0; s < nsteps; ++s) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->p_full[s & 1], (s >> 1) & 1, abort, p.wd));
+    for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ui) {
+      const Unit un = unit_of<MODE>(p, u);
+      for (int s = 0; s < nsteps; ++s, ++gs) {
+        const int b = gs & 1, ph = (gs >> 1) & 1;
+        for (int g = 0; g < 2; ++g) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars->a_ready[g][w][b], ph, abort, p.wd));
+          if (!ok) break;
+          const float alpha = alpha_s[(g * 2 + b) * 128 + L];
+          const bool has = MODE == 0 ? 2 * s + g < p.kc : true;
+          if (s > 0 && has && __any_sync(0xffffffffu, alpha != 1.f)) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[g], (gs - 1) & 1, abort, p.wd));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t ob = tmem + lane_base + (g ? kColO1 : kColO0);
+            const uint64_t a2 = f32x2_pack(alpha, alpha);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint32_t o[64];
+              const uint32_t c0 = ob + 64 * half;
+              SAGESLA_TMEM_LD16(c0 + 0, o + 0);
+              SAGESLA_TMEM_LD16(c0 + 16, o + 16);
+              SAGESLA_TMEM_LD16(c0 + 32, o + 32);
+              SAGESLA_TMEM_LD16(c0 + 48, o + 48);
+              tmem_ld_wait();
+#pragma unroll
+              for (int z = 0; z < 64; z += 2) {
+                const uint64_t v = f32x2_pack(__uint_as_float(o[z]), __uint_as_float(o[z + 1]));
+                float a0, a1;
+                f32x2_unpack(f32x2_mul(v, a2), a0, a1);
+                o[z] = __float_as_uint(a0);
+                o[z + 1] = __float_as_uint(a1);
+              }
+              SAGESLA_TMEM_ST16(c0 + 0, o + 0);
+              SAGESLA_TMEM_ST16(c0 + 16, o + 16);
+              SAGESLA_TMEM_ST16(c0 + 32, o + 32);
+              SAGESLA_TMEM_ST16(c0 + 48, o + 48);
+            }
+            {
+              uint32_t o[16];  // the row-sum columns
+              SAGESLA_TMEM_LD16(ob + 128, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int z = 0; z < 16; ++z) o[z] = __float_as_uint(__uint_as_float(o[z]) * alpha);
+              SAGESLA_TMEM_ST16(ob + 128, o);
+            }
+            tmem_st_wait();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->o_ready[g][b]);
+        }
+        if (!ok) break;
+      }
+      if (!ok) break;
+      // ------------------------------ epilogue ----------------------------
+      // out = (O_0 f_0 + O_1 f_1) / (l_0 f_0 + l_1 f_1) * s_v (+ the linear
+      // branch already in out), f_g = exp(frame_g - max of both frames).
+      int r, i;
+      bool active;
+      if (MODE == 0) {
+        r = 16 * w + (lane & 15);
+        i = lane >= 16 ? un.iB : un.iA;
+        active = lane >= 16 ? un.hasB : true;
+      } else {
+        r = L;
+        i = un.iA;
+        active = true;
+      }
+      const int n = i * (MODE == 0 ? 64 : 128) + r;
+      const bool store = active && n < p.N;
+      const bool has1 = MODE == 1 || p.kc >= 2;
+      __nv_bfloat16* orow = p.out + ((size_t)un.bh * p.N + (store ? n : 0)) * kD;
+      const bool add = p.add_out && store;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[0], (gs - 1) & 1, abort, p.wd));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[1], (gs - 1) & 1, abort, p.wd));
       if (!ok) break;
       tc_fence_after();
-      const float alpha = alpha_s[(s & 1) * 128 + xrow];
-      // PV(s-1) must be complete before O is touched, before PV(s) may start
-      // and before QK^T(s+2) may release the P buffer softmax(s+3) writes.
-      if (s > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (s - 1) & 1, abort, p.wd));
-        if (!ok) break;
-        tc_fence_after();
+      const float fr0 = frame_s[((ui & 1) * 2 + 0) * 128 + L];
+      const float fr1 = has1 ? frame_s[((ui & 1) * 2 + 1) * 128 + L] : -INFINITY;
+      const float fm = fmaxf(fr0, fr1);
+      const float f0 = fr0 == -INFINITY ? 0.f : ex2(fr0 - fm);
+      const float f1 = fr1 == -INFINITY ? 0.f : ex2(fr1 - fm);
+      const uint32_t ob0 = tmem + lane_base + kColO0, ob1 = tmem + lane_base + kColO1;
+      float l0, l1 = 0.f;
+      {
+        uint32_t t0[16], t1[16];
+        SAGESLA_TMEM_LD16(ob0 + 128, t0);
+        if (has1) SAGESLA_TMEM_LD16(ob1 + 128, t1);
+        tmem_ld_wait();
+        l0 = __uint_as_float(t0[0]);
+        if (has1) l1 = __uint_as_float(t1[0]);
       }
-      tc_fence_before();
-      mbar_arrive(&bars->s_free[s & 1]);
-      if (s > 0) {
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      const float inv = 1.f / (l0 * f0 + l1 * f1);
+      const float g0 = f0 * inv, g1 = f1 * inv;
+      const float* svh = p.sv + (size_t)un.bh * kD;
 #pragma unroll 1
-          for (int c = 0; c < kNO; c += 16) {
-            uint32_t o[16];
-            SAGESLA_TMEM_LD16(obase + c, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int z = 0; z < 16; ++z) o[z] = __float_as_uint(__uint_as_float(o[z]) * alpha);
-            SAGESLA_TMEM_ST16(obase + c, o);
-          }
-          tmem_st_wait();
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bars->o_ready);
-    }
-    // Epilogue: O_s = O / l * s_v (+ the linear branch already in out) -> bf16.
-    __nv_bfloat16* orow = p.out + ((size_t)bh * p.N + (store ? n : 0)) * kD;
-    uint4 yrow[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c)
-      yrow[c] = (p.add_out && store) ? *reinterpret_cast<const uint4*>(orow + 8 * c) : make_uint4(0, 0, 0, 0);
-    if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->fin, 0, abort, p.wd));
-    if (ok && nsteps > 0) {
-      tc_fence_after();
-      uint32_t lw[16];
-      SAGESLA_TMEM_LD16(obase + 128, lw);
-      tmem_ld_wait();
-      const float inv_l = 1.f / __uint_as_float(lw[0]);
-#pragma unroll
       for (int c = 0; c < kD; c += 16) {
-        uint32_t o[16];
-        SAGESLA_TMEM_LD16(obase + c, o);
+        uint32_t o0[16], o1[16];
+        const uint4 y0 = add ? *reinterpret_cast<const uint4*>(orow + c) : make_uint4(0, 0, 0, 0);
+        const uint4 y1 = add ? *reinterpret_cast<const uint4*>(orow + c + 8) : make_uint4(0, 0, 0, 0);
+        SAGESLA_TMEM_LD16(ob0 + c, o0);
+        if (has1) SAGESLA_TMEM_LD16(ob1 + c, o1);
         tmem_ld_wait();
         if (store) {
+          const uint32_t yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
           uint32_t pk[8];
 #pragma unroll
           for (int z = 0; z < 8; ++z) {
-            const uint32_t yw = z < 4 ? (&yrow[c / 8].x)[z] : (&yrow[c / 8 + 1].x)[z - 4];
+            const uint32_t yw = yv[z];
             const int ch = c + 2 * z;
-            const float a = __uint_as_float(o[2 * z]) * inv_l * __ldg(p.sv + (size_t)bh * kD + ch) + bf16_lo(yw);
-            const float b = __uint_as_float(o[2 * z + 1]) * inv_l * __ldg(p.sv + (size_t)bh * kD + ch + 1) + bf16_hi(yw);
-            const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+            float a = __uint_as_float(o0[2 * z]) * g0, bq = __uint_as_float(o0[2 * z + 1]) * g0;
+            if (has1) {
+              a = fmaf(__uint_as_float(o1[2 * z]), g1, a);
+              bq = fmaf(__uint_as_float(o1[2 * z + 1]), g1, bq);
+            }
+            a = fmaf(a, __ldg(svh + ch), bf16_lo(yw));
+            bq = fmaf(bq, __ldg(svh + ch + 1), bf16_hi(yw));
+            const __nv_bfloat162 h = __floats2bfloat162_rn(a, bq);
             pk[z] = *reinterpret_cast<const uint32_t*>(&h);
           }
           *reinterpret_cast<uint4*>(orow + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           *reinterpret_cast<uint4*>(orow + c + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
+      tc_fence_before();
     }
   }
   // Every MMA has completed once `fin` has both issuers' arrivals.
-  if (warp == 1) {
+  if (warp == kWarpQK) {
     if (lane == 0) mbar_wait_drain(&bars->fin, 0, p.wd);
     __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kWarpQK) tmem_dealloc(tmem, kTmemCols);
 }
 
 cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int* wd) {
@@ -575,18 +665,28 @@ cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int
   p.nq = g.nq;
   p.kc = g.kc;
   p.add_out = a.add_out;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (g.block == 64) {
+    p.upb = (g.nb + 1) / 2;
     p.nsteps = (g.kc + 1) / 2;
+  } else {
+    p.upb = g.nb;
+    p.nsteps = g.kc;
+  }
+  p.units = g.BH * p.upb;
+  const int grid = p.units < sms ? p.units : sms;
+  if (g.block == 64) {
     const int smem = Cfg<0>::kSmem;
     cudaError_t e = cudaFuncSetAttribute(flash_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    flash_kernel<0><<<dim3((g.nb + 1) / 2, g.BH), kThreads, smem, st>>>(p);
+    flash_kernel<0><<<grid, kThreads, smem, st>>>(p);
   } else {
-    p.nsteps = g.kc;
     const int smem = Cfg<1>::kSmem;
     cudaError_t e = cudaFuncSetAttribute(flash_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    flash_kernel<1><<<dim3(g.nb, g.BH), kThreads, smem, st>>>(p);
+    flash_kernel<1><<<grid, kThreads, smem, st>>>(p);
   }
   return cudaGetLastError();
 }
