@@ -143,9 +143,13 @@ int sagesla_get_mask(const void* q, const void* k, int B, int H, int N, int d, i
  * (cudaGetSymbolAddress, with that device current); make that first call
  * before any stream capture.  All calls share the scratch: calls that
  * overlap on the GPU (other streams or host threads on the same device) race
- * and must be serialised by the caller.  Sizes whose partial sums do not fit
- * the scratch (B*H above about 2000) return SAGESLA_ERR_INVALID without
- * launching; other argument errors as for sagesla_attn.
+ * and must be serialised by the caller.  The rows are split as in the
+ * regular path, so mu and sv have the same bits as sagesla_get_quant's; when
+ * the partial sums of all heads do not fit the scratch the heads run in
+ * chunks, one after another on `stream`.  A length whose partial sums for a
+ * single head exceed the scratch (N above 2 795 520 tokens) returns
+ * SAGESLA_ERR_INVALID without launching; other argument errors as for
+ * sagesla_attn.
  */
 int sagesla_smooth_stats_noalloc(const void* k, const void* v, int B, int H, int N, int d, float* mu,
                                  float* sv, sagesla_stream_t stream);

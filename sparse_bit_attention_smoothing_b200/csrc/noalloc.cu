@@ -15,6 +15,14 @@
 // different host threads on the same device) race on it; the caller must
 // serialise them.  Each call writes every scratch word it later reads, so
 // nothing has to start at zero.
+//
+// The rows of each head are split exactly as in the regular path (one split
+// per 1024 tokens), so the fp64 partial sums of the K mean are added in the
+// same order and mu comes out with the same bits.  When the partial sums of
+// all heads do not fit the scratch, the heads are processed in chunks, one
+// after another on the stream; only a single head whose partial sums exceed
+// the scratch (N above about 2.8 million tokens) is refused.
+#include <algorithm>
 #include <cstdint>
 #include <map>
 #include <mutex>
@@ -61,14 +69,10 @@ extern "C" int sagesla_smooth_stats_noalloc(const void* k, const void* v, int B,
   if (B < 1 || H < 1 || N < 1 || d != sagesla::kD) return SAGESLA_ERR_INVALID;
   const long long BH = (long long)B * H;
   if (BH > 65535 || (double)BH * N * d >= 1099511627776.0) return SAGESLA_ERR_INVALID;
-  // Same row split as the regular path (one per 1024 tokens, so the same
-  // fp64 summation order and the same bits), reduced only if the partial sums
-  // would not fit the scratch; one split per head at minimum.
-  const size_t room = kNoAllocScratchBytes - (size_t)BH * kPerHeadBytes;
-  if ((size_t)BH * kPerHeadBytes + (size_t)BH * kPerSplitBytes > kNoAllocScratchBytes) return SAGESLA_ERR_INVALID;
-  int split = (N + 1023) / 1024;
-  const int fit = (int)(room / ((size_t)BH * kPerSplitBytes));
-  if (split > fit) split = fit;
+  const int split = (N + 1023) / 1024;
+  const size_t per_head = (size_t)split * kPerSplitBytes + kPerHeadBytes;
+  if (per_head > kNoAllocScratchBytes) return SAGESLA_ERR_INVALID;
+  const int chunk = (int)std::min<long long>(BH, (long long)(kNoAllocScratchBytes / per_head));
   if ((reinterpret_cast<uintptr_t>(k) & 15u) || (reinterpret_cast<uintptr_t>(v) & 15u) ||
       (reinterpret_cast<uintptr_t>(mu) & 3u) || (reinterpret_cast<uintptr_t>(sv) & 3u))
     return SAGESLA_ERR_MISALIGNED;
@@ -83,19 +87,27 @@ extern "C" int sagesla_smooth_stats_noalloc(const void* k, const void* v, int B,
   const int rc = scratch_address(dev, &scratch);
   if (rc != SAGESLA_OK) return rc;
 
-  sagesla::Geom g{};
-  g.BH = (int)BH;
-  g.N = N;
-  g.block = 64;
-  g.nb = (N + 63) / 64;
-  g.nq = 2 * ((N + 127) / 128);
-  g.kc = g.nb;
-  g.split = split;
-  double* psum = reinterpret_cast<double*>(scratch);
-  float* pmax = reinterpret_cast<float*>(scratch + (size_t)BH * split * sagesla::kD * sizeof(double));
-  float* mv = reinterpret_cast<float*>(scratch + (size_t)BH * split * kPerSplitBytes);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (sagesla::launch_stats_partial(k, v, g, psum, pmax, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
-  if (sagesla::launch_stats_final(psum, pmax, g, mu, sv, mv, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
+  const size_t head_elems = (size_t)N * d;
+  for (long long h0 = 0; h0 < BH; h0 += chunk) {
+    const int nh = (int)std::min<long long>(chunk, BH - h0);
+    sagesla::Geom g{};
+    g.BH = nh;
+    g.N = N;
+    g.block = 64;
+    g.nb = (N + 63) / 64;
+    g.nq = 2 * ((N + 127) / 128);
+    g.kc = g.nb;
+    g.split = split;
+    double* psum = reinterpret_cast<double*>(scratch);
+    float* pmax = reinterpret_cast<float*>(scratch + (size_t)nh * split * sagesla::kD * sizeof(double));
+    float* mv = reinterpret_cast<float*>(scratch + (size_t)nh * split * kPerSplitBytes);
+    const uint16_t* kh = static_cast<const uint16_t*>(k) + h0 * head_elems;
+    const uint16_t* vh = static_cast<const uint16_t*>(v) + h0 * head_elems;
+    if (sagesla::launch_stats_partial(kh, vh, g, psum, pmax, st) != cudaSuccess) return SAGESLA_ERR_LAUNCH;
+    if (sagesla::launch_stats_final(psum, pmax, g, mu + h0 * sagesla::kD, sv + h0 * sagesla::kD, mv, st) !=
+        cudaSuccess)
+      return SAGESLA_ERR_LAUNCH;
+  }
   return SAGESLA_OK;
 }
