@@ -113,12 +113,13 @@ def flash_traffic(w):
     return t["dram_bytes"] / t["elements"] * (w.B * w.H * w.N * w.d)
 
 
-def flops(w) -> dict:
-    """Dense-equivalent and computed-block FLOPs of one call, and algorithmic HBM bytes."""
-    from sparse_bit_attention_smoothing_b200 import topk_count
+def flops(w, kc: int) -> dict:
+    """Dense-equivalent and computed-block FLOPs of one call, and algorithmic HBM bytes.
+
+    kc = key blocks kept per query block (the caller's topk_count: the library's
+    in the GPU arm, the oracle's in the reference arm)."""
     BH, N, d = w.B * w.H, w.N, w.d
     nb = (N + w.block - 1) // w.block
-    kc = topk_count(nb, w.topk)
     dense = 4.0 * BH * N * N * d
     blocks = 4.0 * BH * nb * kc * w.block * w.block * d
     E = BH * N * d
@@ -126,38 +127,152 @@ def flops(w) -> dict:
     return dict(dense=dense, computed=blocks, hbm_bytes=float(hbm), nb=nb, kc=kc)
 
 
-def cpu_baseline(w, q, k, v, pw, heads: int = 8, qblocks: int = 4) -> dict:
-    """The oracle, as it stands, on a bounded sample of the workload; extrapolated to one call."""
-    import numpy as np
+def _oracle():
     from oracle import oracle as orc
     orc.lib()
+    return orc
+
+
+def cpu_sample_plan(w, cores: int, qblocks: int = 2):
+    """The oracle's bounded sample of a workload: one head per host core (all
+    heads if there are fewer) x `qblocks` evenly spaced query blocks per head."""
+    import numpy as np
+    BH = w.B * w.H
+    nb = (w.N + w.block - 1) // w.block
+    heads = min(BH, max(1, cores))
+    picks = np.unique(np.linspace(0, nb - 1, qblocks).round().astype(int))
+    return heads, picks, nb
+
+
+def cpu_fixed_part(w, q, k, v, pw, heads: int) -> float:
+    """Seconds of the oracle's per-head work outside the query blocks (smoothing,
+    quantisation, mask, linear-branch blocks) for `heads` heads run together."""
+    import numpy as np
+    orc = _oracle()
     BH, N, d = w.B * w.H, w.N, w.d
     nb = (N + w.block - 1) // w.block
-    hs = min(heads, BH)
-    qf = q.reshape(BH, N, d)[:hs].contiguous()
-    kf = k.reshape(BH, N, d)[:hs].contiguous()
-    vf = v.reshape(BH, N, d)[:hs].contiguous()
-    sel0 = np.zeros((hs, nb), np.uint8)
+    qf, kf, vf = (t.reshape(BH, N, d)[:heads].contiguous() for t in (q, k, v))
     t0 = time.perf_counter()
-    orc.sagesla(qf, kf, vf, pw, w.block, w.topk, qsel=sel0)
-    t_fixed = time.perf_counter() - t0
-    sel = np.zeros((hs, nb), np.uint8)
-    picks = np.unique(np.linspace(0, nb - 1, qblocks).round().astype(int))
+    orc.sagesla(qf, kf, vf, pw, w.block, w.topk, qsel=np.zeros((heads, nb), np.uint8))
+    return time.perf_counter() - t0
+
+
+def cpu_sample(w, q, k, v, pw, heads: int, picks, t_fixed: float) -> dict:
+    """The oracle, as it stands, on the sample (the fixed part plus the picked
+    query blocks of `heads` heads, one per core), extrapolated to one call:
+    along query blocks (x nb / picks) and along heads by whole waves of one
+    head per core (x ceil(BH / heads)).  Returns the rate and the sampled rows."""
+    import numpy as np
+    orc = _oracle()
+    BH, N, d = w.B * w.H, w.N, w.d
+    nb = (N + w.block - 1) // w.block
+    qf, kf, vf = (t.reshape(BH, N, d)[:heads].contiguous() for t in (q, k, v))
+    sel = np.zeros((heads, nb), np.uint8)
     sel[:, picks] = 1
     t0 = time.perf_counter()
-    orc.sagesla(qf, kf, vf, pw, w.block, w.topk, qsel=sel)
+    out, idx = orc.sagesla(qf, kf, vf, pw, w.block, w.topk, qsel=sel)
     t_sample = time.perf_counter() - t0
-    cores = orc.threads()
-    t_qb = max(0.0, (t_sample - t_fixed) / len(picks))
-    waves = math.ceil(BH / min(cores, hs)) if hs < cores else math.ceil(BH / cores)
-    full_s = waves * (t_fixed + nb * t_qb)
-    f = flops(w)
-    return dict(value=f["dense"] / full_s / 1e12, unit="TFLOPS", cores=cores, kind="oracle",
-                ms_per_call=full_s * 1e3,
-                sample=(f"{hs} heads x {len(picks)} query blocks of {w.name} (fp64 C oracle, OpenMP over heads); "
-                        f"per-head fixed part {t_fixed:.2f}s, {t_qb * 1e3:.1f} ms per query block; "
-                        f"extrapolated to {BH} heads x {nb} query blocks"),
-                sample_seconds=t_fixed + t_sample)
+    t_q = max(0.0, t_sample - t_fixed) / len(picks)
+    waves = math.ceil(BH / heads)
+    full_s = waves * (t_fixed + nb * t_q)
+    f = flops(w, orc.topk_count(nb, w.topk))
+    return dict(value=f["dense"] / full_s / 1e12, unit="TFLOPS", cores=orc.threads(), kind="oracle",
+                ms_per_call=full_s * 1e3, extrapolated=True,
+                sample=(f"{heads} heads (one per host core) x {len(picks)} query blocks of {w.name} (fp64 C oracle, "
+                        f"OpenMP over heads): fixed part {t_fixed:.2f} s, {t_q * 1e3:.1f} ms per query block; "
+                        f"extrapolated to {nb} query blocks and to {BH} heads in {waves} waves"),
+                sample_seconds=t_fixed + t_sample, out=out, idx=idx, heads=heads, picks=picks)
+
+
+def cpu_baseline(w, q, k, v, pw, qblocks: int = 2) -> dict:
+    orc = _oracle()
+    heads, picks, _ = cpu_sample_plan(w, orc.threads(), qblocks)
+    t_fixed = cpu_fixed_part(w, q, k, v, pw, heads)
+    return cpu_sample(w, q, k, v, pw, heads, picks, t_fixed)
+
+
+def _bf16_half_ulp(x):
+    import numpy as np
+    x = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.maximum(x, 2.0 ** -126)))
+    return np.ldexp(1.0, (e - 8).astype(np.int64))
+
+
+def parity(w, q, k, gpu_out, gpu_idx, cb, near_tie: float = 1e-5) -> dict:
+    """Parity figures of the timed call: the block mask of every head against
+    the oracle's (equal rows, and rows that differ only in near-ties of the
+    k-th pooled score within `near_tie`); the sampled output rows against the
+    oracle's quantised emulation (max-abs error beyond half a bf16 ulp, and
+    cosine), on rows whose mask the two sides share."""
+    import numpy as np
+    orc = _oracle()
+    BH, N, d = w.B * w.H, w.N, w.d
+    nb = (N + w.block - 1) // w.block
+    qf, kf = q.reshape(BH, N, d), k.reshape(BH, N, d)
+    om = orc.mask(qf, kf, w.block, w.topk)["idx"]
+    gi = gpu_idx.reshape(BH, nb, -1)
+    eq_rows = (gi == om).all(axis=2)
+    near = other = 0
+    for h in np.nonzero(~eq_rows.all(axis=1))[0]:
+        s64 = orc.block_scores_f64(qf[h:h + 1].contiguous(), kf[h:h + 1].contiguous(), w.block)[0]
+        for i in np.nonzero(~eq_rows[h])[0]:
+            kth = np.sort(s64[i])[::-1][gi.shape[2] - 1]
+            diff = set(gi[h, i].tolist()) ^ set(om[h, i].tolist())
+            if all(abs(s64[i, j] - kth) <= near_tie for j in diff):
+                near += 1
+            else:
+                other += 1
+    got, ref = [], []
+    go = gpu_out.reshape(BH, N, d)
+    for h in range(cb["heads"]):
+        for i in cb["picks"]:
+            if eq_rows[h, i]:
+                r0, r1 = i * w.block, min(N, (i + 1) * w.block)
+                got.append(go[h, r0:r1])
+                ref.append(cb["out"][h, r0:r1])
+    got = np.concatenate(got).astype(np.float64) if got else np.zeros((0, d))
+    ref = np.concatenate(ref) if ref else np.zeros((0, d))
+    err = float(np.max(np.abs(got - ref) - _bf16_half_ulp(ref))) if got.size else None
+    cos = float((got * ref).sum() / np.sqrt((got * got).sum() * (ref * ref).sum())) if got.size else None
+    return {"mask_rows": int(BH * nb), "mask_rows_equal": int(eq_rows.sum()), "mask_rows_near_tie": near,
+            "mask_rows_other": other, "out_rows_compared": int(got.shape[0]), "max_abs_excess": err,
+            "cosine": cos, "tolerance": {"max_abs_excess": 1e-2, "cosine": 0.9999, "near_tie": near_tie}}
+
+
+def measure_8bit_peaks(n: int = 8192, reps: int = 10) -> dict:
+    """Dense 8-bit library GEMM throughput on this GPU: torch._int_mm (INT8 x
+    INT8 -> INT32) and torch._scaled_mm (E4M3 x E4M3 -> bf16), n^3, best of
+    `reps`, CUDA events; 2 n^3 FLOP each."""
+    import torch
+    dev = torch.device("cuda")
+    out = {}
+    a8 = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+    b8 = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+    af = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    bf = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=dev)
+
+    def best(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return min(ts)
+    for name, fn in (("int8", lambda: torch._int_mm(a8, b8.t().contiguous().t())),
+                     ("e4m3", lambda: torch._scaled_mm(af, bf, scale_a=one, scale_b=one, out_dtype=torch.bfloat16))):
+        try:
+            ms = best(fn)
+            out[name] = {"ms": ms, "tflops": 2.0 * n ** 3 / (ms * 1e-3) / 1e12}
+        except Exception as e:  # report what failed, keep the other
+            out[name] = {"error": str(e).splitlines()[0][:200]}
+    return out
 
 
 def run_all(args):
@@ -194,7 +309,8 @@ def run_all(args):
         prof = sg.profile_read()
         sg.profile(False)
         ms = e0.elapsed_time(e1) / args.steps
-        f = flops(w)
+        nb = (w.N + w.block - 1) // w.block
+        f = flops(w, sg.topk_count(nb, w.topk))
         fl_ms, fl_n = prof.get("flash", (0.0, 0))
         flash_ms = fl_ms / max(1, fl_n)
         achieved = f["computed"] / (flash_ms * 1e-3) / 1e12 if flash_ms > 0 else None
@@ -212,26 +328,33 @@ def run_all(args):
 
 
 def run_reference(args):
+    """The oracle, as it stands, timed on the host cores on the same bounded
+    sample as the GPU arm's cpu_baseline (one head per core x 2 query blocks),
+    one sample per step; rank 0 only.  Loads only the oracle's library."""
     rank = _env_int("RANK", 0)
     if rank != 0:
         return 0
     from sparse_bit_attention_smoothing_b200.inputs import make_workload
+    orc = _oracle()
     w = workloads()[args.workload]
     q, k, v, pw = make_workload(w)
+    heads, picks, nb = cpu_sample_plan(w, orc.threads())
+    t_fixed = cpu_fixed_part(w, q, k, v, pw, heads)
     vals = []
     for s in range(args.warmup + args.steps):
-        cb = cpu_baseline(w, q, k, v, pw, heads=4, qblocks=2)
+        cb = cpu_sample(w, q, k, v, pw, heads, picks, t_fixed)
         if s >= args.warmup:
             vals.append(cb)
     val = statistics.median([c["value"] for c in vals])
     ms = statistics.median([c["ms_per_call"] for c in vals])
+    f = flops(w, orc.topk_count(nb, w.topk))
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "ms_per_step_extrapolated": True,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.block,
-                       "topk": w.topk, "linear": w.linear},
+                       "topk": w.topk, "k_blocks": f["kc"], "nb": nb, "linear": w.linear},
             "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": vals[0]["cores"], "kind": "oracle",
-                             "sample": vals[0]["sample"]},
+                             "sample": vals[0]["sample"], "extrapolated": True},
             "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -247,7 +370,11 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-linear", action="store_true", help="proj_w = NULL (linear branch off)")
+    ap.add_argument("--peaks", action="store_true", help="measure the 8-bit library GEMM peaks and exit")
     args = ap.parse_args()
+    if args.peaks:
+        print(json.dumps({"n": 8192, "peaks": measure_8bit_peaks()}), flush=True)
+        return 0
     if args.impl == "reference":
         return run_reference(args)
     if args.workload == "all":
@@ -305,7 +432,7 @@ def main():
     status = sg.sync_status()
     ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], device="cuda")[0]
 
-    f = flops(w)
+    f = flops(w, sg.topk_count((w.N + w.block - 1) // w.block, w.topk))
     value = job_throughput(f["dense"], world, ms) / 1e12
     pk = peaks()
     peak8 = 2.0 * pk["bf16"]  # 8-bit dense = 2 x bf16 (nominal 4.5 / 2.25 PFLOP/s)
@@ -349,7 +476,11 @@ def main():
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": E}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(w, q, k, v, pw)
-        line["cpu_baseline"] = {kk: cb[kk] for kk in ("value", "unit", "cores", "kind", "sample", "ms_per_call")}
+        line["cpu_baseline"] = {kk: cb[kk] for kk in ("value", "unit", "cores", "kind", "sample", "ms_per_call",
+                                                       "extrapolated")}
+        gidx = sg.sagesla_get_mask(dq, dk, block=w.block, topk=w.topk, stream=st)["idx"]
+        torch.cuda.synchronize()
+        line["parity"] = parity(w, q, k, out.float().cpu().numpy(), gidx.cpu().numpy(), cb)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -94,7 +94,8 @@ struct Cfg {
   static constexpr int kOffP = kOffV + 2 * kVStage;  // [parity b][half g]
   static constexpr int kOffA = kOffP + 4 * kPTile;   // alpha [g][b][128] f32
   static constexpr int kOffF = kOffA + 2 * 2 * 128 * 4;  // final frames [unit parity][g][128] f32
-  static constexpr int kOffBar = kOffF + 2 * 2 * 128 * 4;
+  static constexpr int kOffM = kOffF + 2 * 2 * 128 * 4;  // StepMeta ring [4]
+  static constexpr int kOffBar = kOffM + 4 * 32;
   static constexpr int kSmem = kOffBar + 512 + 1024;  // + alignment slack
 };
 
@@ -108,11 +109,21 @@ struct Bars {
   uint64_t p_empty[2][2];     // [g][b]: PV that read the P~ buffer complete
   uint64_t o_ready[2][2];     // [g][b]: O_g rescaled, PV_g may accumulate
   uint64_t o_done[2];         // [g]: PV_g of the step complete
+  uint64_t m_full[4], m_empty[4];  // step metadata ring (producer -> softmax)
   uint64_t fin;               // every MMA of both issuers complete
   uint32_t tmem;
   int abort;
 };
 static_assert(sizeof(Bars) <= 512, "barrier block");
+
+// Per-step metadata the K producer hands to the softmax warps: the 64-key
+// tiles of the step (block 64: slot 2X+g = list entry 2s+g of query block X,
+// -1 when absent; block 128: slots 0, 1 = the two halves of list entry s)
+// and their INT8 key scales.
+struct StepMeta {
+  int tile[4];
+  float sk[4];
+};
 
 struct Unit {
   int bh, iA, iB;
@@ -141,6 +152,27 @@ __device__ __forceinline__ int list_at(const Params& p, int bh, int i, int t) {
   return p.idx ? __ldg(p.idx + ((size_t)bh * p.nb + i) * p.kc + t) : t;
 }
 
+// Max of the first `nv` of `n` integer scores (n a multiple of 8): four
+// independent chains of three-input maxima when all are valid.
+template <int n>
+__device__ __forceinline__ int max_valid(const uint32_t* t, int nv, int m) {
+  if (nv >= n) {
+    int c4[4] = {m, INT_MIN, INT_MIN, INT_MIN};
+#pragma unroll
+    for (int c = 0; c < n; c += 8) {
+      c4[0] = __vimax3_s32(c4[0], (int)t[c], (int)t[c + 1]);
+      c4[1] = __vimax3_s32(c4[1], (int)t[c + 2], (int)t[c + 3]);
+      c4[2] = __vimax3_s32(c4[2], (int)t[c + 4], (int)t[c + 5]);
+      c4[3] = __vimax3_s32(c4[3], (int)t[c + 6], (int)t[c + 7]);
+    }
+    return max(max(c4[0], c4[1]), max(c4[2], c4[3]));
+  }
+#pragma unroll
+  for (int c = 0; c < n; ++c)
+    if (c < nv) m = max(m, (int)t[c]);
+  return m;
+}
+
 }  // namespace
 
 template <int MODE>
@@ -151,6 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
   float* alpha_s = reinterpret_cast<float*>(smem + C::kOffA);
   float* frame_s = reinterpret_cast<float*>(smem + C::kOffF);
+  StepMeta* meta = reinterpret_cast<StepMeta*>(smem + C::kOffM);
   volatile int* abort = &bars->abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nsteps = p.nsteps;
@@ -170,6 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         mbar_init(&bars->o_ready[x][b], 4);
         for (int w = 0; w < 4; ++w) mbar_init(&bars->a_ready[x][w][b], 1);
       }
+    }
+    for (int x = 0; x < 4; ++x) {
+      mbar_init(&bars->m_full[x], 1);
+      mbar_init(&bars->m_empty[x], 8);
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, 8);
@@ -243,6 +280,18 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
             if (tiles[x] >= 0)
               bulk_g2s(ring + st * stage_bytes + x * slot_bytes, src + (head_tiles + tiles[x]) * kTile, kTile,
                        &full[st]);
+          if (is_k) {
+            // the step's metadata for the softmax warps (a 4-deep ring)
+            const int ms = gs & 3;
+            float skv[4];
+            for (int x = 0; x < 4; ++x) skv[x] = (x < C::kSlots && tiles[x] >= 0) ? __ldg(p.sk + head_tiles + tiles[x]) : 0.f;
+            if (gs >= 4 && !(ok = mbar_wait(&bars->m_empty[ms], ((gs >> 2) - 1) & 1, abort, p.wd))) break;
+            for (int x = 0; x < 4; ++x) {
+              meta[ms].tile[x] = x < C::kSlots ? tiles[x] : -1;
+              meta[ms].sk[x] = skv[x];
+            }
+            mbar_arrive(&bars->m_full[ms]);
+          }
         }
       }
       // Drain: every copy issued must land before the CTA may exit.
@@ -342,50 +391,37 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ui) {
       const Unit un = unit_of<MODE>(p, u);
-      int r, i, qtile;
+      int r, qtile, xs;
       bool active;
       if (MODE == 0) {
         const bool isB = lane >= 16;
         r = 16 * w + (lane & 15);
-        i = isB ? un.iB : un.iA;
         active = isB ? un.hasB : true;
-        qtile = i;
+        qtile = isB ? un.iB : un.iA;
+        xs = isB ? 2 : 0;  // metadata slots of this row's query block
       } else {
         r = L;
-        i = un.iA;
         active = true;
         qtile = 2 * un.iA + (r >> 6);
+        xs = 0;
       }
-      const size_t tb = (size_t)un.bh * p.nq;
-      const float c0 = active ? __ldg(p.sq + tb + qtile) * (kLog2e * kRsqrtD) : 0.f;
+      const float c0 = active ? __ldg(p.sq + (size_t)un.bh * p.nq + qtile) * (kLog2e * kRsqrtD) : 0.f;
       uint8_t* prow = smem + C::kOffP + g * C::kPTile + (MODE == 0 && lane >= 16 ? 4096 : 0);
       float m_all = -INFINITY, frame = -INFINITY;
-      // Key tiles (64 keys each) of this row's own half and of the other half
-      // of step s, and their scales; fetched one step ahead of use.
-      auto tiles_of = [&](int s, int& t_own, int& t_oth) {
-        t_own = t_oth = -1;
-        if (s >= nsteps || !active) return;
-        if (MODE == 0) {
-          const int e0 = 2 * s + g, e1 = 2 * s + 1 - g;
-          if (e0 < p.kc) t_own = list_at(p, un.bh, i, e0);
-          if (e1 < p.kc) t_oth = list_at(p, un.bh, i, e1);
-        } else {
-          const int j = list_at(p, un.bh, i, s);
-          t_own = 2 * j + g;
-          t_oth = 2 * j + 1 - g;
-        }
-      };
-      auto nvalid = [&](int t) { return t >= 0 ? max(0, min(64, p.N - 64 * t)) : 0; };
-      int t_own, t_oth;
-      tiles_of(0, t_own, t_oth);
-      float sk_own = nvalid(t_own) > 0 ? __ldg(p.sk + tb + t_own) : 0.f;
-      float sk_oth = nvalid(t_oth) > 0 ? __ldg(p.sk + tb + t_oth) : 0.f;
-      int n_own, n_oth;
-      tiles_of(1, n_own, n_oth);
       for (int s = 0; s < nsteps; ++s, ++gs) {
         const int b = gs & 1;
-        const int nv_own = nvalid(t_own), nv_oth = nvalid(t_oth);
-        const float cu_own = c0 * sk_own, cu_oth = c0 * sk_oth;
+        // Key tiles of this row's own half and of the other half, and their
+        // scales, from the producer's metadata ring (no global loads here).
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->m_full[gs & 3], (gs >> 2) & 1, abort, p.wd));
+        if (!ok) break;
+        const StepMeta& mt = meta[gs & 3];
+        const int t_own = active ? mt.tile[xs + g] : -1;
+        const int t_oth = active ? mt.tile[xs + 1 - g] : -1;
+        const int nv_own = t_own >= 0 ? max(0, min(64, p.N - 64 * t_own)) : 0;
+        const int nv_oth = t_oth >= 0 ? max(0, min(64, p.N - 64 * t_oth)) : 0;
+        const float cu_own = c0 * mt.sk[xs + g], cu_oth = c0 * mt.sk[xs + 1 - g];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->m_empty[gs & 3]);
         // The P~ buffer b was read by PV_g(gs-2); waiting for it first keeps
         // every barrier this warp publishes on at most one phase ahead.
         if (gs >= 2) {
@@ -408,40 +444,16 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
           SAGESLA_TMEM_LD16(sx + 0, t + 0);
           SAGESLA_TMEM_LD16(sx + 16, t + 16);
           tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c < nv_oth) mx_oth = max(mx_oth, (int)t[c]);
+          mx_oth = max_valid<32>(t, nv_oth, mx_oth);
           SAGESLA_TMEM_LD16(sx + 32, t + 0);
           SAGESLA_TMEM_LD16(sx + 48, t + 16);
           tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c + 32 < nv_oth) mx_oth = max(mx_oth, (int)t[c]);
+          mx_oth = max_valid<32>(t, nv_oth - 32, mx_oth);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_free);
-        // Scales of the next step (its list entries arrived during this one)
-        // and the list entries of the step after; issued only now, since an
-        // mbarrier arrive has release semantics and would wait for them.
-        const float sk_own_n = nvalid(n_own) > 0 ? __ldg(p.sk + tb + n_own) : 0.f;
-        const float sk_oth_n = nvalid(n_oth) > 0 ? __ldg(p.sk + tb + n_oth) : 0.f;
-        int a_own, a_oth;
-        tiles_of(s + 2, a_own, a_oth);
-        int mx_own = INT_MIN;
-        if (nv_own == 64) {
-          int m2[2] = {INT_MIN, INT_MIN};
-#pragma unroll
-          for (int c = 0; c < 64; c += 4) {
-            m2[0] = __vimax3_s32(m2[0], (int)acc[c], (int)acc[c + 1]);
-            m2[1] = __vimax3_s32(m2[1], (int)acc[c + 2], (int)acc[c + 3]);
-          }
-          mx_own = max(m2[0], m2[1]);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < nv_own) mx_own = max(mx_own, (int)acc[c]);
-        }
+        const int mx_own = max_valid<64>(acc, nv_own, INT_MIN);
         const float mf_own = nv_own > 0 ? __int2float_rn(mx_own) * cu_own : -INFINITY;
         const float mf_oth = nv_oth > 0 ? __int2float_rn(mx_oth) * cu_oth : -INFINITY;
         // Frame of O_g after this step: at block 64 half 0 is walk block 2s
@@ -457,49 +469,54 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->a_ready[g][w][b]);
         // P~ of the own half: exponent of 448*P = S*c - frame + log2(448), one
-        // fused multiply-add per key, two keys per f32x2 instruction; keys
-        // past the sequence end get P~ = 0.
+        // fused multiply-add per key on the converted integer score, two keys
+        // per f32x2 instruction; keys past the sequence end get P~ = 0.  Each
+        // phase runs over all 64 keys so that the conversions, the
+        // exponentials and the FP8 packing of different keys overlap.
         uint8_t* pbuf = prow + 2 * b * C::kPTile;
         // (block 128: a half past the sequence end still feeds the PV, with P~ = 0)
         if (nv_own > 0 || (MODE == 1 && active)) {
           const float kk = kLog2_448 - frame;
           const uint64_t cc = f32x2_pack(cu_own, cu_own), ko = f32x2_pack(kk, kk);
+          // Software-pipelined over 16-key chunks: the conversions and FMAs of
+          // chunk ch+1 (I2F and FMA pipes) are issued next to the exponentials
+          // of chunk ch (ex2 unit), so the two pipes overlap.
+          float xc[16], xn[16];
+          auto conv = [&](int ch, float (&x)[16]) {
+#pragma unroll
+            for (int z = 0; z < 16; z += 2) {
+              const int c = 16 * ch + z;
+              const uint64_t dd =
+                  f32x2_fma(f32x2_pack(__int2float_rn((int)acc[c]), __int2float_rn((int)acc[c + 1])), cc, ko);
+              f32x2_unpack(dd, x[z], x[z + 1]);
+            }
+          };
+          conv(0, xc);
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
+            if (ch < 3) conv(ch + 1, xn);
+#pragma unroll
+            for (int z = 0; z < 16; ++z) xc[z] = ex2(xc[z]);
+            if (nv_own < 64) {
+#pragma unroll
+              for (int z = 0; z < 16; ++z)
+                if (16 * ch + z >= nv_own) xc[z] = 0.f;
+            }
             uint32_t wv[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float x[4];
-#pragma unroll
-              for (int z = 0; z < 4; z += 2) {
-                const int c = 16 * ch + 4 * e + z;
-                const uint64_t dd =
-                    f32x2_fma(f32x2_pack(__int2float_rn((int)acc[c]), __int2float_rn((int)acc[c + 1])), cc, ko);
-                float a0, a1;
-                f32x2_unpack(dd, a0, a1);
-                x[z] = ex2(a0);
-                x[z + 1] = ex2(a1);
-              }
-              if (nv_own < 64) {
-#pragma unroll
-                for (int z = 0; z < 4; ++z)
-                  if (16 * ch + 4 * e + z >= nv_own) x[z] = 0.f;
-              }
-              wv[e] = __byte_perm(e4m3x2(x[0], x[1]), e4m3x2(x[2], x[3]), 0x5410);
-            }
+            for (int e = 0; e < 4; ++e)
+              wv[e] = __byte_perm(e4m3x2(xc[4 * e], xc[4 * e + 1]), e4m3x2(xc[4 * e + 2], xc[4 * e + 3]), 0x5410);
             *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, 16 * ch, kP_LBO, kP_SBO)) =
                 make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            if (ch < 3) {
+#pragma unroll
+              for (int z = 0; z < 16; ++z) xc[z] = xn[z];
+            }
           }
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->p_full[g][b]);
-        t_own = n_own;
-        t_oth = n_oth;
-        sk_own = sk_own_n;
-        sk_oth = sk_oth_n;
-        n_own = a_own;
-        n_oth = a_oth;
       }
     }
   } else {
@@ -521,41 +538,46 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
           if (!ok) break;
           const float alpha = alpha_s[(g * 2 + b) * 128 + L];
           const bool has = MODE == 0 ? 2 * s + g < p.kc : true;
-          if (s > 0 && has && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // PV_g(gs-1) must be complete before O_g is touched; the wait is
+          // taken at every step (not only when rescaling) so that each parity
+          // wait on o_done, the epilogue's included, is one phase ahead at most.
+          if (s > 0) {
             ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[g], (gs - 1) & 1, abort, p.wd));
             if (!ok) break;
+          }
+          if (s > 0 && has && __any_sync(0xffffffffu, alpha != 1.f)) {
             tc_fence_after();
             const uint32_t ob = tmem + lane_base + (g ? kColO1 : kColO0);
             const uint64_t a2 = f32x2_pack(alpha, alpha);
+            // 144 columns (128 channels + the row-sum columns) in chunks of 32
+            // (the last 16): the load of chunk c+1 is in flight while chunk c
+            // is multiplied and stored.
+            uint32_t o[2][32];
+            SAGESLA_TMEM_LD16(ob + 0, o[0]);
+            SAGESLA_TMEM_LD16(ob + 16, o[0] + 16);
+            tmem_ld_wait();
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              uint32_t o[64];
-              const uint32_t c0 = ob + 64 * half;
-              SAGESLA_TMEM_LD16(c0 + 0, o + 0);
-              SAGESLA_TMEM_LD16(c0 + 16, o + 16);
-              SAGESLA_TMEM_LD16(c0 + 32, o + 32);
-              SAGESLA_TMEM_LD16(c0 + 48, o + 48);
-              tmem_ld_wait();
-#pragma unroll
-              for (int z = 0; z < 64; z += 2) {
-                const uint64_t v = f32x2_pack(__uint_as_float(o[z]), __uint_as_float(o[z + 1]));
-                float a0, a1;
-                f32x2_unpack(f32x2_mul(v, a2), a0, a1);
-                o[z] = __float_as_uint(a0);
-                o[z + 1] = __float_as_uint(a1);
+            for (int ch = 0; ch < 5; ++ch) {
+              uint32_t* cur = o[ch & 1];
+              uint32_t* nxt = o[(ch + 1) & 1];
+              if (ch < 3) {
+                SAGESLA_TMEM_LD16(ob + 32 * (ch + 1), nxt);
+                SAGESLA_TMEM_LD16(ob + 32 * (ch + 1) + 16, nxt + 16);
+              } else if (ch == 3) {
+                SAGESLA_TMEM_LD16(ob + 128, nxt);
               }
-              SAGESLA_TMEM_ST16(c0 + 0, o + 0);
-              SAGESLA_TMEM_ST16(c0 + 16, o + 16);
-              SAGESLA_TMEM_ST16(c0 + 32, o + 32);
-              SAGESLA_TMEM_ST16(c0 + 48, o + 48);
-            }
-            {
-              uint32_t o[16];  // the row-sum columns
-              SAGESLA_TMEM_LD16(ob + 128, o);
-              tmem_ld_wait();
+              const int n = ch < 4 ? 32 : 16;
 #pragma unroll
-              for (int z = 0; z < 16; ++z) o[z] = __float_as_uint(__uint_as_float(o[z]) * alpha);
-              SAGESLA_TMEM_ST16(ob + 128, o);
+              for (int z = 0; z < 32; z += 2) {
+                if (z >= n) break;
+                float a0, a1;
+                f32x2_unpack(f32x2_mul(f32x2_pack(__uint_as_float(cur[z]), __uint_as_float(cur[z + 1])), a2), a0, a1);
+                cur[z] = __float_as_uint(a0);
+                cur[z + 1] = __float_as_uint(a1);
+              }
+              SAGESLA_TMEM_ST16(ob + 32 * ch, cur);
+              if (n == 32) SAGESLA_TMEM_ST16(ob + 32 * ch + 16, cur + 16);
+              if (ch < 4) tmem_ld_wait();
             }
             tmem_st_wait();
           }
@@ -649,7 +671,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
   if (warp == kWarpQK) tmem_dealloc(tmem, kTmemCols);
 }
 
-cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int* wd) {
+// Block 128 (one 128-row query block per unit, M = 128); block 64 runs the
+// two-slot kernel of k_flash64.cu.
+cudaError_t launch_flash128(const FlashArgs& a, const Geom& g, cudaStream_t st, int* wd) {
   Params p;
   p.q8t = a.q8t;
   p.k8t = a.k8t;
@@ -668,26 +692,14 @@ cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (g.block == 64) {
-    p.upb = (g.nb + 1) / 2;
-    p.nsteps = (g.kc + 1) / 2;
-  } else {
-    p.upb = g.nb;
-    p.nsteps = g.kc;
-  }
+  p.upb = g.nb;
+  p.nsteps = g.kc;
   p.units = g.BH * p.upb;
   const int grid = p.units < sms ? p.units : sms;
-  if (g.block == 64) {
-    const int smem = Cfg<0>::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(flash_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    flash_kernel<0><<<grid, kThreads, smem, st>>>(p);
-  } else {
-    const int smem = Cfg<1>::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(flash_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    flash_kernel<1><<<grid, kThreads, smem, st>>>(p);
-  }
+  const int smem = Cfg<1>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(flash_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  flash_kernel<1><<<grid, kThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 

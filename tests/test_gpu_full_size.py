@@ -1,10 +1,12 @@
-"""Parity at full size, on sampled outputs, for every benchmark configuration:
-Wan2.1-1.3B-480P (H=12, N=32760), 14B-480P (H=40, N=32760), 14B-720P
-(H=40, N=75600) at topk 0.1 and 0.05, block 128, and the dense point
-(topk 1, linear branch off).  Each runs the whole call on the GPU in the
-launch configuration bench.py times; two heads are checked against the
-oracle: the whole mask, and the first, a middle and the ragged last query
-block of the output, which the oracle computes one by one."""
+"""Parity at full size for every benchmark configuration: Wan2.1-1.3B-480P
+(H=12, N=32760), 14B-480P (H=40, N=32760), 14B-720P (H=40, N=75600) at topk
+0.1 and 0.05, and every point of the 720p sparsity sweep (block 64 and 128,
+topk 0.05 / 0.1 / 0.15, and the dense point: topk 1, linear branch off).
+Each runs the whole call on the GPU in the launch configuration bench.py
+times.  The mask of EVERY head is compared with the oracle's (exact up to
+counted near-ties of the k-th pooled score); on two heads the first, a
+middle and the ragged last query block of the output are compared with the
+oracle run on those query blocks alone."""
 import numpy as np
 import pytest
 import torch
@@ -18,9 +20,11 @@ _INPUTS = {}
 
 def _workloads():
     from sparse_bit_attention_smoothing_b200 import inputs as I
+    # the 720p sweep at block 64, topk 0.05 / 0.1, is WAN14_720P_K05 / WAN14_720P
     sw = {w.name: w for w in I.sweep()}
-    return [I.WAN13_480P, I.WAN14_480P, I.WAN14_720P, I.WAN14_720P_K05, sw["sweep_b128_topk0.1"],
-            sw["sweep_b64_dense"]]
+    return [I.WAN13_480P, I.WAN14_480P, I.WAN14_720P, I.WAN14_720P_K05, sw["sweep_b64_topk0.15"],
+            sw["sweep_b64_dense"], sw["sweep_b128_topk0.05"], sw["sweep_b128_topk0.1"], sw["sweep_b128_topk0.15"],
+            sw["sweep_b128_dense"]]
 
 
 def _inputs_for(w):
@@ -60,17 +64,24 @@ def _head(t, h, N):
     return t.reshape(-1, N, 128)[h:h + 1]
 
 
-def test_full_size_mask_of_sampled_heads(orc, full_run):
+def test_full_size_mask_of_every_head(orc, full_run):
     w, N = full_run["w"], full_run["w"].N
-    for h in _heads(w):
+    BH = w.B * w.H
+    if w.topk >= 1.0:
+        pytest.skip("dense point: every key block is selected")
+    o = orc.mask(full_run["q"].reshape(BH, N, 128), full_run["k"].reshape(BH, N, 128), w.block, w.topk)
+    nb = o["idx"].shape[1]
+    assert full_run["k_blocks"] == o["k"]
+    gi = full_run["idx"].reshape(BH, nb, o["k"])
+    equal_heads = [h for h in range(BH) if np.array_equal(gi[h], o["idx"][h])]
+    near = 0
+    for h in sorted(set(range(BH)) - set(equal_heads)):
         qh, kh = _head(full_run["q"], h, N), _head(full_run["k"], h, N)
-        o = orc.mask(qh, kh, w.block, w.topk)
-        nb = o["idx"].shape[1]
-        assert full_run["k_blocks"] == o["k"]
-        gi = full_run["idx"].reshape(-1, nb, o["k"])[h]
         s64 = orc.block_scores_f64(qh, kh, w.block)
-        eq, near = compare_masks(gi, o["idx"].reshape(nb, -1), s64.reshape(nb, nb), o["k"])
-        assert eq + near == nb
+        eq, nt = compare_masks(gi[h], o["idx"][h], s64.reshape(nb, nb), o["k"])
+        assert eq + nt == nb
+        near += nt
+    print(f"{w.name}: {BH} heads x {nb} query blocks, {near} near-tie rows, all other rows equal")
 
 
 def test_full_size_sampled_query_blocks(orc, full_run):
