@@ -159,8 +159,12 @@ int sagesla_topk_count(int nb, float topk);
 
 /*
  * sagesla_sync_status: synchronises `stream` and returns SAGESLA_OK, or
- * SAGESLA_ERR_DEVICE_TIMEOUT if any bounded device-side wait of an earlier
- * call on it gave up (the flag is then cleared), or SAGESLA_ERR_LAUNCH.
+ * SAGESLA_ERR_DEVICE_TIMEOUT if a bounded device-side wait of an earlier
+ * call gave up (the flag is then cleared), or SAGESLA_ERR_LAUNCH.  The flag
+ * is one word per DEVICE, shared by all streams: a timeout on any stream of
+ * the current device is reported by the next sagesla_sync_status() on any
+ * stream (after that stream's work, not necessarily the other stream's).
+ * Callers that use several streams synchronise them all, then call this once.
  */
 int sagesla_sync_status(sagesla_stream_t stream);
 
@@ -176,6 +180,30 @@ int sagesla_sync_status(sagesla_stream_t stream);
  * SAGESLA_ERR_NO_DEVICE / SAGESLA_ERR_LAUNCH as the other entry points.
  */
 int sagesla_watchdog_selftest(int probes, sagesla_stream_t stream);
+
+/*
+ * sagesla_debug_flash_stall: the failure-detection path of the real sparse
+ * flash kernel, made to run on purpose without faulting the GPU.  Runs
+ * sagesla_attn(q, k, v, NULL, out, B, H, N, d, 64, topk) with three changes
+ * to its block-64 flash launch:
+ *   - `grid` CTAs (>= 1; capped at the normal persistent grid), so that one
+ *     CTA can be made to serve many query blocks;
+ *   - every bounded wait of the flash kernel gives up after `spin_limit`
+ *     probes (1024 .. 16777216, the default being 16777216);
+ *   - for stall_step >= 0, CTA 0's first pipeline omits the key-tile copies
+ *     of its step `stall_step` (counted over all its query blocks), so the
+ *     wait of the MMA issuer on that stage never completes; it gives up,
+ *     raises the CTA's abort flag (every role stops at its next wait), waits
+ *     for the copies and MMAs already in flight, frees its tensor memory and
+ *     returns, and the device's watchdog word is set.  stall_step == -1
+ *     stalls nothing (the output is then that of sagesla_attn).
+ * The next sagesla_sync_status() returns SAGESLA_ERR_DEVICE_TIMEOUT once;
+ * the context stays usable.  `out` is partly unwritten after a stall.
+ * Returns SAGESLA_ERR_INVALID for arguments out of range (no launch), else
+ * as sagesla_attn.
+ */
+int sagesla_debug_flash_stall(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,
+                              float topk, int grid, int stall_step, long long spin_limit, sagesla_stream_t stream);
 
 /* Human-readable text for a return code (static storage). */
 const char* sagesla_strerror(int code);

@@ -29,7 +29,8 @@ class SageSLAError(RuntimeError):
 
 EXPORTS = ["sagesla_attn", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
            "sagesla_smooth_stats_noalloc", "sagesla_topk_count", "sagesla_sync_status", "sagesla_strerror",
-           "sagesla_release", "sagesla_profile", "sagesla_profile_read", "sagesla_watchdog_selftest"]
+           "sagesla_release", "sagesla_profile", "sagesla_profile_read", "sagesla_watchdog_selftest",
+           "sagesla_debug_flash_stall"]
 KERNELS = ["stats", "stats_final", "quant", "pool_topk", "linear_kv", "linear_sum", "flash", "w_tile",
            "linear_apply"]
 
@@ -51,6 +52,7 @@ def lib():
         L.sagesla_topk_count.argtypes = [i, f]
         L.sagesla_sync_status.argtypes = [P]
         L.sagesla_watchdog_selftest.argtypes = [i, P]
+        L.sagesla_debug_flash_stall.argtypes = [P, P, P, P, i, i, i, i, f, i, i, ctypes.c_longlong, P]
         L.sagesla_strerror.restype = ctypes.c_char_p
         L.sagesla_strerror.argtypes = [i]
         L.sagesla_release.restype = None
@@ -172,6 +174,21 @@ def sagesla_watchdog_selftest(probes: int = 1000, stream=None):
     """Make one bounded device-side wait expire on purpose (nothing faults); the next sync_status() on the stream
     then returns -5 (device watchdog timeout) and clears the flag."""
     _check(lib().sagesla_watchdog_selftest(probes, _stream(stream)), "sagesla_watchdog_selftest")
+
+
+def sagesla_debug_flash_stall(q, k, v, out=None, topk: float = 0.1, grid: int = 1, stall_step: int = -1,
+                              spin_limit: int = 1 << 24, stream=None):
+    """sagesla_attn at block 64 without the linear branch, its flash kernel on `grid` CTAs with bounded waits of
+    `spin_limit` probes; stall_step >= 0 makes CTA 0's first pipeline omit the key copies of that step, so a real
+    wait of the kernel gives up (sync_status() then returns -5 once).  Returns `out`."""
+    import torch
+    B, H, N, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().sagesla_debug_flash_stall(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, ctypes.c_float(topk),
+                                           grid, stall_step, spin_limit, _stream(stream)),
+           "sagesla_debug_flash_stall")
+    return out
 
 
 def sync_status(stream=None) -> int:

@@ -246,7 +246,7 @@ int run_front(const void* q, const void* k, const void* v, const Geom& g, const 
 }
 
 int run_attn(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B, int H, int N, int d,
-             int block, float topk, cudaStream_t st) {
+             int block, float topk, cudaStream_t st, int dbg_grid = 0, int dbg_stall = 0, long dbg_spin = 0) {
   SAGESLA_TRY(validate(q, k, v, out, B, H, N, d, block, topk));
   if (proj_w && !aligned16(proj_w)) return SAGESLA_ERR_MISALIGNED;
   int dev = 0;
@@ -293,6 +293,9 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
   fa.idx = dense ? nullptr : b.idx;
   fa.out = out;
   fa.add_out = linear ? 1 : 0;
+  fa.dbg_grid = dbg_grid;
+  fa.dbg_stall = dbg_stall;
+  fa.dbg_spin = dbg_spin;
   {
     ProfScope ps(6, st);
     SAGESLA_TRY(launch_rc(launch_flash(fa, g, st, wd)));
@@ -489,6 +492,13 @@ int sagesla_watchdog_selftest(int probes, sagesla_stream_t stream) {
   int dev = 0;
   SAGESLA_TRY(check_device(&dev));
   return launch_rc(launch_watchdog_selftest(probes, watchdog(dev), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sagesla_debug_flash_stall(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,
+                              float topk, int grid, int stall_step, long long spin_limit, sagesla_stream_t stream) {
+  if (grid < 1 || stall_step < -1 || spin_limit < 1024 || spin_limit > kSpinLimit) return SAGESLA_ERR_INVALID;
+  return run_attn(q, k, v, nullptr, out, B, H, N, d, 64, topk, reinterpret_cast<cudaStream_t>(stream), grid,
+                  stall_step + 1, (long)spin_limit);
 }
 
 int sagesla_sync_status(sagesla_stream_t stream) {

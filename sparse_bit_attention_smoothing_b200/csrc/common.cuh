@@ -70,12 +70,13 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait.  Returns false if it gave up: then it raises `abort` (a
-// CTA-shared flag, so that every role of the CTA stops) and the global
-// watchdog word `wd`.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* wd) {
+// Bounded wait of at most `limit` probes.  Returns false if it gave up: then
+// it raises `abort` (a CTA-shared flag, so that every role of the CTA stops)
+// and the global watchdog word `wd`.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* wd,
+                                          long limit = kSpinLimit) {
   if (mbar_test(bar, parity)) return true;
-  for (long i = 0; i < kSpinLimit; ++i) {
+  for (long i = 0; i < limit; ++i) {
     if (mbar_try(bar, parity)) return true;
     if ((i & 255) == 255 && *abort) return false;
   }

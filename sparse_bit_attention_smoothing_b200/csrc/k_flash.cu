@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       const int stage_bytes = is_k ? C::kKStage : C::kVStage;
       const int slot_bytes = is_k ? kTile : C::kVSlot;
       uint8_t* ring = smem + (is_k ? C::kOffK : C::kOffV);
-      int gs = 0, ui = 0;
+      int gs = 0, ui = 0, issued = 0;  // issued: steps whose copies are out
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ui) {
         const Unit un = unit_of<MODE>(p, u);
@@ -280,6 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
             if (tiles[x] >= 0)
               bulk_g2s(ring + st * stage_bytes + x * slot_bytes, src + (head_tiles + tiles[x]) * kTile, kTile,
                        &full[st]);
+          issued = gs + 1;
           if (is_k) {
             // the step's metadata for the softmax warps (a 4-deep ring)
             const int ms = gs & 3;
@@ -294,8 +295,11 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
           }
         }
       }
-      // Drain: every copy issued must land before the CTA may exit.
-      for (int g2 = max(0, gs - 2); g2 < gs; ++g2) mbar_wait_drain(&full[g2 & 1], (g2 >> 1) & 1, p.wd);
+      // Drain: every copy issued must land before the CTA may exit.  The
+      // empty-wait of step g proved the copies of step g-2 consumed, so only
+      // the last two steps issued can still be in flight (also when a wait
+      // gave up after the copies of its step were issued).
+      for (int g2 = max(0, issued - 2); g2 < issued; ++g2) mbar_wait_drain(&full[g2 & 1], (g2 >> 1) & 1, p.wd);
       if (is_k)
         for (int u2 = max(0, ui - 2); u2 < ui; ++u2) mbar_wait_drain(&bars->q_full[u2 & 1], (u2 >> 1) & 1, p.wd);
     }

@@ -94,6 +94,8 @@ struct Params {
   int items;   // BH * nb query blocks
   int nsteps;  // steps per query block: ceil(kc / 2)
   int add_out; // 1: out already holds the linear branch (bf16); add O_s to it
+  long spin;    // probe limit of every bounded wait that may give up
+  int stall_gs; // >= 0: slot 0's K producer omits the copy of this step (watchdog test)
 };
 
 // The K producer's hand-off to the softmax warps: the two key tiles of a
@@ -211,14 +213,14 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
       uint8_t* ring = sb + (is_k ? kOffK : kOffV);
       const int stage_bytes = is_k ? 2 * kTile : 2 * kVSlot;
       const int slot_bytes = is_k ? kTile : kVSlot;
-      int gs = 0, ui = 0;
+      int gs = 0, ui = 0, skipped = -1, issued = 0;  // issued: steps whose copies are out
       bool ok = true;
       for (int q = 2 * (int)blockIdx.x + X; ok && q < p.items; q += stride, ++ui) {
         const int bh = q / p.nb, i = q - bh * p.nb;
         const size_t head_tiles = (size_t)bh * p.nq;
         if (is_k) {
           const int qb = ui & 1;
-          if (ui >= 2 && !(ok = mbar_wait(&B.q_empty[qb], ((ui >> 1) - 1) & 1, abort, p.wd))) break;
+          if (ui >= 2 && !(ok = mbar_wait(&B.q_empty[qb], ((ui >> 1) - 1) & 1, abort, p.wd, p.spin))) break;
           mbar_expect_tx(&B.q_full[qb], kTile);
           bulk_g2s(sb + kOffQ + qb * kTile, p.q8t + (head_tiles + i) * kTile, kTile, &B.q_full[qb]);
         }
@@ -226,15 +228,21 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
           const int t0 = list_at(p, bh, i, 2 * s);
           const int t1 = 2 * s + 1 < p.kc ? list_at(p, bh, i, 2 * s + 1) : -1;
           const int st = gs & 1;
-          if (gs >= 2 && !(ok = mbar_wait(&empty[st], ((gs >> 1) - 1) & 1, abort, p.wd))) break;
-          mbar_expect_tx(&full[st], (t1 >= 0 ? 2 : 1) * kTile);
-          bulk_g2s(ring + st * stage_bytes, src + (head_tiles + t0) * kTile, kTile, &full[st]);
-          if (t1 >= 0) bulk_g2s(ring + st * stage_bytes + slot_bytes, src + (head_tiles + t1) * kTile, kTile, &full[st]);
+          if (gs >= 2 && !(ok = mbar_wait(&empty[st], ((gs >> 1) - 1) & 1, abort, p.wd, p.spin))) break;
+          if (is_k && X == 0 && blockIdx.x == 0 && gs == p.stall_gs) {
+            skipped = gs;  // this stage's barrier never completes: its waiter gives up
+          } else {
+            mbar_expect_tx(&full[st], (t1 >= 0 ? 2 : 1) * kTile);
+            bulk_g2s(ring + st * stage_bytes, src + (head_tiles + t0) * kTile, kTile, &full[st]);
+            if (t1 >= 0)
+              bulk_g2s(ring + st * stage_bytes + slot_bytes, src + (head_tiles + t1) * kTile, kTile, &full[st]);
+          }
+          issued = gs + 1;
           if (is_k) {
             const float sk0 = __ldg(p.sk + head_tiles + t0);
             const float sk1 = t1 >= 0 ? __ldg(p.sk + head_tiles + t1) : 0.f;
             const int ms = gs & 3;
-            if (gs >= 4 && !(ok = mbar_wait(&B.m_empty[ms], ((gs >> 2) - 1) & 1, abort, p.wd))) break;
+            if (gs >= 4 && !(ok = mbar_wait(&B.m_empty[ms], ((gs >> 2) - 1) & 1, abort, p.wd, p.spin))) break;
             meta[ms].tile[0] = t0;
             meta[ms].tile[1] = t1;
             meta[ms].sk[0] = sk0;
@@ -243,8 +251,12 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
           }
         }
       }
-      // Drain: every copy issued must land before the CTA may exit.
-      for (int g2 = max(0, gs - 2); g2 < gs; ++g2) mbar_wait_drain(&full[g2 & 1], (g2 >> 1) & 1, p.wd);
+      // Drain: every copy issued must land before the CTA may exit.  The
+      // empty-wait of step g proved the copies of step g-2 consumed, so only
+      // the last two steps issued can still be in flight (also when a wait
+      // gave up after the copies of its step were issued).
+      for (int g2 = max(0, issued - 2); g2 < issued; ++g2)
+        if (g2 != skipped) mbar_wait_drain(&full[g2 & 1], (g2 >> 1) & 1, p.wd);
       if (is_k)
         for (int u2 = max(0, ui - 2); u2 < ui; ++u2) mbar_wait_drain(&B.q_full[u2 & 1], (u2 >> 1) & 1, p.wd);
     }
@@ -267,9 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
       for (int gs = 0; ok && gs <= total; ++gs) {
         if (gs < total) {
           const int ui = gs / nsteps, s = gs - ui * nsteps, qb = ui & 1, st = gs & 1;
-          if (s == 0 && !(ok = mbar_wait(&B.q_full[qb], (ui >> 1) & 1, abort, p.wd))) break;
-          if (!(ok = mbar_wait(&B.k_full[st], (gs >> 1) & 1, abort, p.wd))) break;
-          if (gs > 0 && !(ok = mbar_wait(&B.s_free, (gs - 1) & 1, abort, p.wd))) break;
+          if (s == 0 && !(ok = mbar_wait(&B.q_full[qb], (ui >> 1) & 1, abort, p.wd, p.spin))) break;
+          if (!(ok = mbar_wait(&B.k_full[st], (gs >> 1) & 1, abort, p.wd, p.spin))) break;
+          if (gs > 0 && !(ok = mbar_wait(&B.s_free, (gs - 1) & 1, abort, p.wd, p.spin))) break;
           tc_fence_after();
           const uint32_t id = 2 * s + 1 < p.kc ? idesc_i8(64, 128) : idesc_i8(64, 64);
 #pragma unroll
@@ -282,8 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
         }
         if (gs > 0) {
           const int gp = gs - 1, s = gp % nsteps, b = gp & 1, st = gp & 1;
-          if (!(ok = mbar_wait(&B.v_full[st], (gp >> 1) & 1, abort, p.wd))) break;
-          if (!(ok = mbar_wait(&B.p_full[b], (gp >> 1) & 1, abort, p.wd))) break;
+          if (!(ok = mbar_wait(&B.v_full[st], (gp >> 1) & 1, abort, p.wd, p.spin))) break;
+          if (!(ok = mbar_wait(&B.p_full[b], (gp >> 1) & 1, abort, p.wd, p.spin))) break;
           tc_fence_after();
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
@@ -320,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
       float m_all = -INFINITY, frame = -INFINITY;
       for (int s = 0; s < nsteps; ++s, ++gs) {
         const int b = gs & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&B.m_full[gs & 3], (gs >> 2) & 1, abort, p.wd));
+        ok = __all_sync(0xffffffffu, mbar_wait(&B.m_full[gs & 3], (gs >> 2) & 1, abort, p.wd, p.spin));
         if (!ok) break;
         const StepMeta& mt = meta[gs & 3];
         const int t_own = mt.tile[g], t_oth = mt.tile[1 - g];
@@ -332,10 +344,10 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
         // The P~ buffer b was read by PV(gs-2): wait for it before anything of
         // this step is published.
         if (gs >= 2) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&B.p_empty[b], ((gs >> 1) - 1) & 1, abort, p.wd));
+          ok = __all_sync(0xffffffffu, mbar_wait(&B.p_empty[b], ((gs >> 1) - 1) & 1, abort, p.wd, p.spin));
           if (!ok) break;
         }
-        ok = __all_sync(0xffffffffu, mbar_wait(&B.s_full, gs & 1, abort, p.wd));
+        ok = __all_sync(0xffffffffu, mbar_wait(&B.s_full, gs & 1, abort, p.wd, p.spin));
         if (!ok) break;
         tc_fence_after();
         uint32_t acc[64];
@@ -405,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
         // issuing thread before QK(gs), so this wait is one phase ahead at most).  Threads 0-15 hold O_0 rows, 16-31 O_1 rows (column
         // split 144 = kColO1 - kColO0); alpha is 1 where nothing moved.
         if (s > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&B.o_done, (gs - 1) & 1, abort, p.wd));
+          ok = __all_sync(0xffffffffu, mbar_wait(&B.o_done, (gs - 1) & 1, abort, p.wd, p.spin));
           if (!ok) break;
           tc_fence_after();
           const uint64_t a2 = f32x2_pack(alpha, alpha);
@@ -444,8 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
       // done, but PV(gs-2) may still be running; a parity wait must never be
       // two phases ahead of its barrier, so wait for PV(gs-2) first, then
       // for the last PV(gs-1).
-      if (gs >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&B.o_done, (gs - 2) & 1, abort, p.wd));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&B.o_done, (gs - 1) & 1, abort, p.wd));
+      if (gs >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&B.o_done, (gs - 2) & 1, abort, p.wd, p.spin));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&B.o_done, (gs - 1) & 1, abort, p.wd, p.spin));
       if (!ok) break;
       tc_fence_after();
       const float fr_oth = __shfl_xor_sync(0xffffffffu, frame, 16);
@@ -536,11 +548,14 @@ cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int
   p.add_out = a.add_out;
   p.items = g.BH * g.nb;
   p.nsteps = (g.kc + 1) / 2;
+  p.spin = a.dbg_spin > 0 ? a.dbg_spin : kSpinLimit;
+  p.stall_gs = a.dbg_stall - 1;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int want = (p.items + 1) / 2;
-  const int grid = want < sms ? want : sms;
+  int grid = want < sms ? want : sms;
+  if (a.dbg_grid > 0 && a.dbg_grid < grid) grid = a.dbg_grid;
   cudaError_t e = cudaFuncSetAttribute(flash64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   flash64_kernel<<<grid, kThreads, kSmem, st>>>(p);

@@ -60,6 +60,13 @@ struct FlashArgs {
   const int32_t* idx;  // [BH][nb][kc]; NULL = dense (every block, ascending)
   void* out;           // bf16 [BH][N][128]
   int add_out;          // 1: out already holds the linear branch y (bf16); add O_s to it
+  // Watchdog test of the block-64 kernel (all 0 in a normal call): a grid of
+  // dbg_grid CTAs instead of the persistent grid, dbg_spin probes per
+  // bounded wait instead of the default, and, for dbg_stall > 0, slot 0's K
+  // producer of CTA 0 omits the copies of its step dbg_stall - 1.
+  int dbg_grid;
+  int dbg_stall;
+  long dbg_spin;
 };
 cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int* wd);
 // Waits `probes` times on an mbarrier that never completes, then sets *wd.

@@ -81,6 +81,9 @@ def test_rejects_bad_arguments_without_launch(L):
         assert L.sagesla_attn(a, a, a, None, a, 1, 1, n_max + 1, 128, blk, F(0.1), None) == -1
         assert L.sagesla_attn(a, a, a, None, a, 1, 1, n_max, 128, blk, F(0.1), None) != -1
     assert L.sagesla_watchdog_selftest((1 << 20) + 1, None) == -1
+    ll = ctypes.c_longlong
+    for grid, stall, spin in ((0, -1, 1 << 14), (1, -2, 1 << 14), (1, 0, 1023), (1, 0, (1 << 24) + 1)):
+        assert L.sagesla_debug_flash_stall(a, a, a, a, 1, 1, 64, 128, F(0.1), grid, stall, ll(spin), None) == -1
 
 
 C_CLIENT = r"""
