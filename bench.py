@@ -45,6 +45,9 @@ def workloads():
     return d
 
 
+NOMINAL_8BIT_TFLOPS = 4500.0  # B200 dense INT8 / FP8, nominal
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -320,6 +323,7 @@ def run_all(args):
                 "dense_equiv_tflops": f["dense"] / (ms * 1e-3) / 1e12,
                 "flash_ms": flash_ms, "flash_tflops": achieved,
                 "flash_frac_of_8bit_peak": (achieved / peak8) if achieved else None,
+                "flash_frac_of_nominal_8bit": (achieved / NOMINAL_8BIT_TFLOPS) if achieved else None,
                 "path_frac_of_roofline": t_roof * 1e3 / ms, "device_status": sg.sync_status(),
                 "kernels_ms": {kname: round(t / max(1, n), 4) for kname, (t, n) in prof.items()}}
         print(json.dumps(line), flush=True)
@@ -435,7 +439,10 @@ def main():
     f = flops(w, sg.topk_count((w.N + w.block - 1) // w.block, w.topk))
     value = job_throughput(f["dense"], world, ms) / 1e12
     pk = peaks()
-    peak8 = 2.0 * pk["bf16"]  # 8-bit dense = 2 x bf16 (nominal 4.5 / 2.25 PFLOP/s)
+    # the roofline peak: 8-bit dense = 2 x the measured bf16 burst (the
+    # 60 % target is judged on this measured figure); the fraction of the
+    # chip's nominal 8-bit dense peak (4.5 PFLOP/s) is reported beside it
+    peak8 = 2.0 * pk["bf16"]
     fl_ms, fl_n = prof.get("flash", (0.0, 0))
     flash_ms = fl_ms / max(1, fl_n)
     achieved = f["computed"] / (flash_ms * 1e-3) / 1e12 if flash_ms > 0 else None
@@ -470,6 +477,8 @@ def main():
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak8, "unit": "TFLOP/s",
                          "frac": (achieved / peak8) if achieved else None, "traffic": flash_traffic(w),
                          "kernel": "flash", "peak_note": f"8-bit = 2 x {pk['src']} bf16 burst {pk['bf16']}",
+                         "frac_of_nominal_8bit": (achieved / NOMINAL_8BIT_TFLOPS) if achieved else None,
+                         "nominal_8bit_peak": NOMINAL_8BIT_TFLOPS,
                          "path_t_roof_ms": t_roof * 1e3, "path_frac": t_roof * 1e3 / ms},
             "clocks": clocks,
             "e2e": {"value": job_throughput(f["dense"], world, e2e_ms) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
