@@ -452,12 +452,12 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
       // out = (O_0 f_0 + O_1 f_1) / (l_0 f_0 + l_1 f_1) * s_v (+ the linear
       // branch already in out), f_g = exp(frame_g - max of both frames);
       // threads 0-15 write channels 0-63 of their row, 16-31 channels 64-127.
-      // o_done completes once per PV.  s_full(gs-1) implied that PV(gs-3) is
-      // done, but PV(gs-2) may still be running; a parity wait must never be
-      // two phases ahead of its barrier, so wait for PV(gs-2) first, then
-      // for the last PV(gs-1).
-      if (gs >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&B.o_done, (gs - 2) & 1, abort, p.wd, p.spin));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&B.o_done, (gs - 1) & 1, abort, p.wd, p.spin));
+      // The last PV(gs-1) must be complete.  Here o_done may have completed
+      // PV(gs-2), PV(gs-1), both or neither, which no single parity wait on it
+      // can tell apart; p_empty of the step's parity completes only for
+      // PV(gs-1) and PV(gs-3) (this warp waited for the latter in its last
+      // step, and PV(gs+1) needs this warp's next P~), so its wait is exact.
+      ok = __all_sync(0xffffffffu, mbar_wait(&B.p_empty[(gs - 1) & 1], ((gs - 1) >> 1) & 1, abort, p.wd, p.spin));
       if (!ok) break;
       tc_fence_after();
       const float fr_oth = __shfl_xor_sync(0xffffffffu, frame, 16);

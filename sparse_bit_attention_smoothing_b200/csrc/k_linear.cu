@@ -60,7 +60,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 // columns, ~40 KB of shared memory) so that four share an SM and their load
 // phases overlap each other's compute.  Thread 0 issues the MMAs.  Dynamic
 // smem: A (phi(K) rows) and B (V rows) MN-major, BLK x 128 bf16 each; after
-// the MMAs the same bytes stage the bf16 h image.
+// the MMAs the h image goes from TMEM straight to the mask-GEMM tiles.
 template <int BLK>
 __global__ void __launch_bounds__(256, 4) linear_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                                            int N, int nb, int nbt, uint8_t* __restrict__ hs,
@@ -69,7 +69,6 @@ __global__ void __launch_bounds__(256, 4) linear_kv_kernel(const uint4* __restri
   constexpr uint32_t kSBO = (BLK / 8) * 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* img = smem;  // 32 KB h image, after the MMAs are done with the operands
   __shared__ uint64_t bar;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
@@ -122,11 +121,15 @@ __global__ void __launch_bounds__(256, 4) linear_kv_kernel(const uint4* __restri
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_s;
+  // h_j^T = V_j^T phi(K_j): A = the V rows (M = value channel cv), B = the
+  // phi(K) rows (N = key channel ck), so TMEM lane cv, column ck holds
+  // h_j[ck][cv] and each thread later owns 8 consecutive ck of one cv: one
+  // 16-byte chunk of the image.
   if (t == 0) {
     const uint32_t id = idesc_bf16(128, 128, 1) | (1u << 15);  // A and B MN-major
 #pragma unroll
     for (int ks = 0; ks < BLK / 16; ++ks)
-      mma_bf16(tmem, smem_desc(smem + ks * 256, 128, kSBO), smem_desc(smem + kOpBytes + ks * 256, 128, kSBO), id,
+      mma_bf16(tmem, smem_desc(smem + kOpBytes + ks * 256, 128, kSBO), smem_desc(smem + ks * 256, 128, kSBO), id,
                ks > 0);
     mma_commit(&bar);
   }
@@ -142,27 +145,28 @@ __global__ void __launch_bounds__(256, 4) linear_kv_kernel(const uint4* __restri
   }
   const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar, 0, &abort_s, wd));
   tc_fence_after();
-  // h_j rows: warp w holds ck = 32(w%4) + lane, columns cv in [64(w/4), +64).
-  // Stage the bf16 image (the operands are dead once the MMAs completed).
+  // Warp w holds cv = 32(w%4) + lane, columns ck in [64(w/4), +64); every
+  // 8 columns are one 16-byte chunk of the bf16 image of H^T (element (cv,
+  // ck) at himg_off), stored straight into its place in the mask-GEMM tile.
   {
-    const int ck = 32 * (warp & 3) + lane, cb = 64 * (warp >> 2);
+    const int cv = 32 * (warp & 3) + lane, cb = 64 * (warp >> 2);
+    uint8_t* hsb = hs + (size_t)bh * nbt * 64 * 16384 * 2;
 #pragma unroll 1
     for (int c0 = cb; c0 < cb + 64; c0 += 16) {
       uint32_t r[16];
       SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0, r);
       tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float val = ok ? __uint_as_float(r[e]) : 0.f;
-        *reinterpret_cast<__nv_bfloat16*>(img + himg_off(c0 + e, ck)) = __float2bfloat16_rn(val);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          w4[e] = ok ? pack_bf16(__uint_as_float(r[8 * h + 2 * e]), __uint_as_float(r[8 * h + 2 * e + 1])) : 0u;
+        const int chunk = (int)(himg_off(cv, c0 + 8 * h) >> 4);
+        *reinterpret_cast<uint4*>(hsb + hs_chunk(nbt, j, chunk)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
     }
   }
-  __syncthreads();
-  // 2048 chunks of 16 bytes into the mask-GEMM tiles.
-  for (int c = t; c < 2048; c += 256)
-    *reinterpret_cast<uint4*>(hs + (size_t)bh * nbt * 64 * 16384 * 2 + hs_chunk(nbt, j, c)) =
-        *reinterpret_cast<const uint4*>(img + c * 16);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 128);
