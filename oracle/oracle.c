@@ -28,7 +28,8 @@
  * closed forms for the quantised path (uniform scores, constant V, a
  * two-key worked example); e4m3 encoder exhaustive vs torch's cast; int8
  * quantiser closed forms; mask vs brute-force sort and constructed ties;
- * linear branch vs per-token sum and closed forms.
+ * linear branch vs per-token sum and closed forms; W8A8 linear vs integer
+ * matmul at unit scales and vs the matmul of the dequantised operands.
  */
 #include <math.h>
 #include <stdint.h>
@@ -40,7 +41,7 @@
 
 #define ORC_QBLK 64 /* quantisation block of Q and K: 64 tokens */
 
-int orc_version(void) { return 2; }
+int orc_version(void) { return 3; }
 
 int orc_threads(void) {
 #ifdef _OPENMP
@@ -656,4 +657,59 @@ void orc_linear_direct(const double* q, const double* k, const double* v, int N,
     for (int c = 0; c < d; ++c) num[c] = den > 0.0 ? num[c] / den : 0.0;
     free(in_s);
   }
+}
+
+/* ------------------------------------------------------------------------ */
+/* W8A8 linear layer ("揭秘TurboDiffusion：如何让视频生成实现百倍加速？",   */
+/* 支柱三 W8A8线性层量化; 量子位 news, 技术解密 4): weights and activations   */
+/* are both INT8, quantised in blocks of 128 x 128, and y = x W^T (W is     */
+/* [N][K], the nn.Linear convention).  Reading (the pages give only the     */
+/* block size): one fp32 scale per 128 x 128 block, the same symmetric      */
+/* quantiser as Q and K above (s = fl32(amax/127), code = RNE(fl32(x *      */
+/* fl32(127/amax))) clamped to +-127; amax = 0 -> s = 1, codes 0); a last    */
+/* block of rows shorter than 128 is quantised over its valid rows.          */
+/*   y[m][n] = sum over 128-wide K blocks kb of                              */
+/*             s_x[m/128][kb] * s_w[n/128][kb] * (exact integer dot on kb).  */
+/* ------------------------------------------------------------------------ */
+#define ORC_WBLK 128
+
+/* a: bf16 [rows][cols] (cols a multiple of 128); q: int8 [rows][cols];
+ * s: fp32 [ceil(rows/128)][cols/128]. */
+void orc_w8a8_quant(const uint16_t* a, int rows, int cols, int8_t* q, float* s) {
+  const int nrb = (rows + ORC_WBLK - 1) / ORC_WBLK, ncb = cols / ORC_WBLK;
+  for (int rb = 0; rb < nrb; ++rb)
+    for (int cb = 0; cb < ncb; ++cb) {
+      const int r0 = rb * ORC_WBLK, r1 = r0 + ORC_WBLK < rows ? r0 + ORC_WBLK : rows;
+      const int c0 = cb * ORC_WBLK;
+      float amax = 0.f;
+      for (int r = r0; r < r1; ++r)
+        for (int c = c0; c < c0 + ORC_WBLK; ++c) {
+          float x = fabsf(bf16_f32(a[(int64_t)r * cols + c]));
+          if (x > amax) amax = x;
+        }
+      const float mult = amax > 0.f ? 127.f / amax : 0.f;
+      s[(int64_t)rb * ncb + cb] = amax > 0.f ? amax / 127.f : 1.f;
+      for (int r = r0; r < r1; ++r)
+        for (int c = c0; c < c0 + ORC_WBLK; ++c)
+          q[(int64_t)r * cols + c] = orc_int8_code(bf16_f32(a[(int64_t)r * cols + c]), mult);
+    }
+}
+
+/* y: fp64 [M][N] from the codes and scales of x [M][K] and W [N][K]. */
+void orc_w8a8_gemm(const int8_t* qx, const float* sx, const int8_t* qw, const float* sw, int M, int N, int K,
+                   double* y) {
+  const int nkb = K / ORC_WBLK;
+#pragma omp parallel for schedule(static)
+  for (int m = 0; m < M; ++m)
+    for (int n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        int64_t dot = 0;
+        for (int k = kb * ORC_WBLK; k < (kb + 1) * ORC_WBLK; ++k)
+          dot += (int64_t)qx[(int64_t)m * K + k] * (int64_t)qw[(int64_t)n * K + k];
+        acc += (double)sx[(int64_t)(m / ORC_WBLK) * nkb + kb] * (double)sw[(int64_t)(n / ORC_WBLK) * nkb + kb] *
+               (double)dot;
+      }
+      y[(int64_t)m * N + n] = acc;
+    }
 }

@@ -64,6 +64,8 @@ def lib():
         L.orc_sagesla.restype = i
         L.orc_sagesla.argtypes = [P, P, P, P, i, i, i, i, f, P, P, i, P, P]
         L.orc_linear_direct.argtypes = [P, P, P, i, i, i, i, P, P]
+        L.orc_w8a8_quant.argtypes = [P, i, i, P, P]
+        L.orc_w8a8_gemm.argtypes = [P, P, P, P, i, i, i, P]
         _lib = L
     return _lib
 
@@ -214,3 +216,37 @@ def linear_direct(q, k, v, block: int, idx: np.ndarray) -> np.ndarray:
     out = np.empty((N, d), np.float64)
     lib().orc_linear_direct(_p(q), _p(k), _p(v), N, d, block, kc, _p(idx), _p(out))
     return out
+
+
+# ---------------------------------------------------------------- W8A8 ----
+WBLK = 128  # quantisation block of the W8A8 linear layer (128 x 128)
+
+
+def w8a8_quant(a) -> dict:
+    """INT8 codes [rows][cols] and fp32 scales [ceil(rows/128)][cols/128] of a bf16 matrix in 128 x 128 blocks."""
+    a = _bits(a)
+    rows, cols = a.shape
+    assert cols % WBLK == 0
+    q = np.empty((rows, cols), np.int8)
+    s = np.empty(((rows + WBLK - 1) // WBLK, cols // WBLK), np.float32)
+    lib().orc_w8a8_quant(_p(a), rows, cols, _p(q), _p(s))
+    return {"q": q, "s": s}
+
+
+def w8a8_gemm(qx, sx, qw, sw) -> np.ndarray:
+    """y = sum over K blocks of s_x s_w (integer dot), fp64 [M][N]."""
+    qx, qw = np.ascontiguousarray(qx, np.int8), np.ascontiguousarray(qw, np.int8)
+    sx, sw = np.ascontiguousarray(sx, np.float32), np.ascontiguousarray(sw, np.float32)
+    M, K = qx.shape
+    N = qw.shape[0]
+    assert qw.shape[1] == K and K % WBLK == 0
+    y = np.empty((M, N), np.float64)
+    lib().orc_w8a8_gemm(_p(qx), _p(sx), _p(qw), _p(sw), M, N, K, _p(y))
+    return y
+
+
+def w8a8_linear(x, w) -> dict:
+    """The W8A8 layer from bf16 x [M][K] and W [N][K]: codes, scales and y (fp64)."""
+    qx, qw = w8a8_quant(x), w8a8_quant(w)
+    return {"qx": qx["q"], "sx": qx["s"], "qw": qw["q"], "sw": qw["s"],
+            "y": w8a8_gemm(qx["q"], qx["s"], qw["q"], qw["s"])}
