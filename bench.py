@@ -364,6 +364,66 @@ def run_reference(args):
     return 0
 
 
+W8A8_SHAPES = {  # tokens x in -> out: the Wan2.1-14B hidden size (5120) at the 720p token count
+    "w8a8_wan14b_720p_qkvo": (75600, 5120, 5120),
+    "w8a8_wan14b_720p_ffn_up": (75600, 5120, 13824),
+}
+
+
+def run_w8a8(args):
+    """The W8A8 linear layer (x [M, K] quantised every call, W [N, K] quantised once):
+    dense-equivalent TFLOPS = 2 M N K / t of one sagesla_w8a8_linear call."""
+    import torch
+
+    from sparse_bit_attention_smoothing_b200 import build as sbuild
+    from sparse_bit_attention_smoothing_b200.replicas import job_throughput, max_over_ranks, rank_env
+    rank, world, local = rank_env()
+    torch.cuda.set_device(local)
+    sbuild.build()
+    import sparse_bit_attention_smoothing_b200 as sg
+    M, K, N = W8A8_SHAPES[args.workload]
+    g = torch.Generator().manual_seed(0)
+    x = torch.randn(M, K, generator=g).bfloat16().cuda()
+    w = (torch.randn(N, K, generator=g) * K ** -0.5).bfloat16().cuda()
+    wq, sw = sg.sagesla_w8a8_quant(w)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    st = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        sg.sagesla_w8a8_linear(x, wq, sw, N, y=y, stream=st)
+    torch.cuda.synchronize()
+    sg.profile(True)
+    sg.profile_read()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        sg.sagesla_w8a8_linear(x, wq, sw, N, y=y, stream=st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    prof = sg.profile_read()
+    sg.profile(False)
+    ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], device="cuda")[0]
+    flops = 2.0 * M * N * K
+    pk = peaks()
+    peak8 = 2.0 * pk["bf16"]
+    g_ms = prof["w8a8_gemm"][0] / max(1, prof["w8a8_gemm"][1])
+    achieved = flops / (g_ms * 1e-3) / 1e12
+    line = {"metric": "W8A8 linear dense TFLOPS (2MNK / t)", "value": job_throughput(flops, world, ms) / 1e12,
+            "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "i8 (int32 per 128-block, fp32 promotion, bf16 io)", "data": "synthetic",
+            "config": {"workload": args.workload, "M": M, "K": K, "N": N, "block": 128,
+                       "l2": "x 774 MB > 126 MB L2, no flush"},
+            "kernels_ms": {kname: round(t / max(1, n), 4) for kname, (t, n) in prof.items()},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak8, "unit": "TFLOP/s",
+                         "frac": achieved / peak8, "kernel": "w8a8_gemm",
+                         "frac_of_nominal_8bit": achieved / NOMINAL_8BIT_TFLOPS,
+                         "peak_note": f"8-bit = 2 x {pk['src']} bf16 burst {pk['bf16']}"},
+            "device_status": sg.sync_status()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -383,6 +443,8 @@ def main():
         return run_reference(args)
     if args.workload == "all":
         return run_all(args)
+    if args.workload.startswith("w8a8"):
+        return run_w8a8(args)
 
     import torch
     import torch.distributed as dist

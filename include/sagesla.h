@@ -205,6 +205,41 @@ int sagesla_watchdog_selftest(int probes, sagesla_stream_t stream);
 int sagesla_debug_flash_stall(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,
                               float topk, int grid, int stall_step, long long spin_limit, sagesla_stream_t stream);
 
+/*
+ * W8A8 linear layer: y = x W^T with weights and activations both INT8,
+ * quantised in blocks of 128 x 128 ("揭秘TurboDiffusion：如何让视频生成实现
+ * 百倍加速？", 支柱三 W8A8线性层量化; 量子位 news, 技术解密 4).
+ * Reading (the pages give only the block size): one fp32 scale per 128 x 128
+ * block of x [M][K] and of W [N][K] (the nn.Linear convention), the same
+ * symmetric quantiser as Q and K above (s = amax/127, code = RNE(x*127/amax)
+ * clamped to +-127, amax = 0 -> s = 1, codes 0; a last block of rows shorter
+ * than 128 is quantised over its valid rows), and
+ *   y[m][n] = sum over 128-wide K blocks kb of
+ *             s_x[m/128][kb] * s_w[n/128][kb] * (integer dot on kb),
+ * accumulated in fp32 in kb order, rounded once to bf16.
+ *
+ * Code layout ("tile images"): for a [rows][cols] matrix, ceil(rows/128) x
+ * (cols/128) blocks of 16384 bytes in [row block][column block] order; in a
+ * block, code (r, c) sits at byte (r/8)*1024 + (c/16)*128 + (r%8)*16 + c%16
+ * (the tcgen05 K-major no-swizzle operand image); rows past `rows` hold 0.
+ * Scales: fp32 [ceil(rows/128)][cols/128].
+ *
+ * sagesla_w8a8_quant: codes and scales of a bf16 [rows][cols] device matrix
+ *   (cols a multiple of 128; rows <= 8388480).  Used once for W, and by
+ *   sagesla_w8a8_linear for x.  a, codes 16-byte aligned; scales 4-byte.
+ * sagesla_w8a8_gemm: y (bf16 [M][N] device, 16-byte aligned) from the codes
+ *   and scales of x ([M][K]) and W ([N][K]); N, K multiples of 128.
+ * sagesla_w8a8_linear: quantises x (bf16 [M][K] device) into the library's
+ *   workspace of the stream, then the GEMM.
+ * All three are asynchronous on `stream` and return SAGESLA_ERR_INVALID /
+ * SAGESLA_ERR_MISALIGNED without launching on a bad argument.
+ */
+int sagesla_w8a8_quant(const void* a, int rows, int cols, void* codes, float* scales, sagesla_stream_t stream);
+int sagesla_w8a8_gemm(const void* xq, const float* sx, const void* wq, const float* sw, void* y, int M, int N, int K,
+                      sagesla_stream_t stream);
+int sagesla_w8a8_linear(const void* x, const void* wq, const float* sw, void* y, int M, int N, int K,
+                        sagesla_stream_t stream);
+
 /* Human-readable text for a return code (static storage). */
 const char* sagesla_strerror(int code);
 
@@ -216,10 +251,11 @@ const char* sagesla_strerror(int code);
  * forgets them.  Kernel ids: 0 stats, 1 stats finalise, 2 quantise,
  * 3 pooled top-k, 4 linear per-block phi(K)^T V, 5 linear complement sum,
  * 6 sparse flash, 7 projection-weight tiling, 8 linear output (phi(Q) H,
- * normalisation, projection).  ms / launches are arrays of nkernels entries
- * (either may be NULL).  Profiling is off by default.
+ * normalisation, projection), 9 W8A8 block quantiser, 10 W8A8 GEMM.
+ * ms / launches are arrays of nkernels entries (either may be NULL).
+ * Profiling is off by default.
  */
-#define SAGESLA_NUM_KERNELS 9
+#define SAGESLA_NUM_KERNELS 11
 void sagesla_profile(int enable);
 int sagesla_profile_read(double* ms, int* launches, int nkernels);
 

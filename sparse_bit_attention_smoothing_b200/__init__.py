@@ -30,9 +30,9 @@ class SageSLAError(RuntimeError):
 EXPORTS = ["sagesla_attn", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
            "sagesla_smooth_stats_noalloc", "sagesla_topk_count", "sagesla_sync_status", "sagesla_strerror",
            "sagesla_release", "sagesla_profile", "sagesla_profile_read", "sagesla_watchdog_selftest",
-           "sagesla_debug_flash_stall"]
+           "sagesla_debug_flash_stall", "sagesla_w8a8_quant", "sagesla_w8a8_gemm", "sagesla_w8a8_linear"]
 KERNELS = ["stats", "stats_final", "quant", "pool_topk", "linear_kv", "linear_sum", "flash", "w_tile",
-           "linear_apply"]
+           "linear_apply", "w8a8_quant", "w8a8_gemm"]
 
 
 def lib():
@@ -53,6 +53,9 @@ def lib():
         L.sagesla_sync_status.argtypes = [P]
         L.sagesla_watchdog_selftest.argtypes = [i, P]
         L.sagesla_debug_flash_stall.argtypes = [P, P, P, P, i, i, i, i, f, i, i, ctypes.c_longlong, P]
+        L.sagesla_w8a8_quant.argtypes = [P, i, i, P, P, P]
+        L.sagesla_w8a8_gemm.argtypes = [P, P, P, P, P, i, i, i, P]
+        L.sagesla_w8a8_linear.argtypes = [P, P, P, P, i, i, i, P]
         L.sagesla_strerror.restype = ctypes.c_char_p
         L.sagesla_strerror.argtypes = [i]
         L.sagesla_release.restype = None
@@ -189,6 +192,44 @@ def sagesla_debug_flash_stall(q, k, v, out=None, topk: float = 0.1, grid: int = 
                                            grid, stall_step, spin_limit, _stream(stream)),
            "sagesla_debug_flash_stall")
     return out
+
+
+W8A8_BLOCK = 128
+
+
+def sagesla_w8a8_quant(a, stream=None):
+    """INT8 codes (tile images, uint8 [ceil(rows/128) * cols/128 * 16384]) and fp32 scales
+    [ceil(rows/128), cols/128] of a bf16 CUDA matrix [rows, cols] in 128 x 128 blocks."""
+    import torch
+    assert a.dim() == 2 and a.dtype == torch.bfloat16 and a.is_contiguous()
+    rows, cols = a.shape
+    nrb, ncb = (rows + W8A8_BLOCK - 1) // W8A8_BLOCK, cols // W8A8_BLOCK
+    codes = torch.empty(nrb * ncb * W8A8_BLOCK * W8A8_BLOCK, dtype=torch.uint8, device=a.device)
+    scales = torch.empty(nrb, ncb, dtype=torch.float32, device=a.device)
+    _check(lib().sagesla_w8a8_quant(_ptr(a), rows, cols, _ptr(codes), _ptr(scales), _stream(stream)),
+           "sagesla_w8a8_quant")
+    return codes, scales
+
+
+def sagesla_w8a8_gemm(xq, sx, wq, sw, M: int, N: int, K: int, y=None, stream=None):
+    """y = x W^T (bf16 [M, N]) from the codes and scales of x [M, K] and W [N, K]."""
+    import torch
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=xq.device)
+    _check(lib().sagesla_w8a8_gemm(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(y), M, N, K, _stream(stream)),
+           "sagesla_w8a8_gemm")
+    return y
+
+
+def sagesla_w8a8_linear(x, wq, sw, N: int, y=None, stream=None):
+    """The W8A8 layer: quantise x (bf16 [M, K]) and multiply by the quantised W [N, K]."""
+    import torch
+    M, K = x.shape
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _check(lib().sagesla_w8a8_linear(_ptr(x), _ptr(wq), _ptr(sw), _ptr(y), M, N, K, _stream(stream)),
+           "sagesla_w8a8_linear")
+    return y
 
 
 def sync_status(stream=None) -> int:

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsagesla.so")
-SOURCES = ["k_prologue.cu", "k_topk.cu", "k_linear.cu", "k_flash.cu", "k_flash64.cu", "k_watchdog.cu", "api.cu", "noalloc.cu"]
+SOURCES = ["k_prologue.cu", "k_topk.cu", "k_linear.cu", "k_flash.cu", "k_flash64.cu", "k_watchdog.cu", "k_w8a8.cu", "api.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

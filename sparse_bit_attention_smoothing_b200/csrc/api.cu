@@ -303,6 +303,16 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
   return SAGESLA_OK;
 }
 
+int check_gemm(const void* xq, const float* sx, const void* wq, const float* sw, const void* y, int M, int N, int K) {
+  if (!xq || !sx || !wq || !sw || !y || M < 1 || N < 128 || K < 128 || N % 128 != 0 || K % 128 != 0 ||
+      M > 8388480 || (double)M * N >= 1099511627776.0 || (double)M * K >= 1099511627776.0)
+    return SAGESLA_ERR_INVALID;
+  if (!aligned16(xq) || !aligned16(wq) || !aligned16(y) || (reinterpret_cast<uintptr_t>(sx) & 3u) ||
+      (reinterpret_cast<uintptr_t>(sw) & 3u))
+    return SAGESLA_ERR_MISALIGNED;
+  return SAGESLA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -499,6 +509,51 @@ int sagesla_debug_flash_stall(const void* q, const void* k, const void* v, void*
   if (grid < 1 || stall_step < -1 || spin_limit < 1024 || spin_limit > kSpinLimit) return SAGESLA_ERR_INVALID;
   return run_attn(q, k, v, nullptr, out, B, H, N, d, 64, topk, reinterpret_cast<cudaStream_t>(stream), grid,
                   stall_step + 1, (long)spin_limit);
+}
+
+// ------------------------------------------------------------- W8A8 linear
+int sagesla_w8a8_quant(const void* a, int rows, int cols, void* codes, float* scales, sagesla_stream_t stream) {
+  if (!a || !codes || !scales || rows < 1 || cols < 128 || cols % 128 != 0 || rows > 8388480 ||
+      (double)rows * cols >= 1099511627776.0)
+    return SAGESLA_ERR_INVALID;
+  if (!aligned16(a) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return SAGESLA_ERR_MISALIGNED;
+  int dev = 0;
+  SAGESLA_TRY(check_device(&dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  ProfScope ps(9, st);
+  return launch_rc(launch_w8a8_quant(a, rows, cols, static_cast<uint8_t*>(codes), scales, st));
+}
+
+
+int sagesla_w8a8_gemm(const void* xq, const float* sx, const void* wq, const float* sw, void* y, int M, int N, int K,
+                      sagesla_stream_t stream) {
+  SAGESLA_TRY(check_gemm(xq, sx, wq, sw, y, M, N, K));
+  int dev = 0;
+  SAGESLA_TRY(check_device(&dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  ProfScope ps(10, st);
+  return launch_rc(launch_w8a8_gemm(static_cast<const uint8_t*>(xq), sx, static_cast<const uint8_t*>(wq), sw, y, M, N,
+                                    K, watchdog(dev), st));
+}
+
+int sagesla_w8a8_linear(const void* x, const void* wq, const float* sw, void* y, int M, int N, int K,
+                        sagesla_stream_t stream) {
+  if (!x) return SAGESLA_ERR_INVALID;
+  const float one = 1.f;
+  SAGESLA_TRY(check_gemm(x, &one, wq, sw, y, M, N, K));  // x stands in for its codes in the checks
+  int dev = 0;
+  SAGESLA_TRY(check_device(&dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t cb = up(w8a8_codes_bytes(M, K));
+  uint8_t* base = nullptr;
+  SAGESLA_TRY(get_workspace(dev, st, cb + w8a8_scales_count(M, K) * sizeof(float), &base));
+  float* sx = reinterpret_cast<float*>(base + cb);
+  {
+    ProfScope ps(9, st);
+    SAGESLA_TRY(launch_rc(launch_w8a8_quant(x, M, K, base, sx, st)));
+  }
+  ProfScope ps(10, st);
+  return launch_rc(launch_w8a8_gemm(base, sx, static_cast<const uint8_t*>(wq), sw, y, M, N, K, watchdog(dev), st));
 }
 
 int sagesla_sync_status(sagesla_stream_t stream) {

@@ -69,6 +69,12 @@ struct FlashArgs {
   long dbg_spin;
 };
 cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int* wd);
+// W8A8 linear layer (k_w8a8.cu).
+size_t w8a8_codes_bytes(int rows, int cols);
+size_t w8a8_scales_count(int rows, int cols);
+cudaError_t launch_w8a8_quant(const void* a, int rows, int cols, uint8_t* codes, float* scales, cudaStream_t st);
+cudaError_t launch_w8a8_gemm(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw, void* y, int M,
+                             int N, int K, int* wd, cudaStream_t st);
 // Waits `probes` times on an mbarrier that never completes, then sets *wd.
 cudaError_t launch_watchdog_selftest(int probes, int* wd, cudaStream_t st);
 

@@ -56,3 +56,27 @@ def compare_masks(gpu_idx: np.ndarray, orc_idx: np.ndarray, scores64: np.ndarray
         assert not bad, f"row {r}: blocks {bad} differ and are not near-ties of the k-th score"
         near += 1
     return equal, near
+
+
+def untile_codes(codes: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """W8A8 tile images (16 KB per 128 x 128 block, [row block][column block],
+    code (r, c) at (r/8)*1024 + (c/16)*128 + (r%8)*16 + c%16) -> int8 [rows][cols]."""
+    nrb, ncb = (rows + 127) // 128, cols // 128
+    t = np.asarray(codes, np.uint8).view(np.int8).reshape(nrb, ncb, 16, 8, 8, 16)  # [rb][cb][r/8][c/16][r%8][c%16]
+    full = t.transpose(0, 2, 4, 1, 3, 5).reshape(nrb * 128, ncb * 128)
+    return full[:rows]
+
+
+def w8a8_check(y_gpu, y_orc, abs_dot, nk: int):
+    """W8A8 output rule: |y_gpu - y| <= half a bf16 ulp of the larger of the two
+    plus the fp32 accumulation bound (nk + 2) * 2^-24 * sum |terms| (abs_dot =
+    |x^| |w^|^T of the dequantised operands bounds that sum).  Returns the
+    fraction of outputs equal to the correctly rounded bf16 of the exact y."""
+    g = np.asarray(y_gpu, np.float64)
+    y = np.asarray(y_orc, np.float64)
+    tol = np.maximum(bf16_half_ulp(g), bf16_half_ulp(y)) + (nk + 2) * 2.0 ** -24 * abs_dot
+    bad = np.abs(g - y) > tol
+    assert not bad.any(), f"{int(bad.sum())} outputs beyond the bound, worst excess {float(np.max(np.abs(g - y) - tol))}"
+    import torch
+    rne = torch.from_numpy(y).to(torch.bfloat16).double().numpy()
+    return float(np.mean(g == rne))

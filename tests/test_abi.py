@@ -81,6 +81,17 @@ def test_rejects_bad_arguments_without_launch(L):
         assert L.sagesla_attn(a, a, a, None, a, 1, 1, n_max + 1, 128, blk, F(0.1), None) == -1
         assert L.sagesla_attn(a, a, a, None, a, 1, 1, n_max, 128, blk, F(0.1), None) != -1
     assert L.sagesla_watchdog_selftest((1 << 20) + 1, None) == -1
+    # W8A8: shapes that are not multiples of the 128 x 128 block, null and misaligned pointers
+    sp = P(0x20000)
+    assert L.sagesla_w8a8_quant(a, 128, 100, a, sp, None) == -1
+    assert L.sagesla_w8a8_quant(a, 0, 128, a, sp, None) == -1
+    assert L.sagesla_w8a8_quant(None, 128, 128, a, sp, None) == -1
+    assert L.sagesla_w8a8_quant(P(0x10008), 128, 128, a, sp, None) == -2
+    assert L.sagesla_w8a8_gemm(a, sp, a, sp, a, 128, 100, 128, None) == -1
+    assert L.sagesla_w8a8_gemm(a, sp, a, sp, a, 128, 128, 64, None) == -1
+    assert L.sagesla_w8a8_gemm(a, sp, a, sp, P(0x10008), 128, 128, 128, None) == -2
+    assert L.sagesla_w8a8_linear(None, a, sp, a, 128, 128, 128, None) == -1
+    assert L.sagesla_w8a8_linear(a, a, sp, a, 0, 128, 128, None) == -1
     ll = ctypes.c_longlong
     for grid, stall, spin in ((0, -1, 1 << 14), (1, -2, 1 << 14), (1, 0, 1023), (1, 0, (1 << 24) + 1)):
         assert L.sagesla_debug_flash_stall(a, a, a, a, 1, 1, 64, 128, F(0.1), grid, stall, ll(spin), None) == -1
