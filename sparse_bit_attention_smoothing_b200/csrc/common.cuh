@@ -201,6 +201,13 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x1.b32 {%0}, [%1], " #split ";" \
                : "=r"((r)[0])                                                        \
                : "r"(taddr))
+#define SAGESLA_TMEM_LD2H_X8(taddr, split, r)                                   \
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], " #split ";" \
+               : "=r"((r)[0]), "=r"((r)[1]), "=r"((r)[2]), "=r"((r)[3]), "=r"((r)[4]), "=r"((r)[5]), "=r"((r)[6]), "=r"((r)[7])                                                        \
+               : "r"(taddr))
+#define SAGESLA_TMEM_ST2H_X8(taddr, split, r)                                   \
+  asm volatile("tcgen05.st.sync.aligned.16x32bx2.x8.b32 [%0], " #split ", {%1,%2,%3,%4,%5,%6,%7,%8};" \
+               ::"r"(taddr), "r"((r)[0]), "r"((r)[1]), "r"((r)[2]), "r"((r)[3]), "r"((r)[4]), "r"((r)[5]), "r"((r)[6]), "r"((r)[7]))
 #define SAGESLA_TMEM_LD2H_X16(taddr, split, r)                                   \
   asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], " #split ";" \
                : "=r"((r)[0]), "=r"((r)[1]), "=r"((r)[2]), "=r"((r)[3]), "=r"((r)[4]), "=r"((r)[5]), "=r"((r)[6]), "=r"((r)[7]), "=r"((r)[8]), "=r"((r)[9]), "=r"((r)[10]), "=r"((r)[11]), "=r"((r)[12]), "=r"((r)[13]), "=r"((r)[14]), "=r"((r)[15])                                                        \
