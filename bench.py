@@ -424,6 +424,64 @@ def run_w8a8(args):
     return 0
 
 
+def run_head_parallel(args):
+    """One sagesla_attn call of the workload split over the ranks by head: each rank holds its token shard
+    [B, H, N/P, d] of q, k, v, two all-to-alls (NCCL) regroup by head and back.  value = the whole call's
+    dense-equivalent TFLOPS over the slowest rank's time (strong scaling)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from sparse_bit_attention_smoothing_b200 import build as sbuild
+    from sparse_bit_attention_smoothing_b200.replicas import max_over_ranks, rank_env
+    rank, world, local = rank_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    sbuild.build()
+    import sparse_bit_attention_smoothing_b200 as sg
+    from sparse_bit_attention_smoothing_b200.headpar import sagesla_attn_head_parallel
+    from sparse_bit_attention_smoothing_b200.inputs import make_workload
+    w = workloads()[args.workload]
+    q, k, v, pw = make_workload(w)
+    if w.N % world or w.H % world:
+        raise SystemExit(f"head-parallel run needs N ({w.N}) and H ({w.H}) divisible by {world}")
+    Nl = w.N // world
+    sl = slice(rank * Nl, (rank + 1) * Nl)
+    ql, kl, vl = (t[:, :, sl].contiguous().cuda() for t in (q, k, v))
+    dw = pw.cuda() if (w.linear and not args.no_linear) else None
+    st = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        sagesla_attn_head_parallel(ql, kl, vl, dw, block=w.block, topk=w.topk, stream=st)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        out = sagesla_attn_head_parallel(ql, kl, vl, dw, block=w.block, topk=w.topk, stream=st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], device="cuda")[0]
+    f = flops(w, sg.topk_count((w.N + w.block - 1) // w.block, w.topk))
+    line = {"metric": METRIC + " (one call split by head over the ranks)", "value": f["dense"] / (ms * 1e-3) / 1e12,
+            "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "i8/e4m3 (fp32 accumulate, bf16 io)", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.block, "topk": w.topk,
+                       "linear": dw is not None, "parallelism": f"heads x{world} (all-to-all, NCCL)"},
+            "device_status": sg.sync_status(), "out_shape": list(out.shape)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,6 +493,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-linear", action="store_true", help="proj_w = NULL (linear branch off)")
     ap.add_argument("--peaks", action="store_true", help="measure the 8-bit library GEMM peaks and exit")
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "heads"],
+                    help="replicas: one independent call per rank (weak scaling); heads: one call split over the "
+                         "ranks by head with two all-to-alls (strong scaling)")
     args = ap.parse_args()
     if args.peaks:
         print(json.dumps({"n": 8192, "peaks": measure_8bit_peaks()}), flush=True)
@@ -445,6 +506,8 @@ def main():
         return run_all(args)
     if args.workload.startswith("w8a8"):
         return run_w8a8(args)
+    if args.parallel == "heads":
+        return run_head_parallel(args)
 
     import torch
     import torch.distributed as dist

@@ -185,3 +185,17 @@ def test_host_entry_point_matches_device_path(sg):
         sg.sagesla_attn_host(hq, hk, hv, hw, out=hout, block=64, topk=0.2)
         assert sg.sync_status() == 0
         assert torch.equal(hout, ref.cpu())
+
+
+def test_head_parallel_single_rank_is_the_device_call(sg):
+    """The head-parallel entry on one rank (no process group) runs the library's
+    CUDA call on whole heads: bit-identical to sagesla_attn."""
+    from sparse_bit_attention_smoothing_b200.headpar import sagesla_attn_head_parallel
+    from sparse_bit_attention_smoothing_b200.inputs import make_inputs
+    q, k, v, w = make_inputs(1, 4, 1000, 128, seed=13, outliers=True)
+    dq, dk, dv, dw = q.cuda(), k.cuda(), v.cuda(), w.cuda()
+    a = sg.sagesla_attn(dq, dk, dv, dw, block=64, topk=0.25)
+    b = sagesla_attn_head_parallel(dq, dk, dv, dw, block=64, topk=0.25)
+    torch.cuda.synchronize()
+    assert sg.sync_status() == 0
+    assert torch.equal(a, b)
