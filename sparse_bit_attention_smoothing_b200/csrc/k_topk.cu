@@ -25,6 +25,17 @@ __device__ __forceinline__ uint32_t order_key(float s) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// 16-byte asynchronous global -> shared copy; src_bytes = 0 fills zeros.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Mean over the valid rows of attention block `blk` from the per-64-row sums.
 __device__ __forceinline__ float pooled(const float* __restrict__ sums, int blk, int block, int N, int c) {
   const int sub = block / kQB;
@@ -257,6 +268,159 @@ __global__ void __launch_bounds__(32 * TQ) pool_topk_kernel(const float* __restr
   }
 }
 
+// Sixteen query blocks per CTA, 512 threads (one CTA per SM), for nb <=
+// 1280.  Phase 1: the kbar chunks are double-buffered with cp.async, so the
+// next chunk streams in while this one is scored; thread t takes key t % 64,
+// channel quarter (t / 64) % 4 and query rows 8 * (t / 256) .. + 7.
+// Phase 2 as above, one warp per query row; Z_i gathers 16 rows of z at a
+// time.
+constexpr int kTQ16 = 16, kPER16 = 40;
+__global__ void __launch_bounds__(512, 1) pool_topk16_kernel(const float* __restrict__ qbar,
+                                                            const float* __restrict__ kbar, int nb, int kc,
+                                                            int32_t* __restrict__ idx, const float* __restrict__ zin,
+                                                            const float* __restrict__ ztot,
+                                                            uint32_t* __restrict__ selbits, int nbw,
+                                                            float* __restrict__ zout) {
+  constexpr int kThr = 512;
+  extern __shared__ __align__(16) float sm[];
+  float* qb = sm;                            // [16][128]
+  float* kb = qb + kTQ16 * kD;               // [2][kKC][kPad]
+  float* psc = kb + 2 * kKC * kPad;          // [4][16][kKC] quarter sums
+  float* sc = psc + 4 * kTQ16 * kKC;         // [16][nb]
+  const int bh = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int i0 = blockIdx.x * kTQ16;
+  const float* qh = qbar + (size_t)bh * nb * kD;
+  const float* kh = kbar + (size_t)bh * nb * kD;
+  const float rs = 1.0f / sqrtf((float)kD);
+  const int nchunk = (nb + kKC - 1) / kKC;
+  // Chunk c of kbar into buffer c % 2 (rows past nb read as zeros).
+  auto stage = [&](int c) {
+    float* dst = kb + (c & 1) * kKC * kPad;
+#pragma unroll
+    for (int m = 0; m < kKC * kD / 4 / kThr; ++m) {
+      const int e = t + m * kThr;
+      const int r = e / (kD / 4), c4 = e % (kD / 4);
+      const int j = c * kKC + r;
+      cp_async16(dst + r * kPad + 4 * c4, kh + (size_t)(j < nb ? j : 0) * kD + 4 * c4, j < nb ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+  stage(0);
+  for (int e = t; e < kTQ16 * kD; e += kThr) {
+    const int r = e / kD;
+    qb[e] = i0 + r < nb ? qh[(size_t)i0 * kD + e] : 0.f;
+  }
+  const int jj = t & 63, qg = (t >> 6) & 3, rg = t >> 8;
+  for (int c = 0; c < nchunk; ++c) {
+    if (c + 1 < nchunk) {
+      stage(c + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();  // chunk c is in buffer c % 2 for every thread
+    const float* kr = kb + (c & 1) * kKC * kPad + jj * kPad + 32 * qg;
+    float a[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) a[r] = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < 32; cc += 4) {
+      const float4 k4 = *reinterpret_cast<const float4*>(kr + cc);
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const float4 x = *reinterpret_cast<const float4*>(qb + (8 * rg + r) * kD + 32 * qg + cc);
+        a[r] = fmaf(x.x, k4.x, a[r]);
+        a[r] = fmaf(x.y, k4.y, a[r]);
+        a[r] = fmaf(x.z, k4.z, a[r]);
+        a[r] = fmaf(x.w, k4.w, a[r]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) psc[(qg * kTQ16 + 8 * rg + r) * kKC + jj] = a[r];
+    __syncthreads();  // quarter sums complete; buffer c % 2 may be refilled
+    for (int e = t; e < kTQ16 * kKC; e += kThr) {
+      const int r = e / kKC, k = e % kKC, jk = c * kKC + k;
+      if (jk < nb)
+        sc[r * nb + jk] = ((psc[(0 * kTQ16 + r) * kKC + k] + psc[(1 * kTQ16 + r) * kKC + k]) +
+                           (psc[(2 * kTQ16 + r) * kKC + k] + psc[(3 * kTQ16 + r) * kKC + k])) * rs;
+    }
+  }
+  __syncthreads();
+  // Phase 2: one warp per query row.
+  const int i = i0 + warp;
+  if (i >= nb) return;
+  const float* row = sc + warp * nb;
+  int* lst = reinterpret_cast<int*>(sc + warp * nb);
+  uint32_t keys[kPER16];
+#pragma unroll
+  for (int u = 0; u < kPER16; ++u) {
+    const int j = 32 * u + lane;
+    keys[u] = j < nb ? order_key(row[j]) : 0u;  // 0 is never counted: every candidate is >= 1
+  }
+  uint32_t T = 0;
+  for (int b = 31; b >= 0; --b) {
+    const uint32_t cand = T | (1u << b);
+    int c4[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int u = 0; u < kPER16; ++u) c4[u & 3] += keys[u] >= cand ? 1 : 0;
+    const int cnt = __reduce_add_sync(0xffffffffu, (c4[0] + c4[1]) + (c4[2] + c4[3]));
+    if (cnt >= kc) T = cand;
+  }
+  int gt = 0;
+#pragma unroll
+  for (int u = 0; u < kPER16; ++u) gt += (32 * u + lane < nb && keys[u] > T) ? 1 : 0;
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  const int need_eq = kc - gt;
+  int32_t* out = idx + ((size_t)bh * nb + i) * kc;
+  int pos = 0, eq_seen = 0;
+  const int nch = (nb + 31) >> 5;
+#pragma unroll
+  for (int u = 0; u < kPER16; ++u) {
+    if (u >= nch) break;
+    const int j = 32 * u + lane;
+    const uint32_t key = j < nb ? keys[u] : 0u;
+    const bool is_eq = j < nb && key == T;
+    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+    const int eq_rank = eq_seen + __popc(eqm & ((1u << lane) - 1u));
+    const bool sel = j < nb && (key > T || (is_eq && eq_rank < need_eq));
+    const unsigned sm_ = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const int at = pos + __popc(sm_ & ((1u << lane) - 1u));
+      out[at] = j;
+      lst[at] = j;
+    }
+    if (selbits && lane == 0) selbits[((size_t)bh * nb + i) * nbw + u] = sm_;
+    pos += __popc(sm_);
+    eq_seen += __popc(eqm);
+  }
+  if (selbits)
+    for (int w = nch + lane; w < nbw; w += 32) selbits[((size_t)bh * nb + i) * nbw + w] = 0u;
+  if (zin) {
+    __syncwarp();
+    float zs[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) zs[m] = 0.f;
+    const float* zh = zin + (size_t)bh * nb * kD + lane;
+    // Sixteen rows of z in flight per lane; added in list order.
+    for (int t0 = 0; t0 < kc; t0 += 16) {
+      float v[16][4];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int j = t0 + u < kc ? lst[t0 + u] : -1;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) v[u][m] = j >= 0 ? __ldg(zh + (size_t)j * kD + 32 * m) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) zs[m] += v[u][m];
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      zout[((size_t)bh * nb + i) * kD + lane + 32 * m] = ztot[(size_t)bh * kD + lane + 32 * m] - zs[m];
+  }
+}
+
 namespace {
 
 size_t topk_smem(int tq, int nb) {
@@ -289,10 +453,20 @@ cudaError_t launch_pool_topk(const float* qsum, const float* ksum, const Geom& g
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  // Eight query blocks per CTA where the scores fit in shared memory (82 KB
-  // and 256 threads at nb = 1182: two CTAs per SM), and the order keys in
-  // registers up to nb = 1280.
+  // Sixteen query blocks per CTA (512 threads, double-buffered kbar chunks,
+  // one CTA per SM) up to nb = 1280, where the order keys fit in registers;
+  // else eight query blocks per CTA where the scores fit in shared memory;
+  // else four.
   constexpr size_t kSmemMax = 227 * 1024;
+  if (g.nb <= 32 * kPER16) {
+    const size_t smem = sizeof(float) * ((size_t)kTQ16 * kD + 2 * (size_t)kKC * kPad + 4 * (size_t)kTQ16 * kKC +
+                                         (size_t)kTQ16 * g.nb);
+    e = cudaFuncSetAttribute(pool_topk16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    pool_topk16_kernel<<<dim3((g.nb + kTQ16 - 1) / kTQ16, g.BH), 512, smem, st>>>(
+        qbar, kbar, g.nb, g.kc, idx, zin, ztot, selbits, 2 * ((g.nb + 63) / 64), zout);
+    return cudaGetLastError();
+  }
   if (topk_smem(8, g.nb) <= kSmemMax)
     return g.nb <= 32 * 40 ? launch_topk_cfg<8, 40>(qbar, kbar, g, idx, zin, ztot, selbits, zout, st)
                            : launch_topk_cfg<8, 0>(qbar, kbar, g, idx, zin, ztot, selbits, zout, st);
