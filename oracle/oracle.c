@@ -114,6 +114,14 @@ int8_t orc_int8_code(float x, float mult) {
   if (r < -127.f) r = -127.f;
   return (int8_t)r;
 }
+/* Same with a symmetric range of +-qmax (127: INT8; 7: the INT4 variant). */
+static int8_t orc_qcode(float x, float mult, int qmax) {
+  float p = x * mult;
+  float r = nearbyintf(p);
+  if (r > (float)qmax) r = (float)qmax;
+  if (r < -(float)qmax) r = -(float)qmax;
+  return (int8_t)r;
+}
 void orc_int8_code_array(const float* x, float mult, int8_t* out, int64_t n) {
   for (int64_t i = 0; i < n; ++i) out[i] = orc_int8_code(x[i], mult);
 }
@@ -208,9 +216,12 @@ static void smooth_mean(const uint16_t* k, int N, int d, float* mu) {
   }
 }
 
+/* qmax = 127 (INT8) or 7 (the INT4 variant); q_per_token != 0: one Q scale
+ * per token (sq has N entries) instead of one per 64-token block. */
 static void quant_head(const uint16_t* q, const uint16_t* k, const uint16_t* v, int N, int d,
                        float* mu, float* ks_out /* [N][d] or NULL */, int8_t* q8, int8_t* k8,
-                       uint8_t* v8, float* sq, float* sk, float* sv) {
+                       uint8_t* v8, float* sq, float* sk, float* sv, int qmax, int q_per_token) {
+  const float fq = (float)qmax;
   smooth_mean(k, N, d, mu);
   float* ks = ks_out ? ks_out : (float*)malloc(sizeof(float) * (int64_t)N * d);
   for (int n = 0; n < N; ++n)
@@ -227,15 +238,26 @@ static void quant_head(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
         if (xq > aq) aq = xq;
         if (xk > ak) ak = xk;
       }
-    float mq = aq > 0.f ? 127.f / aq : 0.f;
-    float mk = ak > 0.f ? 127.f / ak : 0.f;
-    sq[t] = aq > 0.f ? aq / 127.f : 1.f;
-    sk[t] = ak > 0.f ? ak / 127.f : 1.f;
-    for (int n = n0; n < n1; ++n)
-      for (int c = 0; c < d; ++c) {
-        q8[(int64_t)n * d + c] = orc_int8_code(bf16_f32(q[(int64_t)n * d + c]), mq);
-        k8[(int64_t)n * d + c] = orc_int8_code(ks[(int64_t)n * d + c], mk);
+    float mq = aq > 0.f ? fq / aq : 0.f;
+    float mk = ak > 0.f ? fq / ak : 0.f;
+    if (!q_per_token) sq[t] = aq > 0.f ? aq / fq : 1.f;
+    sk[t] = ak > 0.f ? ak / fq : 1.f;
+    for (int n = n0; n < n1; ++n) {
+      float mqn = mq;
+      if (q_per_token) { /* the row's own absmax over its d channels */
+        float an = 0.f;
+        for (int c = 0; c < d; ++c) {
+          float x = fabsf(bf16_f32(q[(int64_t)n * d + c]));
+          if (x > an) an = x;
+        }
+        mqn = an > 0.f ? fq / an : 0.f;
+        sq[n] = an > 0.f ? an / fq : 1.f;
       }
+      for (int c = 0; c < d; ++c) {
+        q8[(int64_t)n * d + c] = orc_qcode(bf16_f32(q[(int64_t)n * d + c]), mqn, qmax);
+        k8[(int64_t)n * d + c] = orc_qcode(ks[(int64_t)n * d + c], mk, qmax);
+      }
+    }
   }
   for (int c = 0; c < d; ++c) {
     float a = 0.f;
@@ -260,7 +282,7 @@ void orc_quant(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, 
   for (int bh = 0; bh < BH; ++bh) {
     int64_t o = (int64_t)bh * N * d;
     quant_head(q + o, k + o, v + o, N, d, mu + (int64_t)bh * d, NULL, q8 + o, k8 + o, v8 + o,
-               sq + (int64_t)bh * nq, sk + (int64_t)bh * nq, sv + (int64_t)bh * d);
+               sq + (int64_t)bh * nq, sk + (int64_t)bh * nq, sv + (int64_t)bh * d, 127, 0);
   }
 }
 
@@ -398,6 +420,12 @@ void orc_block_scores_f64(const uint16_t* q, const uint16_t* k, int BH, int N, i
  * is flags = 0. */
 #define ORC_ALT_WALK128 2 /* update the running max once per 128 keys of the list */
 #define ORC_ALT_LSUM_P 4  /* row sum over the unquantised P instead of P~        */
+/* SageAttention2++ variants (量子位 news, 技术解密 1: INT8 "or even INT4", with
+ * "thread-level quantisation calibration"): one Q scale per token (the unit
+ * a softmax thread owns) instead of per 64-token block, and Q/K codes in
+ * +-7 (4-bit) instead of +-127. */
+#define ORC_Q_PER_TOKEN 8
+#define ORC_QK_INT4 16
 
 typedef struct {
   int N, d, block, nb, kc;
@@ -459,7 +487,8 @@ static void emul_qblock(const orc_head* H, int i, const int32_t* sel, double* ou
             int64_t acc = 0;
             for (int c = 0; c < d; ++c)
               acc += (int64_t)H->q8[(int64_t)n * d + c] * (int64_t)H->k8[(int64_t)kk * d + c];
-            s = (double)acc * (double)H->sq[n / ORC_QBLK] * (double)H->sk[kk / ORC_QBLK] * rsd;
+            s = (double)acc * (double)H->sq[(H->flags & ORC_Q_PER_TOKEN) ? n : n / ORC_QBLK] *
+                (double)H->sk[kk / ORC_QBLK] * rsd;
           }
           sc[(t - t0) * block + (kk - k0)] = s;
           if (s > mj) mj = s;
@@ -581,10 +610,11 @@ int orc_sagesla(const uint16_t* q, const uint16_t* k, const uint16_t* v, const u
     int8_t* q8 = (int8_t*)malloc((size_t)N * d);
     int8_t* k8 = (int8_t*)malloc((size_t)N * d);
     uint8_t* v8 = (uint8_t*)malloc((size_t)N * d);
-    float* sq = (float*)malloc(sizeof(float) * nq);
+    float* sq = (float*)malloc(sizeof(float) * (nq > N ? nq : N));
     float* sk = (float*)malloc(sizeof(float) * nq);
     float* sv = (float*)malloc(sizeof(float) * d);
-    quant_head(Hd.q, Hd.k, Hd.v, N, d, mu, ks, q8, k8, v8, sq, sk, sv);
+    quant_head(Hd.q, Hd.k, Hd.v, N, d, mu, ks, q8, k8, v8, sq, sk, sv, (flags & ORC_QK_INT4) ? 7 : 127,
+               (flags & ORC_Q_PER_TOKEN) != 0);
     Hd.q8 = q8;
     Hd.k8 = k8;
     Hd.v8 = v8;

@@ -22,6 +22,9 @@ NOQUANT = 1  # test switch: no quantisation anywhere (reduction to dense)
 # readings the pages leave open (the method's reading is flags = 0).
 ALT_WALK128 = 2  # running max updated once per 128 keys of the list
 ALT_LSUM_P = 4  # row sum over the unquantised P instead of P~
+# SageAttention2++ variants (method options, not alternative readings):
+Q_PER_TOKEN = 8  # one Q scale per token instead of per 64-token block
+QK_INT4 = 16     # Q and K codes in +-7 (4-bit) instead of +-127
 
 
 def build(force: bool = False) -> str:
