@@ -106,6 +106,23 @@ int sagesla_attn_host(const void* q, const void* k, const void* v, const void* p
                       int B, int H, int N, int d, int block, float topk, sagesla_stream_t stream);
 
 /*
+ * sagesla_attn_opts: sagesla_attn with the SageAttention2++ quantisation
+ * options (量子位 news, 技术解密 1: codes of 8 and, further, 4 bits, and a
+ * quantisation calibrated per thread):
+ *   qk_bits      8: Q and K codes in +-127 (the default path); 4: codes in
+ *                +-7 with scale amax/7.  tcgen05 has no 4-bit integer MMA, so
+ *                the 4-bit codes run through the same INT8 tensor-core path:
+ *                an accuracy option, not a faster one.
+ *   q_per_token  0: one Q scale per 64-token block (the default path); 1: one
+ *                Q scale per token (the row a softmax thread owns), K keeps
+ *                one scale per 64-token block.
+ * Other arguments and behaviour as sagesla_attn; SAGESLA_ERR_INVALID for
+ * other option values.  sagesla_attn is sagesla_attn_opts(..., 8, 0, ...).
+ */
+int sagesla_attn_opts(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B, int H,
+                      int N, int d, int block, float topk, int qk_bits, int q_per_token, sagesla_stream_t stream);
+
+/*
  * sagesla_get_quant: the smoothing + quantisation step alone (for parity).
  *   q8, k8   int8 [B][H][N][d] device: INT8 codes, row-major.
  *   v8       uint8 [B][H][N][d] device: FP8 E4M3 codes, row-major.

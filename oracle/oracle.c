@@ -420,8 +420,8 @@ void orc_block_scores_f64(const uint16_t* q, const uint16_t* k, int BH, int N, i
  * is flags = 0. */
 #define ORC_ALT_WALK128 2 /* update the running max once per 128 keys of the list */
 #define ORC_ALT_LSUM_P 4  /* row sum over the unquantised P instead of P~        */
-/* SageAttention2++ variants (量子位 news, 技术解密 1: INT8 "or even INT4", with
- * "thread-level quantisation calibration"): one Q scale per token (the unit
+/* SageAttention2++ variants (量子位 news, 技术解密 1: codes of 8 and, further,
+ * 4 bits, and a quantisation calibrated per thread): one Q scale per token (the unit
  * a softmax thread owns) instead of per 64-token block, and Q/K codes in
  * +-7 (4-bit) instead of +-127. */
 #define ORC_Q_PER_TOKEN 8

@@ -27,7 +27,7 @@ class SageSLAError(RuntimeError):
         super().__init__(f"{where}: {ERRORS.get(code, 'error')} ({code})")
 
 
-EXPORTS = ["sagesla_attn", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
+EXPORTS = ["sagesla_attn", "sagesla_attn_opts", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
            "sagesla_smooth_stats_noalloc", "sagesla_topk_count", "sagesla_sync_status", "sagesla_strerror",
            "sagesla_release", "sagesla_profile", "sagesla_profile_read", "sagesla_watchdog_selftest",
            "sagesla_debug_flash_stall", "sagesla_w8a8_quant", "sagesla_w8a8_gemm", "sagesla_w8a8_linear"]
@@ -45,6 +45,7 @@ def lib():
         P, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.sagesla_attn.argtypes = [P, P, P, P, P, i, i, i, i, i, f, P]
         L.dense_int8_attn.argtypes = [P, P, P, P, i, i, i, i, P]
+        L.sagesla_attn_opts.argtypes = [P, P, P, P, P, i, i, i, i, i, f, i, i, P]
         L.sagesla_attn_host.argtypes = [P, P, P, P, P, i, i, i, i, i, f, P]
         L.sagesla_get_quant.argtypes = [P, P, P, i, i, i, i, P, P, P, P, P, P, P, P]
         L.sagesla_get_mask.argtypes = [P, P, i, i, i, i, i, f, P, P, P, P, P]
@@ -100,6 +101,20 @@ def sagesla_attn(q, k, v, proj_w=None, out=None, block: int = 64, topk: float = 
         out = torch.empty_like(q)
     _check(lib().sagesla_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(proj_w), _ptr(out), B, H, N, d, block,
                               ctypes.c_float(topk), _stream(stream)), "sagesla_attn")
+    return out
+
+
+def sagesla_attn_opts(q, k, v, proj_w=None, out=None, block: int = 64, topk: float = 0.1, qk_bits: int = 8,
+                      q_per_token: bool = False, stream=None):
+    """sagesla_attn with the SageAttention2++ quantisation options: qk_bits 8 or 4 (Q/K codes in +-127 or +-7),
+    q_per_token (one Q scale per token instead of per 64-token block)."""
+    import torch
+    B, H, N, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().sagesla_attn_opts(_ptr(q), _ptr(k), _ptr(v), _ptr(proj_w), _ptr(out), B, H, N, d, block,
+                                   ctypes.c_float(topk), qk_bits, 1 if q_per_token else 0, _stream(stream)),
+           "sagesla_attn_opts")
     return out
 
 

@@ -175,7 +175,7 @@ struct Buffers {
   size_t total;
 };
 
-Buffers carve(uint8_t* base, const Geom& g, bool linear = false) {
+Buffers carve(uint8_t* base, const Geom& g, bool linear = false, bool q_tok = false) {
   Buffers b;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -192,7 +192,7 @@ Buffers carve(uint8_t* base, const Geom& g, bool linear = false) {
   b.q8t = take(BH * g.nq * kTile);
   b.k8t = take(BH * g.nq * kTile);
   b.v8t = take(BH * g.nq * kTile);
-  b.sq = reinterpret_cast<float*>(take(BH * g.nq * sizeof(float)));
+  b.sq = reinterpret_cast<float*>(take(BH * g.nq * (q_tok ? kQB : 1) * sizeof(float)));
   b.sk = reinterpret_cast<float*>(take(BH * g.nq * sizeof(float)));
   b.qsum = reinterpret_cast<float*>(take(BH * g.nq * kD * sizeof(float)));
   b.ksum = reinterpret_cast<float*>(take(BH * g.nq * kD * sizeof(float)));
@@ -228,7 +228,7 @@ inline int launch_rc(cudaError_t e) { return e == cudaSuccess ? SAGESLA_OK : SAG
 
 // Stats + quantisation (the front shared by every entry point).
 int run_front(const void* q, const void* k, const void* v, const Geom& g, const Buffers& b, int dev,
-              cudaStream_t st) {
+              cudaStream_t st, int qmax = 127, int q_tok = 0) {
   {
     ProfScope ps(0, st);
     SAGESLA_TRY(launch_rc(launch_stats_partial(k, v, g, b.psum, b.pmax, st)));
@@ -240,13 +240,15 @@ int run_front(const void* q, const void* k, const void* v, const Geom& g, const 
   {
     ProfScope ps(2, st);
     SAGESLA_TRY(launch_rc(
-        launch_quant(q, k, v, b.mu, b.mv, g, b.q8t, b.k8t, b.v8t, b.sq, b.sk, b.qsum, b.ksum, watchdog(dev), st)));
+        launch_quant(q, k, v, b.mu, b.mv, g, b.q8t, b.k8t, b.v8t, b.sq, b.sk, b.qsum, b.ksum, watchdog(dev), st,
+                     qmax, q_tok)));
   }
   return SAGESLA_OK;
 }
 
 int run_attn(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B, int H, int N, int d,
-             int block, float topk, cudaStream_t st, int dbg_grid = 0, int dbg_stall = 0, long dbg_spin = 0) {
+             int block, float topk, cudaStream_t st, int dbg_grid = 0, int dbg_stall = 0, long dbg_spin = 0,
+             int qmax = 127, int q_tok = 0) {
   SAGESLA_TRY(validate(q, k, v, out, B, H, N, d, block, topk));
   if (proj_w && !aligned16(proj_w)) return SAGESLA_ERR_MISALIGNED;
   int dev = 0;
@@ -255,11 +257,11 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
   const bool dense = g.kc == g.nb;
   // An empty complement (every key block selected) makes the linear branch 0.
   const bool linear = proj_w != nullptr && !dense;
-  const Buffers sizes = carve(nullptr, g, linear);
+  const Buffers sizes = carve(nullptr, g, linear, q_tok != 0);
   uint8_t* base = nullptr;
   SAGESLA_TRY(get_workspace(dev, st, sizes.total, &base));
-  const Buffers b = carve(base, g, linear);
-  SAGESLA_TRY(run_front(q, k, v, g, b, dev, st));
+  const Buffers b = carve(base, g, linear, q_tok != 0);
+  SAGESLA_TRY(run_front(q, k, v, g, b, dev, st, qmax, q_tok));
   int* wd = watchdog(dev);
   if (linear) {
     {
@@ -293,6 +295,7 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
   fa.idx = dense ? nullptr : b.idx;
   fa.out = out;
   fa.add_out = linear ? 1 : 0;
+  fa.q_tok = q_tok;
   fa.dbg_grid = dbg_grid;
   fa.dbg_stall = dbg_stall;
   fa.dbg_spin = dbg_spin;
@@ -329,6 +332,13 @@ int sagesla_topk_count(int nb, float topk) {
 int sagesla_attn(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B, int H, int N,
                  int d, int block, float topk, sagesla_stream_t stream) {
   return run_attn(q, k, v, proj_w, out, B, H, N, d, block, topk, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int sagesla_attn_opts(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B, int H,
+                      int N, int d, int block, float topk, int qk_bits, int q_per_token, sagesla_stream_t stream) {
+  if ((qk_bits != 8 && qk_bits != 4) || (q_per_token != 0 && q_per_token != 1)) return SAGESLA_ERR_INVALID;
+  return run_attn(q, k, v, proj_w, out, B, H, N, d, block, topk, reinterpret_cast<cudaStream_t>(stream), 0, 0, 0,
+                  qk_bits == 8 ? 127 : 7, q_per_token);
 }
 
 int dense_int8_attn(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,

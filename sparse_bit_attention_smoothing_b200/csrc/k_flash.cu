@@ -76,6 +76,7 @@ struct Params {
   int units;   // BH * upb
   int nsteps;  // steps per unit
   int add_out; // 1: out already holds the linear branch (bf16); add O_s to it
+  int q_tok;   // 1: one Q scale per token (sq [BH][nq*64])
 };
 
 template <int MODE>
@@ -409,7 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
         qtile = 2 * un.iA + (r >> 6);
         xs = 0;
       }
-      const float c0 = active ? __ldg(p.sq + (size_t)un.bh * p.nq + qtile) * (kLog2e * kRsqrtD) : 0.f;
+      const size_t sqi = (size_t)un.bh * p.nq + qtile;
+      const float c0 = active ? __ldg(p.sq + (p.q_tok ? sqi * kQB + (r & 63) : sqi)) * (kLog2e * kRsqrtD) : 0.f;
       uint8_t* prow = smem + C::kOffP + g * C::kPTile + (MODE == 0 && lane >= 16 ? 4096 : 0);
       float m_all = -INFINITY, frame = -INFINITY;
       for (int s = 0; s < nsteps; ++s, ++gs) {
@@ -683,6 +685,7 @@ cudaError_t launch_flash128(const FlashArgs& a, const Geom& g, cudaStream_t st, 
   p.k8t = a.k8t;
   p.v8t = a.v8t;
   p.sq = a.sq;
+  p.q_tok = a.q_tok;
   p.sk = a.sk;
   p.sv = a.sv;
   p.idx = a.idx;

@@ -94,6 +94,7 @@ struct Params {
   int items;   // BH * nb query blocks
   int nsteps;  // steps per query block: ceil(kc / 2)
   int add_out; // 1: out already holds the linear branch (bf16); add O_s to it
+  int q_tok;    // 1: one Q scale per token (sq [BH][nq*64])
   long spin;    // probe limit of every bounded wait that may give up
   int stall_gs; // >= 0: slot 0's K producer omits the copy of this step (watchdog test)
 };
@@ -328,7 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
     bool ok = true;
     for (int q = 2 * (int)blockIdx.x + X; ok && q < p.items; q += stride) {
       const int bh = q / p.nb, i = q - bh * p.nb;
-      const float c0 = __ldg(p.sq + (size_t)bh * p.nq + i) * (kLog2e * kRsqrtD);
+      const size_t sqi = (size_t)bh * p.nq + i;
+      const float c0 = __ldg(p.sq + (p.q_tok ? sqi * kQB + r : sqi)) * (kLog2e * kRsqrtD);
       float m_all = -INFINITY, frame = -INFINITY;
       for (int s = 0; s < nsteps; ++s, ++gs) {
         const int b = gs & 1;
@@ -546,6 +548,7 @@ cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int
   p.nq = g.nq;
   p.kc = g.kc;
   p.add_out = a.add_out;
+  p.q_tok = a.q_tok;
   p.items = g.BH * g.nb;
   p.nsteps = (g.kc + 1) / 2;
   p.spin = a.dbg_spin > 0 ? a.dbg_spin : kSpinLimit;

@@ -107,12 +107,14 @@ struct QuantSmem {
   uint8_t img[3][kTile];                        // Q^, K^ and V^T tile images
   float psum[2][16][kSumPitch];                 // per-thread column sums of Q and K - mu
   float red[2][8];
+  float rowmax[4][kQB];  // per-token Q absmax: the four channel-quarter warps' partial maxima
   uint64_t full[kQStages];
   int abort;
 };
 
-// rne(fl32(x * mult)) as a byte.  |x| <= amax and mult = fl32(127/amax), so
-// the product lies within 127 * (1 + 2^-23) and no clamp is needed; adding
+// rne(fl32(x * mult)) as a byte.  |x| <= amax and mult = fl32(qmax/amax)
+// (qmax = 127, or 7 for the 4-bit option), so the product lies within
+// qmax * (1 + 2^-23) and no clamp is needed; adding
 // 1.5 * 2^23 rounds it to the nearest integer (ties to even) in the low
 // mantissa bits, on the FMA pipe rather than the conversion unit.
 __device__ __forceinline__ uint32_t i8code(float x, float mult) {
@@ -124,7 +126,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
                  const float* __restrict__ mu, const float* __restrict__ mv, int N, int nq, int ntiles,
                  uint8_t* __restrict__ q8t, uint8_t* __restrict__ k8t, uint8_t* __restrict__ v8t,
                  float* __restrict__ sq, float* __restrict__ sk, float* __restrict__ qsum, float* __restrict__ ksum,
-                 int* wd) {
+                 int* wd, int qmax, int q_tok) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   QuantSmem& S = *reinterpret_cast<QuantSmem*>(smem_raw);
   volatile int* abort = &S.abort;
@@ -249,11 +251,36 @@ __global__ void __launch_bounds__(kQThreads, 1)
       aq = fmaxf(aq, S.red[0][w]);
       ak = fmaxf(ak, S.red[1][w]);
     }
-    const float mq = aq > 0.f ? __fdiv_rn(127.f, aq) : 0.f;
-    const float mk = ak > 0.f ? __fdiv_rn(127.f, ak) : 0.f;
+    const float fq = (float)qmax;
+    const float mq = aq > 0.f ? __fdiv_rn(fq, aq) : 0.f;
+    const float mk = ak > 0.f ? __fdiv_rn(fq, ak) : 0.f;
     if (t == 0) {
-      sq[gt] = aq > 0.f ? __fdiv_rn(aq, 127.f) : 1.f;
-      sk[gt] = ak > 0.f ? __fdiv_rn(ak, 127.f) : 1.f;
+      if (!q_tok) sq[gt] = aq > 0.f ? __fdiv_rn(aq, fq) : 1.f;
+      sk[gt] = ak > 0.f ? __fdiv_rn(ak, fq) : 1.f;
+    }
+    // Per-token Q scales (option): the absmax of each row over its 128
+    // channels.  A row's channels are held by lanes rr, rr+8, rr+16, rr+24 of
+    // the four warps 4h .. 4h+3: shuffles, then the warps' partial maxima
+    // through shared memory (S.rowmax[warp % 4][row]).
+    float mqr[4] = {mq, mq, mq, mq};
+    if (q_tok) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float a = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) a = fmaxf(a, fabsf((c & 1) ? bf16_hi(rq[i][c >> 1]) : bf16_lo(rq[i][c >> 1])));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 16));
+        if (lane < 8) S.rowmax[warp & 3][rr + 32 * h + 8 * i] = a;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = rr + 32 * h + 8 * i;
+        const float a = fmaxf(fmaxf(S.rowmax[0][r], S.rowmax[1][r]), fmaxf(S.rowmax[2][r], S.rowmax[3][r]));
+        mqr[i] = a > 0.f ? __fdiv_rn(fq, a) : 0.f;
+        if ((t & 0x78) == 0) sq[(size_t)gt * kQB + r] = a > 0.f ? __fdiv_rn(a, fq) : 1.f;  // cg == 0 writes
+      }
     }
 
     // ---- Q, K codes into the tile images; partial column sums ----
@@ -270,8 +297,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const float xk1 =
             r < nvalid ? __fsub_rn((c & 1) ? bf16_hi(rk[i][2 + (c >> 1)]) : bf16_lo(rk[i][2 + (c >> 1)]), muc[c + 4])
                        : 0.f;
-        qa |= i8code(xq0, mq) << (8 * c);
-        qb |= i8code(xq1, mq) << (8 * c);
+        qa |= i8code(xq0, mqr[i]) << (8 * c);
+        qb |= i8code(xq1, mqr[i]) << (8 * c);
         ka |= i8code(xk0, mk) << (8 * c);
         kb |= i8code(xk1, mk) << (8 * c);
       }
@@ -339,7 +366,7 @@ cudaError_t launch_stats_final(const double* psum, const float* pmax, const Geom
 
 cudaError_t launch_quant(const void* q, const void* k, const void* v, const float* mu, const float* mv, const Geom& g,
                          uint8_t* q8t, uint8_t* k8t, uint8_t* v8t, float* sq, float* sk, float* qsum, float* ksum,
-                         int* wd, cudaStream_t st) {
+                         int* wd, cudaStream_t st, int qmax, int q_tok) {
   const int smem = (int)sizeof(QuantSmem);
   cudaError_t e = cudaFuncSetAttribute(quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -348,7 +375,8 @@ cudaError_t launch_quant(const void* q, const void* k, const void* v, const floa
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int ntiles = g.BH * g.nq;
   quant_kernel<<<min(ntiles, sms), kQThreads, smem, st>>>((const uint8_t*)q, (const uint8_t*)k, (const uint8_t*)v, mu,
-                                                          mv, g.N, g.nq, ntiles, q8t, k8t, v8t, sq, sk, qsum, ksum, wd);
+                                                          mv, g.N, g.nq, ntiles, q8t, k8t, v8t, sq, sk, qsum, ksum, wd,
+                                                          qmax, q_tok);
   return cudaGetLastError();
 }
 

@@ -27,7 +27,7 @@ cudaError_t launch_stats_final(const double* psum, const float* pmax, const Geom
 // K2: smoothing + INT8 Q/K tiles + FP8 V^T tiles + per-64-row pooled sums.
 cudaError_t launch_quant(const void* q, const void* k, const void* v, const float* mu, const float* mv,
                          const Geom& g, uint8_t* q8t, uint8_t* k8t, uint8_t* v8t, float* sq, float* sk,
-                         float* qsum, float* ksum, int* wd, cudaStream_t st);
+                         float* qsum, float* ksum, int* wd, cudaStream_t st, int qmax = 127, int q_tok = 0);
 // Untile the quantised tiles back to row-major codes (parity entry only).
 cudaError_t launch_untile(const uint8_t* q8t, const uint8_t* k8t, const uint8_t* v8t, const Geom& g, int8_t* q8,
                           int8_t* k8, uint8_t* v8, cudaStream_t st);
@@ -60,6 +60,7 @@ struct FlashArgs {
   const int32_t* idx;  // [BH][nb][kc]; NULL = dense (every block, ascending)
   void* out;           // bf16 [BH][N][128]
   int add_out;          // 1: out already holds the linear branch y (bf16); add O_s to it
+  int q_tok;            // 1: sq holds one Q scale per token ([BH][nq*64]) instead of per 64-token tile
   // Watchdog test of the block-64 kernel (all 0 in a normal call): a grid of
   // dbg_grid CTAs instead of the persistent grid, dbg_spin probes per
   // bounded wait instead of the default, and, for dbg_stall > 0, slot 0's K

@@ -81,6 +81,10 @@ def test_rejects_bad_arguments_without_launch(L):
         assert L.sagesla_attn(a, a, a, None, a, 1, 1, n_max + 1, 128, blk, F(0.1), None) == -1
         assert L.sagesla_attn(a, a, a, None, a, 1, 1, n_max, 128, blk, F(0.1), None) != -1
     assert L.sagesla_watchdog_selftest((1 << 20) + 1, None) == -1
+    # quantisation options out of range
+    assert L.sagesla_attn_opts(a, a, a, None, a, 1, 1, 64, 128, 64, F(0.1), 5, 0, None) == -1
+    assert L.sagesla_attn_opts(a, a, a, None, a, 1, 1, 64, 128, 64, F(0.1), 8, 2, None) == -1
+    assert L.sagesla_attn_opts(None, a, a, None, a, 1, 1, 64, 128, 64, F(0.1), 4, 1, None) == -1
     # W8A8: shapes that are not multiples of the 128 x 128 block, null and misaligned pointers
     sp = P(0x20000)
     assert L.sagesla_w8a8_quant(a, 128, 100, a, sp, None) == -1

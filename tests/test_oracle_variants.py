@@ -1,7 +1,7 @@
 """Pins of the oracle's SageAttention2++ variants (CPU only).
 
-量子位 news, 技术解密 1: SageAttention2++ quantises to INT8 "or even INT4" and
-uses "thread-level quantisation calibration".  The oracle takes them as two
+量子位 news, 技术解密 1: SageAttention2++ quantises to 8 and, further, 4 bits and
+calibrates the quantisation per thread.  The oracle takes these as two
 options of the quantisation step: one Q scale per token (the row a softmax
 thread owns) instead of per 64-token block, and Q/K codes in +-7 instead of
 +-127.  The pins:
