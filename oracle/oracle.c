@@ -29,7 +29,9 @@
  * two-key worked example); e4m3 encoder exhaustive vs torch's cast; int8
  * quantiser closed forms; mask vs brute-force sort and constructed ties;
  * linear branch vs per-token sum and closed forms; W8A8 linear vs integer
- * matmul at unit scales and vs the matmul of the dequantised operands.
+ * matmul at unit scales and vs the matmul of the dequantised operands;
+ * QK RMSNorm vs its fp64 definition, power-of-two closed forms, and the
+ * coupling of the heads of a token.
  */
 #include <math.h>
 #include <stdint.h>
@@ -742,4 +744,39 @@ void orc_w8a8_gemm(const int8_t* qx, const float* sx, const int8_t* qw, const fl
       }
       y[(int64_t)m * N + n] = acc;
     }
+}
+
+/* ------------------------------------------------------------------------ */
+/* QK RMSNorm before the path ("thu-ml/TurboDiffusion" radar page §二 step 5:  */
+/* the DiT's norms run in its own kernels; 量子位 news, 技术解密 4: custom      */
+/* RMSNorm kernels).  Reading: per token, over the model dimension (all H   */
+/* heads x d channels), y = x / sqrt(mean(x^2) + eps) * gamma, gamma of     */
+/* length H*d; the mean in fp64, inv = fl32(1/sqrt(mean + eps)), then       */
+/* y = bf16(fl32(fl32(x * inv) * gamma)) -- the normalised activations are  */
+/* bf16, the DiT's activation type.  x, y: bf16 [B][H][N][d].               */
+/* ------------------------------------------------------------------------ */
+void orc_rmsnorm_bf16(const uint16_t* x, const uint16_t* gamma, int B, int H, int N, int d, double eps,
+                      uint16_t* y) {
+#pragma omp parallel for schedule(static)
+  for (int64_t bn = 0; bn < (int64_t)B * N; ++bn) {
+    const int b = (int)(bn / N), n = (int)(bn % N);
+    double ss = 0.0;
+    for (int h = 0; h < H; ++h)
+      for (int c = 0; c < d; ++c) {
+        const double v = bf16_f32(x[(((int64_t)b * H + h) * N + n) * d + c]);
+        ss += v * v;
+      }
+    const float inv = (float)(1.0 / sqrt(ss / ((double)H * d) + eps));
+    for (int h = 0; h < H; ++h)
+      for (int c = 0; c < d; ++c) {
+        const int64_t o = (((int64_t)b * H + h) * N + n) * d + c;
+        const float t = bf16_f32(x[o]) * inv;
+        const float r = t * bf16_f32(gamma[(int64_t)h * d + c]);
+        /* round to bf16, nearest even (r is finite) */
+        uint32_t u;
+        memcpy(&u, &r, 4);
+        u += 0x7FFFu + ((u >> 16) & 1u);
+        y[o] = (uint16_t)(u >> 16);
+      }
+  }
 }

@@ -69,6 +69,7 @@ def lib():
         L.orc_linear_direct.argtypes = [P, P, P, i, i, i, i, P, P]
         L.orc_w8a8_quant.argtypes = [P, i, i, P, P]
         L.orc_w8a8_gemm.argtypes = [P, P, P, P, i, i, i, P]
+        L.orc_rmsnorm_bf16.argtypes = [P, P, i, i, i, i, ctypes.c_double, P]
         _lib = L
     return _lib
 
@@ -253,3 +254,13 @@ def w8a8_linear(x, w) -> dict:
     qx, qw = w8a8_quant(x), w8a8_quant(w)
     return {"qx": qx["q"], "sx": qx["s"], "qw": qw["q"], "sw": qw["s"],
             "y": w8a8_gemm(qx["q"], qx["s"], qw["q"], qw["s"])}
+
+
+def rmsnorm_bf16(x, gamma, eps: float = 1e-6) -> np.ndarray:
+    """QK RMSNorm over each token's H*d channels: bf16 [B][H][N][d] -> bf16 bits (uint16), same shape."""
+    xb, gb = _bits(x), _bits(gamma)
+    B, H, N, d = xb.shape
+    assert gb.size == H * d
+    y = np.empty_like(xb)
+    lib().orc_rmsnorm_bf16(_p(xb), _p(gb), B, H, N, d, float(eps), _p(y))
+    return y
