@@ -123,6 +123,22 @@ int sagesla_attn_opts(const void* q, const void* k, const void* v, const void* p
                       int N, int d, int block, float topk, int qk_bits, int q_per_token, sagesla_stream_t stream);
 
 /*
+ * sagesla_attn_qknorm: sagesla_attn on RMS-normalised q and k, the norm
+ * fused into the kernels that load them (the DiT normalises q and k right
+ * before attention: "thu-ml/TurboDiffusion" radar page §二 step 5, 量子位 news
+ * 技术解密 4).  Reading: per token, over all H heads x d channels,
+ *   x_n = bf16( fl32( fl32(x * inv) * gamma[h*d + c] ) ),
+ *   inv = fl32( 1 / sqrt(sum of x^2 / (H*d) + eps) )  (the sum in fp64),
+ * for q with gamma_q and for k with gamma_k (bf16 [H*d] device, 16-byte
+ * aligned; eps in [0, 1]).  The result equals sagesla_attn on the
+ * normalised tensors, without writing them: one extra read of q and k for
+ * the per-token sums instead of a write and a read of both.
+ */
+int sagesla_attn_qknorm(const void* q, const void* k, const void* v, const void* gamma_q, const void* gamma_k,
+                        float eps, const void* proj_w, void* out, int B, int H, int N, int d, int block, float topk,
+                        sagesla_stream_t stream);
+
+/*
  * sagesla_get_quant: the smoothing + quantisation step alone (for parity).
  *   q8, k8   int8 [B][H][N][d] device: INT8 codes, row-major.
  *   v8       uint8 [B][H][N][d] device: FP8 E4M3 codes, row-major.
@@ -268,11 +284,12 @@ const char* sagesla_strerror(int code);
  * forgets them.  Kernel ids: 0 stats, 1 stats finalise, 2 quantise,
  * 3 pooled top-k, 4 linear per-block phi(K)^T V, 5 linear complement sum,
  * 6 sparse flash, 7 projection-weight tiling, 8 linear output (phi(Q) H,
- * normalisation, projection), 9 W8A8 block quantiser, 10 W8A8 GEMM.
+ * normalisation, projection), 9 W8A8 block quantiser, 10 W8A8 GEMM,
+ * 11 QK RMSNorm per-token sums.
  * ms / launches are arrays of nkernels entries (either may be NULL).
  * Profiling is off by default.
  */
-#define SAGESLA_NUM_KERNELS 11
+#define SAGESLA_NUM_KERNELS 12
 void sagesla_profile(int enable);
 int sagesla_profile_read(double* ms, int* launches, int nkernels);
 

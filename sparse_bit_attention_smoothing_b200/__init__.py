@@ -27,12 +27,12 @@ class SageSLAError(RuntimeError):
         super().__init__(f"{where}: {ERRORS.get(code, 'error')} ({code})")
 
 
-EXPORTS = ["sagesla_attn", "sagesla_attn_opts", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
+EXPORTS = ["sagesla_attn", "sagesla_attn_opts", "sagesla_attn_qknorm", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
            "sagesla_smooth_stats_noalloc", "sagesla_topk_count", "sagesla_sync_status", "sagesla_strerror",
            "sagesla_release", "sagesla_profile", "sagesla_profile_read", "sagesla_watchdog_selftest",
            "sagesla_debug_flash_stall", "sagesla_w8a8_quant", "sagesla_w8a8_gemm", "sagesla_w8a8_linear"]
 KERNELS = ["stats", "stats_final", "quant", "pool_topk", "linear_kv", "linear_sum", "flash", "w_tile",
-           "linear_apply", "w8a8_quant", "w8a8_gemm"]
+           "linear_apply", "w8a8_quant", "w8a8_gemm", "rms_inv"]
 
 
 def lib():
@@ -46,6 +46,7 @@ def lib():
         L.sagesla_attn.argtypes = [P, P, P, P, P, i, i, i, i, i, f, P]
         L.dense_int8_attn.argtypes = [P, P, P, P, i, i, i, i, P]
         L.sagesla_attn_opts.argtypes = [P, P, P, P, P, i, i, i, i, i, f, i, i, P]
+        L.sagesla_attn_qknorm.argtypes = [P, P, P, P, P, f, P, P, i, i, i, i, i, f, P]
         L.sagesla_attn_host.argtypes = [P, P, P, P, P, i, i, i, i, i, f, P]
         L.sagesla_get_quant.argtypes = [P, P, P, i, i, i, i, P, P, P, P, P, P, P, P]
         L.sagesla_get_mask.argtypes = [P, P, i, i, i, i, i, f, P, P, P, P, P]
@@ -115,6 +116,20 @@ def sagesla_attn_opts(q, k, v, proj_w=None, out=None, block: int = 64, topk: flo
     _check(lib().sagesla_attn_opts(_ptr(q), _ptr(k), _ptr(v), _ptr(proj_w), _ptr(out), B, H, N, d, block,
                                    ctypes.c_float(topk), qk_bits, 1 if q_per_token else 0, _stream(stream)),
            "sagesla_attn_opts")
+    return out
+
+
+def sagesla_attn_qknorm(q, k, v, gamma_q, gamma_k, eps: float = 1e-6, proj_w=None, out=None, block: int = 64,
+                        topk: float = 0.1, stream=None):
+    """sagesla_attn on RMS-normalised q and k (per token over H*d channels, weights gamma_q / gamma_k: bf16 [H*d]),
+    the norm applied inside the kernels that load q and k."""
+    import torch
+    B, H, N, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().sagesla_attn_qknorm(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma_q), _ptr(gamma_k), ctypes.c_float(eps),
+                                     _ptr(proj_w), _ptr(out), B, H, N, d, block, ctypes.c_float(topk), _stream(stream)),
+           "sagesla_attn_qknorm")
     return out
 
 

@@ -164,6 +164,7 @@ struct Buffers {
   float *sq, *sk, *qsum, *ksum;
   int32_t* idx;
   float *qbar, *kbar;  // pooled means [BH][nb][128]
+  float *inv_q, *inv_k;  // QK RMSNorm: per-token 1 / rms [B][N]
   // linear branch
   uint8_t* hs;        // mask-GEMM B tiles of h_j (bf16)
   float* z;           // z_j [BH][nb][128]
@@ -175,7 +176,7 @@ struct Buffers {
   size_t total;
 };
 
-Buffers carve(uint8_t* base, const Geom& g, bool linear = false, bool q_tok = false) {
+Buffers carve(uint8_t* base, const Geom& g, bool linear = false, bool q_tok = false, int norm_B = 0) {
   Buffers b;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -199,6 +200,8 @@ Buffers carve(uint8_t* base, const Geom& g, bool linear = false, bool q_tok = fa
   b.idx = reinterpret_cast<int32_t*>(take(BH * g.nb * (size_t)g.kc * sizeof(int32_t)));
   b.qbar = reinterpret_cast<float*>(take(BH * g.nb * kD * sizeof(float)));
   b.kbar = reinterpret_cast<float*>(take(BH * g.nb * kD * sizeof(float)));
+  b.inv_q = norm_B ? reinterpret_cast<float*>(take((size_t)norm_B * g.N * sizeof(float))) : nullptr;
+  b.inv_k = norm_B ? reinterpret_cast<float*>(take((size_t)norm_B * g.N * sizeof(float))) : nullptr;
   if (linear) {
     const size_t nbt = (size_t)(g.nb + 63) / 64;
     b.hs = take(BH * nbt * 64 * 16384 * 2);
@@ -227,11 +230,36 @@ inline int launch_rc(cudaError_t e) { return e == cudaSuccess ? SAGESLA_OK : SAG
   } while (0)
 
 // Stats + quantisation (the front shared by every entry point).
+// QK RMSNorm inputs of the path (gq == nullptr: off).
+struct NormIn {
+  const void* gq = nullptr;
+  const void* gk = nullptr;
+  double eps = 0.0;
+  int B = 0, H = 0;
+};
+
+QKNorm qk_norm(const float* inv, const void* gamma, const NormIn* n, const Geom& g) {
+  QKNorm r;
+  if (n && n->gq) {
+    r.inv = inv;
+    r.gamma = static_cast<const uint4*>(gamma);
+    r.H = n->H;
+    r.N = g.N;
+  }
+  return r;
+}
+
 int run_front(const void* q, const void* k, const void* v, const Geom& g, const Buffers& b, int dev,
-              cudaStream_t st, int qmax = 127, int q_tok = 0) {
+              cudaStream_t st, int qmax = 127, int q_tok = 0, const NormIn* nrm = nullptr) {
+  if (nrm && nrm->gq) {
+    ProfScope ps(11, st);
+    SAGESLA_TRY(launch_rc(launch_rms_inv(q, k, nrm->B, nrm->H, g.N, nrm->eps, b.inv_q, b.inv_k, st)));
+  }
+  const QKNorm nq = qk_norm(b.inv_q, nrm ? nrm->gq : nullptr, nrm, g);
+  const QKNorm nk = qk_norm(b.inv_k, nrm ? nrm->gk : nullptr, nrm, g);
   {
     ProfScope ps(0, st);
-    SAGESLA_TRY(launch_rc(launch_stats_partial(k, v, g, b.psum, b.pmax, st)));
+    SAGESLA_TRY(launch_rc(launch_stats_partial(k, v, g, b.psum, b.pmax, st, nk)));
   }
   {
     ProfScope ps(1, st);
@@ -241,14 +269,14 @@ int run_front(const void* q, const void* k, const void* v, const Geom& g, const 
     ProfScope ps(2, st);
     SAGESLA_TRY(launch_rc(
         launch_quant(q, k, v, b.mu, b.mv, g, b.q8t, b.k8t, b.v8t, b.sq, b.sk, b.qsum, b.ksum, watchdog(dev), st,
-                     qmax, q_tok)));
+                     qmax, q_tok, nq, nk)));
   }
   return SAGESLA_OK;
 }
 
 int run_attn(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B, int H, int N, int d,
              int block, float topk, cudaStream_t st, int dbg_grid = 0, int dbg_stall = 0, long dbg_spin = 0,
-             int qmax = 127, int q_tok = 0) {
+             int qmax = 127, int q_tok = 0, const NormIn* nrm = nullptr) {
   SAGESLA_TRY(validate(q, k, v, out, B, H, N, d, block, topk));
   if (proj_w && !aligned16(proj_w)) return SAGESLA_ERR_MISALIGNED;
   int dev = 0;
@@ -257,11 +285,14 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
   const bool dense = g.kc == g.nb;
   // An empty complement (every key block selected) makes the linear branch 0.
   const bool linear = proj_w != nullptr && !dense;
-  const Buffers sizes = carve(nullptr, g, linear, q_tok != 0);
+  const int norm_B = (nrm && nrm->gq) ? B : 0;
+  const Buffers sizes = carve(nullptr, g, linear, q_tok != 0, norm_B);
   uint8_t* base = nullptr;
   SAGESLA_TRY(get_workspace(dev, st, sizes.total, &base));
-  const Buffers b = carve(base, g, linear, q_tok != 0);
-  SAGESLA_TRY(run_front(q, k, v, g, b, dev, st, qmax, q_tok));
+  const Buffers b = carve(base, g, linear, q_tok != 0, norm_B);
+  SAGESLA_TRY(run_front(q, k, v, g, b, dev, st, qmax, q_tok, nrm));
+  const QKNorm nq = qk_norm(b.inv_q, nrm ? nrm->gq : nullptr, nrm, g);
+  const QKNorm nk = qk_norm(b.inv_k, nrm ? nrm->gk : nullptr, nrm, g);
   int* wd = watchdog(dev);
   if (linear) {
     {
@@ -269,7 +300,7 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
       SAGESLA_TRY(launch_rc(launch_w_tile(proj_w, b.wimg, st)));
     }
     ProfScope ps(4, st);
-    SAGESLA_TRY(launch_rc(launch_linear_kv(k, v, g, b.hs, b.z, wd, st)));
+    SAGESLA_TRY(launch_rc(launch_linear_kv(k, v, g, b.hs, b.z, wd, st, nk)));
   }
   if (!dense) {
     ProfScope ps(3, st);
@@ -282,7 +313,7 @@ int run_attn(const void* q, const void* k, const void* v, const void* proj_w, vo
       SAGESLA_TRY(launch_rc(launch_linear_sum(b.hs, b.selbits, g, b.himg, wd, st)));
     }
     ProfScope ps(8, st);
-    SAGESLA_TRY(launch_rc(launch_linear_apply(q, b.himg, b.zl, b.wimg, g, out, wd, st)));
+    SAGESLA_TRY(launch_rc(launch_linear_apply(q, b.himg, b.zl, b.wimg, g, out, wd, st, nq)));
   }
   FlashArgs fa;
   std::memset(&fa, 0, sizeof(fa));
@@ -339,6 +370,21 @@ int sagesla_attn_opts(const void* q, const void* k, const void* v, const void* p
   if ((qk_bits != 8 && qk_bits != 4) || (q_per_token != 0 && q_per_token != 1)) return SAGESLA_ERR_INVALID;
   return run_attn(q, k, v, proj_w, out, B, H, N, d, block, topk, reinterpret_cast<cudaStream_t>(stream), 0, 0, 0,
                   qk_bits == 8 ? 127 : 7, q_per_token);
+}
+
+int sagesla_attn_qknorm(const void* q, const void* k, const void* v, const void* gamma_q, const void* gamma_k,
+                        float eps, const void* proj_w, void* out, int B, int H, int N, int d, int block, float topk,
+                        sagesla_stream_t stream) {
+  if (!gamma_q || !gamma_k || !(eps >= 0.f) || eps > 1.f) return SAGESLA_ERR_INVALID;
+  if (!aligned16(gamma_q) || !aligned16(gamma_k)) return SAGESLA_ERR_MISALIGNED;
+  NormIn n;
+  n.gq = gamma_q;
+  n.gk = gamma_k;
+  n.eps = (double)eps;
+  n.B = B;
+  n.H = H;
+  return run_attn(q, k, v, proj_w, out, B, H, N, d, block, topk, reinterpret_cast<cudaStream_t>(stream), 0, 0, 0, 127,
+                  0, &n);
 }
 
 int dense_int8_attn(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,

@@ -95,6 +95,22 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   return false;
 }
 
+// ------------------------------ QK RMSNorm --------------------------------
+// The DiT's RMSNorm of q and k, applied where the path loads them: per token,
+// x / sqrt(mean over its H*d channels of x^2 + eps) * gamma, rounded to bf16
+// (the per-token factor inv comes from rms_inv_kernel; see QKNorm).
+__device__ __forceinline__ uint32_t rms_bf16x2(uint32_t w, float inv, uint32_t gw) {
+  const float a = __fmul_rn(__fmul_rn(__uint_as_float(w << 16), inv), __uint_as_float(gw << 16));
+  const float b = __fmul_rn(__fmul_rn(__uint_as_float(w & 0xFFFF0000u), inv), __uint_as_float(gw & 0xFFFF0000u));
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// Eight bf16 channels of one row: x * inv * gamma.
+__device__ __forceinline__ uint4 rms_row8(uint4 x, float inv, uint4 g) {
+  return make_uint4(rms_bf16x2(x.x, inv, g.x), rms_bf16x2(x.y, inv, g.y), rms_bf16x2(x.z, inv, g.z),
+                    rms_bf16x2(x.w, inv, g.w));
+}
+
 // --------------------------- bulk async copy -----------------------------
 // Global -> shared, completion counted in bytes on `bar`.  Both addresses
 // 16-byte aligned, size a multiple of 16.

@@ -64,7 +64,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 template <int BLK>
 __global__ void __launch_bounds__(256, 4) linear_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                                            int N, int nb, int nbt, uint8_t* __restrict__ hs,
-                                                           float* __restrict__ z, int* wd) {
+                                                           float* __restrict__ z, int* wd, const QKNorm nk) {
   constexpr int kOpBytes = BLK * 128 * 2;  // one operand tile
   constexpr uint32_t kSBO = (BLK / 8) * 128;
   extern __shared__ uint8_t smem_raw[];
@@ -95,6 +95,14 @@ __global__ void __launch_bounds__(256, 4) linear_kv_kernel(const uint4* __restri
       const bool valid = j < nb && n < N;
       kk[r] = valid ? __ldg(k + base + (size_t)n * 16 + cg) : make_uint4(0, 0, 0, 0);
       vv[r] = valid ? __ldg(v + base + (size_t)n * 16 + cg) : make_uint4(0, 0, 0, 0);
+    }
+    if (nk.inv) {  // QK RMSNorm of the key rows
+      const uint4 gk = __ldg(nk.gamma + (bh % nk.H) * 16 + cg);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int n = j * BLK + 64 * rd + r0 + 16 * r;
+        if (j < nb && n < N) kk[r] = rms_row8(kk[r], __ldg(nk.inv + (size_t)(bh / nk.H) * N + n), gk);
+      }
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
@@ -327,7 +335,8 @@ __global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __res
                                                            const uint8_t* __restrict__ himg,
                                                            const float* __restrict__ zl,
                                                            const uint8_t* __restrict__ wimg, int N, int nb,
-                                                           __nv_bfloat16* __restrict__ out, int* wd) {
+                                                           __nv_bfloat16* __restrict__ out, int* wd,
+                                                           const QKNorm nq) {
   constexpr int kImg = 32768;
   constexpr int nH = MODE == 0 ? 2 : 1;
   extern __shared__ uint8_t smem_raw[];
@@ -386,6 +395,12 @@ __global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __res
   uint4 qq[16];
 #pragma unroll
   for (int ch = 0; ch < 16; ++ch) qq[ch] = store ? __ldg(qrow + ch) : make_uint4(0, 0, 0, 0);
+  if (nq.inv && store) {  // QK RMSNorm of the query row
+    const float inv = __ldg(nq.inv + (size_t)(bh / nq.H) * N + n);
+    const uint4* gq = nq.gamma + (bh % nq.H) * 16;
+#pragma unroll
+    for (int ch = 0; ch < 16; ++ch) qq[ch] = rms_row8(qq[ch], inv, __ldg(gq + ch));
+  }
 #pragma unroll
   for (int ch = 0; ch < 16; ++ch) {
     const uint32_t w4[4] = {qq[ch].x, qq[ch].y, qq[ch].z, qq[ch].w};
@@ -490,19 +505,19 @@ __global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __res
 int linear_apply_smem(int block) { return (block == 64 ? 3 : 2) * 32768 + 1024; }
 
 cudaError_t launch_linear_apply(const void* q, const uint16_t* himg, const float* zl, const uint16_t* wimg,
-                                const Geom& g, void* out, int* wd, cudaStream_t st) {
+                                const Geom& g, void* out, int* wd, cudaStream_t st, QKNorm nq) {
   const int smem = linear_apply_smem(g.block);
   cudaError_t e;
   if (g.block == 64) {
     e = cudaFuncSetAttribute(linear_apply_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     linear_apply_kernel<0><<<dim3((g.nb + 1) / 2, g.BH), 128, smem, st>>>(
-        (const uint16_t*)q, (const uint8_t*)himg, zl, (const uint8_t*)wimg, g.N, g.nb, (__nv_bfloat16*)out, wd);
+        (const uint16_t*)q, (const uint8_t*)himg, zl, (const uint8_t*)wimg, g.N, g.nb, (__nv_bfloat16*)out, wd, nq);
   } else {
     e = cudaFuncSetAttribute(linear_apply_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     linear_apply_kernel<1><<<dim3(g.nb, g.BH), 128, smem, st>>>(
-        (const uint16_t*)q, (const uint8_t*)himg, zl, (const uint8_t*)wimg, g.N, g.nb, (__nv_bfloat16*)out, wd);
+        (const uint16_t*)q, (const uint8_t*)himg, zl, (const uint8_t*)wimg, g.N, g.nb, (__nv_bfloat16*)out, wd, nq);
   }
   return cudaGetLastError();
 }
@@ -518,7 +533,7 @@ int linear_kv_smem(int block) { return 2 * block * 128 * 2 + 1024; }
 int linear_sum_smem() { return kLStages * (kHsTile + kSumTiles * kATile) + (int)sizeof(LBars) + 1024; }
 
 cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_t* hs, float* z, int* wd,
-                             cudaStream_t st) {
+                             cudaStream_t st, QKNorm nk) {
   const int nbt = (g.nb + 63) / 64;
   const int smem = linear_kv_smem(g.block);
   cudaError_t e;
@@ -526,12 +541,12 @@ cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_
     e = cudaFuncSetAttribute(linear_kv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     linear_kv_kernel<64><<<dim3(nbt * 64, g.BH), 256, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt, hs,
-                                                                  z, wd);
+                                                                  z, wd, nk);
   } else {
     e = cudaFuncSetAttribute(linear_kv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     linear_kv_kernel<128><<<dim3(nbt * 64, g.BH), 256, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt,
-                                                                   hs, z, wd);
+                                                                   hs, z, wd, nk);
   }
   return cudaGetLastError();
 }

@@ -21,7 +21,7 @@ namespace sagesla {
 // rows t/16, t/16+8, ... of its split.
 __global__ void __launch_bounds__(128) stats_partial_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                                             int N, int rows_per_split, double* __restrict__ psum,
-                                                            float* __restrict__ pmax) {
+                                                            float* __restrict__ pmax, const QKNorm nk) {
   const int bh = blockIdx.y, sp = blockIdx.x, t = threadIdx.x;
   const int cg = t & 15, r0 = t >> 4;
   const int n_begin = sp * rows_per_split;
@@ -34,10 +34,13 @@ __global__ void __launch_bounds__(128) stats_partial_kernel(const uint4* __restr
     m[i] = 0.f;
   }
   const size_t base = (size_t)bh * N * 16;  // in uint4 (8 bf16) units
+  const uint4 gk = nk.inv ? __ldg(nk.gamma + (bh % nk.H) * 16 + cg) : make_uint4(0, 0, 0, 0);
+  const float* invk = nk.inv ? nk.inv + (size_t)(bh / max(1, nk.H)) * N : nullptr;
 #pragma unroll 4
   for (int n = n_begin + r0; n < n_end; n += 8) {  // unrolled: four row pairs of loads in flight
     uint4 kk = __ldg(k + base + (size_t)n * 16 + cg);
     uint4 vv = __ldg(v + base + (size_t)n * 16 + cg);
+    if (invk) kk = rms_row8(kk, __ldg(invk + n), gk);
     uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};
     uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
@@ -126,7 +129,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
                  const float* __restrict__ mu, const float* __restrict__ mv, int N, int nq, int ntiles,
                  uint8_t* __restrict__ q8t, uint8_t* __restrict__ k8t, uint8_t* __restrict__ v8t,
                  float* __restrict__ sq, float* __restrict__ sk, float* __restrict__ qsum, float* __restrict__ ksum,
-                 int* wd, int qmax, int q_tok) {
+                 int* wd, int qmax, int q_tok, const QKNorm nrq, const QKNorm nrk) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   QuantSmem& S = *reinterpret_cast<QuantSmem*>(smem_raw);
   volatile int* abort = &S.abort;
@@ -174,6 +177,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const uint8_t* sV = S.stage[st][2];
 
     // ---- Q, K rows: absmax and column sums (rows past N read as 0) ----
+    // QK RMSNorm (option): this thread's eight channels of gamma for the head
+    const uint4 gq = nrq.inv ? __ldg(nrq.gamma + (bh % nrq.H) * 16 + cg) : make_uint4(0, 0, 0, 0);
+    const uint4 gk = nrk.inv ? __ldg(nrk.gamma + (bh % nrk.H) * 16 + cg) : make_uint4(0, 0, 0, 0);
+    const size_t tok0 = (size_t)(bh / max(1, nrq.inv ? nrq.H : nrk.H)) * N + n0;
     const float4 mu0 = *reinterpret_cast<const float4*>(mu + (size_t)bh * kD + cg * 8);
     const float4 mu1 = *reinterpret_cast<const float4*>(mu + (size_t)bh * kD + cg * 8 + 4);
     const float muc[8] = {mu0.x, mu0.y, mu0.z, mu0.w, mu1.x, mu1.y, mu1.z, mu1.w};
@@ -191,6 +198,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if (r < nvalid) {
         qq = *reinterpret_cast<const uint4*>(sQ + r * kRowBytes + cg * 16);
         kk = *reinterpret_cast<const uint4*>(sK + r * kRowBytes + cg * 16);
+        if (nrq.inv) qq = rms_row8(qq, __ldg(nrq.inv + tok0 + r), gq);
+        if (nrk.inv) kk = rms_row8(kk, __ldg(nrk.inv + tok0 + r), gk);
       }
       rq[i][0] = qq.x; rq[i][1] = qq.y; rq[i][2] = qq.z; rq[i][3] = qq.w;
       rk[i][0] = kk.x; rk[i][1] = kk.y; rk[i][2] = kk.z; rk[i][3] = kk.w;
@@ -335,6 +344,49 @@ __global__ void __launch_bounds__(kQThreads, 1)
     for (int jj = j; jj < issued; ++jj) mbar_wait_drain(&S.full[jj % kQStages], (uint32_t)(jj / kQStages) & 1u, wd);
 }
 
+// Per-token 1 / rms of q and k over all H heads x d channels (QK RMSNorm):
+// grid (ceil(N / 8), B), 256 threads, one warp per token; lane l reads
+// channels 4l .. 4l+3 of every head's row.  The squares of bf16 values are
+// exact in fp64 and their sum is rounded far below the fp32 rounding of the
+// result, so the order of the sum does not change inv = fl32(1 / sqrt(sum /
+// (H d) + eps)), computed in fp64.
+__global__ void __launch_bounds__(256) rms_inv_kernel(const uint2* __restrict__ q, const uint2* __restrict__ k, int H,
+                                                      int N, double eps, float* __restrict__ inv_q,
+                                                      float* __restrict__ inv_k) {
+  const int b = blockIdx.y, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (n >= N) return;
+  double sq = 0.0, sk = 0.0;
+  for (int h = 0; h < H; ++h) {
+    const size_t row = (((size_t)b * H + h) * N + n) * 32 + lane;  // uint2 = 4 bf16
+    const uint2 a = __ldg(q + row), c = __ldg(k + row);
+    const uint32_t wa[2] = {a.x, a.y}, wc[2] = {c.x, c.y};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const double a0 = bf16_lo(wa[e]), a1 = bf16_hi(wa[e]), c0 = bf16_lo(wc[e]), c1 = bf16_hi(wc[e]);
+      sq += a0 * a0 + a1 * a1;
+      sk += c0 * c0 + c1 * c1;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    sk += __shfl_xor_sync(0xffffffffu, sk, o);
+  }
+  if (lane == 0) {
+    const double hd = (double)H * kD;
+    inv_q[(size_t)b * N + n] = (float)(1.0 / sqrt(sq / hd + eps));
+    inv_k[(size_t)b * N + n] = (float)(1.0 / sqrt(sk / hd + eps));
+  }
+}
+
+cudaError_t launch_rms_inv(const void* q, const void* k, int B, int H, int N, double eps, float* inv_q, float* inv_k,
+                           cudaStream_t st) {
+  rms_inv_kernel<<<dim3((N + 7) / 8, B), 256, 0, st>>>(static_cast<const uint2*>(q), static_cast<const uint2*>(k), H, N,
+                                                        eps, inv_q, inv_k);
+  return cudaGetLastError();
+}
+
 // Row-major codes from the tiles (parity entry point only).
 __global__ void untile_kernel(const uint8_t* __restrict__ q8t, const uint8_t* __restrict__ k8t,
                               const uint8_t* __restrict__ v8t, int N, int nq, int8_t* __restrict__ q8,
@@ -352,9 +404,10 @@ __global__ void untile_kernel(const uint8_t* __restrict__ q8t, const uint8_t* __
 }
 
 cudaError_t launch_stats_partial(const void* k, const void* v, const Geom& g, double* psum, float* pmax,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, QKNorm nk) {
   const int rows = (g.N + g.split - 1) / g.split;
-  stats_partial_kernel<<<dim3(g.split, g.BH), 128, 0, st>>>((const uint4*)k, (const uint4*)v, g.N, rows, psum, pmax);
+  stats_partial_kernel<<<dim3(g.split, g.BH), 128, 0, st>>>((const uint4*)k, (const uint4*)v, g.N, rows, psum, pmax,
+                                                            nk);
   return cudaGetLastError();
 }
 
@@ -366,7 +419,7 @@ cudaError_t launch_stats_final(const double* psum, const float* pmax, const Geom
 
 cudaError_t launch_quant(const void* q, const void* k, const void* v, const float* mu, const float* mv, const Geom& g,
                          uint8_t* q8t, uint8_t* k8t, uint8_t* v8t, float* sq, float* sk, float* qsum, float* ksum,
-                         int* wd, cudaStream_t st, int qmax, int q_tok) {
+                         int* wd, cudaStream_t st, int qmax, int q_tok, QKNorm nq, QKNorm nk) {
   const int smem = (int)sizeof(QuantSmem);
   cudaError_t e = cudaFuncSetAttribute(quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -376,7 +429,7 @@ cudaError_t launch_quant(const void* q, const void* k, const void* v, const floa
   const int ntiles = g.BH * g.nq;
   quant_kernel<<<min(ntiles, sms), kQThreads, smem, st>>>((const uint8_t*)q, (const uint8_t*)k, (const uint8_t*)v, mu,
                                                           mv, g.N, g.nq, ntiles, q8t, k8t, v8t, sq, sk, qsum, ksum, wd,
-                                                          qmax, q_tok);
+                                                          qmax, q_tok, nq, nk);
   return cudaGetLastError();
 }
 

@@ -18,16 +18,27 @@ struct Geom {
   int split;   // row splits of the statistics pass
 };
 
+// QK RMSNorm applied where a kernel loads q or k (inv == nullptr: off):
+// x * inv[b][n] * gamma[h*d + c], rounded to bf16.
+struct QKNorm {
+  const float* inv = nullptr;  // [B][N] per-token 1 / rms over the H*d channels
+  const uint4* gamma = nullptr;  // bf16 [H*d] as 16-byte units (8 channels each)
+  int H = 1, N = 1;
+};
+// Per-token 1 / rms of q and k (QK RMSNorm), [B][N] each.
+cudaError_t launch_rms_inv(const void* q, const void* k, int B, int H, int N, double eps, float* inv_q, float* inv_k,
+                           cudaStream_t st);
 // K1: per-split fp64 sums of K and fp32 max|V| per channel.
 cudaError_t launch_stats_partial(const void* k, const void* v, const Geom& g, double* psum, float* pmax,
-                                 cudaStream_t st);
+                                 cudaStream_t st, QKNorm nk = QKNorm());
 // K1b: mu = fl32(sum/N); V scale amax/448 and multiplier 448/amax per channel.
 cudaError_t launch_stats_final(const double* psum, const float* pmax, const Geom& g, float* mu, float* sv,
                                float* mv, cudaStream_t st);
 // K2: smoothing + INT8 Q/K tiles + FP8 V^T tiles + per-64-row pooled sums.
 cudaError_t launch_quant(const void* q, const void* k, const void* v, const float* mu, const float* mv,
                          const Geom& g, uint8_t* q8t, uint8_t* k8t, uint8_t* v8t, float* sq, float* sk,
-                         float* qsum, float* ksum, int* wd, cudaStream_t st, int qmax = 127, int q_tok = 0);
+                         float* qsum, float* ksum, int* wd, cudaStream_t st, int qmax = 127, int q_tok = 0,
+                         QKNorm nq = QKNorm(), QKNorm nk = QKNorm());
 // Untile the quantised tiles back to row-major codes (parity entry only).
 cudaError_t launch_untile(const uint8_t* q8t, const uint8_t* k8t, const uint8_t* v8t, const Geom& g, int8_t* q8,
                           int8_t* k8, uint8_t* v8, cudaStream_t st);
@@ -40,13 +51,13 @@ cudaError_t launch_pool_topk(const float* qsum, const float* ksum, const Geom& g
                              cudaStream_t st);
 // K4a: per key block h_j = phi(K_j)^T V_j (bf16 mask-GEMM tiles) and z_j.
 cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_t* hs, float* z, int* wd,
-                             cudaStream_t st);
+                             cudaStream_t st, QKNorm nk = QKNorm());
 // K4b: H_i = sum over unselected j of h_j, as bf16 operand images [nb][128*128].
 cudaError_t launch_linear_sum(const uint8_t* hs, const uint32_t* selbits, const Geom& g, uint16_t* hout, int* wd,
                               cudaStream_t st);
 // K4c: y = (phi(Q_i) H_i / phi(Q_i) Z_i) W^T per row, written (bf16) to out.
 cudaError_t launch_linear_apply(const void* q, const uint16_t* himg, const float* zl, const uint16_t* wimg,
-                                const Geom& g, void* out, int* wd, cudaStream_t st);
+                                const Geom& g, void* out, int* wd, cudaStream_t st, QKNorm nq = QKNorm());
 // proj_w [d][d] -> the bf16 B-operand image read by the flash epilogue.
 cudaError_t launch_w_tile(const void* w, uint16_t* wt, cudaStream_t st);
 // K5: block-sparse INT8/FP8 flash attention over the index lists.

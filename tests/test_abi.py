@@ -81,6 +81,10 @@ def test_rejects_bad_arguments_without_launch(L):
         assert L.sagesla_attn(a, a, a, None, a, 1, 1, n_max + 1, 128, blk, F(0.1), None) == -1
         assert L.sagesla_attn(a, a, a, None, a, 1, 1, n_max, 128, blk, F(0.1), None) != -1
     assert L.sagesla_watchdog_selftest((1 << 20) + 1, None) == -1
+    # QK RMSNorm: missing or misaligned weights, eps out of range
+    assert L.sagesla_attn_qknorm(a, a, a, None, a, F(1e-6), None, a, 1, 1, 64, 128, 64, F(0.1), None) == -1
+    assert L.sagesla_attn_qknorm(a, a, a, a, a, F(-1.0), None, a, 1, 1, 64, 128, 64, F(0.1), None) == -1
+    assert L.sagesla_attn_qknorm(a, a, a, P(0x10008), a, F(1e-6), None, a, 1, 1, 64, 128, 64, F(0.1), None) == -2
     # quantisation options out of range
     assert L.sagesla_attn_opts(a, a, a, None, a, 1, 1, 64, 128, 64, F(0.1), 5, 0, None) == -1
     assert L.sagesla_attn_opts(a, a, a, None, a, 1, 1, 64, 128, 64, F(0.1), 8, 2, None) == -1
