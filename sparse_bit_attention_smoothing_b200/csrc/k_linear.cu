@@ -53,131 +53,300 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }  // namespace
 
 // ---------------------------------------------------------------- K4a ----
-// grid (nbt*64, BH): CTA x handles key block j = x (zeros past nb, so the
-// mask-GEMM tiles hold no garbage).  256 threads; thread t owns channels
-// 8*(t%16).. and token rows t/16 + 16r of 64-row rounds: all its K and V
-// loads of a round are issued before any is used.  Small CTAs (128 TMEM
-// columns, ~40 KB of shared memory) so that four share an SM and their load
-// phases overlap each other's compute.  Thread 0 issues the MMAs.  Dynamic
-// smem: A (phi(K) rows) and B (V rows) MN-major, BLK x 128 bf16 each; after
-// the MMAs the h image goes from TMEM straight to the mask-GEMM tiles.
+// Persistent, one CTA per SM.  An item is kKvJ consecutive key blocks
+// j0..j0+kKvJ-1 of one head (j < nbt*64; zeros past nb, so the mask-GEMM
+// tiles hold no garbage); items are dealt round-robin.  In the mask-GEMM
+// tiles the 16-byte pieces of consecutive j are adjacent, so the blocks of an
+// item are stored as 16*kKvJ-byte runs.  TMEM holds 4/kKvJ sets of kKvJ
+// accumulators, so the MMAs of the next item can run while the epilogue
+// drains the last one when kKvJ = 2.  A key block is consumed as BLK/64 chunks
+// of 64 tokens:
+//   warp 0      bulk-copies a chunk's K and V rows (16 KB each, contiguous
+//               in [BH][N][128]) into a 3-stage ring;
+//   warps 2-9   (converters) apply the QK norm and phi to K, add phi(K) into
+//               z, and write phi(K) and V as MN-major bf16 MMA operands into
+//               one of two operand buffers;
+//   warp 1      issues h_j^T += V^T phi(K) (M = 128 value channels, N = 128
+//               key channels, K = 64 tokens) into TMEM accumulator j - j0
+//               of the item's set;
+//   warps 10-17 (epilogue) read the item's accumulators 16 columns at a
+//               time, regroup the bf16 pieces through shared memory so that
+//               kKvJ consecutive lanes hold the kKvJ blocks of one piece, and
+//               store them.
+// Converter slot (r0, cg) owns channels 8*cg.. and rows r0 + 16r of each
+// chunk; z_j adds a slot's rows in token order, then the 16 row slots in
+// slot order.  Every wait is bounded.
+namespace {
+constexpr int kKvJ = 4;                           // key blocks per item (2 or 4)
+constexpr int kKvAcc = 4 / kKvJ;                  // item accumulator sets in TMEM (512 columns)
+constexpr int kKvP = 2 * kKvJ;                    // regrouped pieces per lane per round
+constexpr int kKvFs = kKvP == 8 ? 0 : 1;          // lane shift of the regrouping swizzle
+constexpr int kKvStages = 3;                      // raw chunk ring
+constexpr int kKvHalf = 64 * kD * 2;              // 16 KB: 64 bf16 rows
+constexpr int kKvRaw = 2 * kKvHalf;               // K rows, then V rows
+constexpr int kKvOps = 2;                         // operand buffers
+constexpr int kKvConv = 8, kKvEpi = 8;            // warps
+constexpr int kKvThreads = 32 * (2 + kKvConv + kKvEpi);
+constexpr uint32_t kKvSBO = 8 * 128;              // MN-major operand of 64 tokens
+constexpr int kKvOffOp = kKvStages * kKvRaw;      // phi(K) (B), then V (A)
+constexpr int kKvOffZ = kKvOffOp + kKvOps * kKvRaw;
+constexpr int kKvStage = 32 * kKvP * 16;          // regrouping space per epilogue warp
+constexpr int kKvOffSt = kKvOffZ + 2 * 16 * kD * 4;
+constexpr int kKvOffBars = kKvOffSt + kKvEpi * kKvStage;
+struct KvBars {
+  uint64_t raw_full[kKvStages], raw_empty[kKvStages], op_full[kKvOps], op_empty[kKvOps];
+  uint64_t acc_full[kKvAcc], acc_empty[kKvAcc], z_ready[2], fin;
+  uint32_t tmem;
+  int abort;
+};
+constexpr int kKvSmem = kKvOffBars + (int)sizeof(KvBars) + 1024;
+}  // namespace
+
 template <int BLK>
-__global__ void __launch_bounds__(256, 4) linear_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
-                                                           int N, int nb, int nbt, uint8_t* __restrict__ hs,
-                                                           float* __restrict__ z, int* wd, const QKNorm nk) {
-  constexpr int kOpBytes = BLK * 128 * 2;  // one operand tile
-  constexpr uint32_t kSBO = (BLK / 8) * 128;
+__global__ void __launch_bounds__(kKvThreads, 1) linear_kv_kernel(const uint4* __restrict__ k,
+                                                                 const uint4* __restrict__ v, int N, int nb, int nbt,
+                                                                 int nitems, uint8_t* __restrict__ hs,
+                                                                 float* __restrict__ z, int* wd, const QKNorm nk) {
+  constexpr int kChunks = BLK / 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t bar;
-  __shared__ uint32_t tmem_s;
-  __shared__ int abort_s;
-  __shared__ float zred[16][kD];
-  const int bh = blockIdx.y, t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int j = blockIdx.x;
-  const size_t base = (size_t)bh * N * 16;
-  if (t == 0) {
-    mbar_init(&bar, 1);
-    abort_s = 0;
+  KvBars* bars = reinterpret_cast<KvBars*>(smem + kKvOffBars);
+  float* zred = reinterpret_cast<float*>(smem + kKvOffZ);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nit = nbt * (64 / kKvJ);  // items per head
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kKvStages; ++s) {
+      mbar_init(&bars->raw_full[s], 1);
+      mbar_init(&bars->raw_empty[s], kKvConv);
+    }
+    for (int b = 0; b < kKvOps; ++b) {
+      mbar_init(&bars->op_full[b], kKvConv);
+      mbar_init(&bars->op_empty[b], 1);
+    }
+    for (int a = 0; a < kKvAcc; ++a) {
+      mbar_init(&bars->acc_full[a], 1);
+      mbar_init(&bars->acc_empty[a], kKvEpi);
+    }
+    mbar_init(&bars->z_ready[0], kKvConv);
+    mbar_init(&bars->z_ready[1], kKvConv);
+    mbar_init(&bars->fin, 1);
+    bars->abort = 0;
     mbar_fence_init();
   }
-  if (warp == 0) tmem_alloc(&tmem_s, 128);
-  const int cg = t & 15, r0 = t >> 4;
-  float zacc[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) zacc[c] = 0.f;
-#pragma unroll
-  for (int rd = 0; rd < BLK / 64; ++rd) {
-    uint4 kk[4], vv[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int row = 64 * rd + r0 + 16 * r, n = j * BLK + row;
-      const bool valid = j < nb && n < N;
-      kk[r] = valid ? __ldg(k + base + (size_t)n * 16 + cg) : make_uint4(0, 0, 0, 0);
-      vv[r] = valid ? __ldg(v + base + (size_t)n * 16 + cg) : make_uint4(0, 0, 0, 0);
-    }
-    if (nk.inv) {  // QK RMSNorm of the key rows
-      const uint4 gk = __ldg(nk.gamma + (bh % nk.H) * 16 + cg);
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int n = j * BLK + 64 * rd + r0 + 16 * r;
-        if (j < nb && n < N) kk[r] = rms_row8(kk[r], __ldg(nk.inv + (size_t)(bh / nk.H) * N + n), gk);
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int row = 64 * rd + r0 + 16 * r, n = j * BLK + row;
-      const bool valid = j < nb && n < N;
-      const uint32_t kw[4] = {kk[r].x, kk[r].y, kk[r].z, kk[r].w};
-      uint32_t pw[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float f0 = valid ? phi(bf16_lo(kw[e])) : 0.f;
-        const float f1 = valid ? phi(bf16_hi(kw[e])) : 0.f;
-        zacc[2 * e] += f0;
-        zacc[2 * e + 1] += f1;
-        pw[e] = pack_bf16(f0, f1);
-      }
-      // MN-major core matrix: (m/8)*SBO + (tok/8)*128 + (tok%8)*16 + (m%8)*2
-      const uint32_t off = cg * kSBO + (row >> 3) * 128 + (row & 7) * 16;
-      *reinterpret_cast<uint4*>(smem + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-      *reinterpret_cast<uint4*>(smem + kOpBytes + off) = vv[r];
-    }
-  }
-  fence_proxy_async_smem();
+  if (warp == 1) tmem_alloc(&bars->tmem, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tmem_s;
-  // h_j^T = V_j^T phi(K_j): A = the V rows (M = value channel cv), B = the
-  // phi(K) rows (N = key channel ck), so TMEM lane cv, column ck holds
-  // h_j[ck][cv] and each thread later owns 8 consecutive ck of one cv: one
-  // 16-byte chunk of the image.
-  if (t == 0) {
-    const uint32_t id = idesc_bf16(128, 128, 1) | (1u << 15);  // A and B MN-major
+  const uint32_t tmem = bars->tmem;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      int u = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < nitems; item += gridDim.x) {
+        const int bh = item / nit, j0 = (item - bh * nit) * kKvJ;
+        for (int jj = 0; ok && jj < kKvJ; ++jj) {
+          const int j = j0 + jj;
+          for (int c = 0; c < kChunks; ++c, ++u) {
+            const int s = u % kKvStages;
+            if (u >= kKvStages && !(ok = mbar_wait(&bars->raw_empty[s], ((u / kKvStages) - 1) & 1, abort, wd)))
+              break;
+            const int n0 = j * BLK + 64 * c;
+            const int rows = j < nb ? max(0, min(64, N - n0)) : 0;
+            const uint32_t bytes = (uint32_t)rows * (kD * 2);
+            mbar_expect_tx(&bars->raw_full[s], 2 * bytes);
+            if (rows) {
+              const size_t off = ((size_t)bh * N + n0) * 16;
+              bulk_g2s(smem + s * kKvRaw, k + off, bytes, &bars->raw_full[s]);
+              bulk_g2s(smem + s * kKvRaw + kKvHalf, v + off, bytes, &bars->raw_full[s]);
+            }
+          }
+        }
+      }
+      // Drain: only the uses issued after the last proven-consumed one can
+      // still have copies in flight.
+      for (int g = max(0, u - kKvStages); g < u; ++g)
+        mbar_wait_drain(&bars->raw_full[g % kKvStages], (g / kKvStages) & 1, wd);
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ----------------------------
+    if (lane == 0) {
+      const uint32_t id = idesc_bf16(128, 128, 1) | (1u << 15);  // A and B MN-major
+      int u = 0, it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < nitems; item += gridDim.x, ++it) {
+        const int a = it % kKvAcc;
+        if (it >= kKvAcc && !(ok = mbar_wait(&bars->acc_empty[a], ((it / kKvAcc) - 1) & 1, abort, wd))) break;
+        for (int jj = 0; ok && jj < kKvJ; ++jj) {
+          for (int c = 0; c < kChunks; ++c, ++u) {
+            const int b = u % kKvOps;
+            if (!(ok = mbar_wait(&bars->op_full[b], (u / kKvOps) & 1, abort, wd))) break;
+            tc_fence_after();
+            // h_j^T = V_j^T phi(K_j): A = the V rows (M = value channel cv), B
+            // = the phi(K) rows (N = key channel ck): TMEM lane cv, column ck.
+            const uint8_t* op = smem + kKvOffOp + b * kKvRaw;
 #pragma unroll
-    for (int ks = 0; ks < BLK / 16; ++ks)
-      mma_bf16(tmem, smem_desc(smem + kOpBytes + ks * 256, 128, kSBO), smem_desc(smem + ks * 256, 128, kSBO), id,
-               ks > 0);
-    mma_commit(&bar);
-  }
-  // z_j: the 16 row slots' channel sums, added in slot order.
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16(tmem + (a * kKvJ + jj) * 128, smem_desc(op + kKvHalf + ks * 256, 128, kKvSBO),
+                       smem_desc(op + ks * 256, 128, kKvSBO), id, (c > 0 || ks > 0) ? 1u : 0u);
+            mma_commit(&bars->op_empty[b]);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&bars->acc_full[a]);
+      }
+      mma_commit(&bars->fin);
+    }
+  } else if (warp < 2 + kKvConv) {
+    // ------------------------------ converters ----------------------------
+    // Slot of this thread: row%8 differs across each group of eight lanes
+    // (conflict-free operand stores) and so does cg%8 (conflict-free row
+    // reads); over the 256 threads every (r0, cg) occurs once.
+    const int cw = warp - 2, qd = lane & 7, hi = lane >> 3;
+    const int r0 = qd + 8 * (cw & 1), cg = (qd + hi + 4 * (cw >> 1)) & 15;
+    const int ct = threadIdx.x - 64;
+    int u = 0, zi = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < nitems; item += gridDim.x) {
+      const int bh = item / nit, j0 = (item - bh * nit) * kKvJ;
+      uint4 gk = make_uint4(0, 0, 0, 0);
+      if (nk.inv) gk = __ldg(nk.gamma + (bh % nk.H) * 16 + cg);
+      for (int jj = 0; ok && jj < kKvJ; ++jj, ++zi) {
+        const int j = j0 + jj;
+        float zacc[8];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) zred[r0][cg * 8 + c] = zacc[c];
-  __syncthreads();
-  if (t < kD) {
-    float a = 0.f;
+        for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
+        for (int c = 0; c < kChunks; ++c, ++u) {
+          const int s = u % kKvStages, b = u % kKvOps;
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars->raw_full[s], (u / kKvStages) & 1, abort, wd));
+          if (ok && u >= kKvOps)
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars->op_empty[b], ((u / kKvOps) - 1) & 1, abort, wd));
+          if (!ok) break;
+          const uint8_t* raw = smem + s * kKvRaw;
+          uint8_t* op = smem + kKvOffOp + b * kKvRaw;
+          uint4 kk[4], vv[4];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) a += zred[r][t];
-    if (j < nb) z[((size_t)bh * nb + j) * kD + t] = a;
-  }
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar, 0, &abort_s, wd));
-  tc_fence_after();
-  // Warp w holds cv = 32(w%4) + lane, columns ck in [64(w/4), +64); every
-  // 8 columns are one 16-byte chunk of the bf16 image of H^T (element (cv,
-  // ck) at himg_off), stored straight into its place in the mask-GEMM tile.
-  {
-    const int cv = 32 * (warp & 3) + lane, cb = 64 * (warp >> 2);
-    uint8_t* hsb = hs + (size_t)bh * nbt * 64 * 16384 * 2;
+          for (int r = 0; r < 4; ++r) {
+            const int row = r0 + 16 * r;
+            kk[r] = *reinterpret_cast<const uint4*>(raw + row * (kD * 2) + cg * 16);
+            vv[r] = *reinterpret_cast<const uint4*>(raw + kKvHalf + row * (kD * 2) + cg * 16);
+          }
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int row = r0 + 16 * r, n = j * BLK + 64 * c + row;
+            const bool valid = j < nb && n < N;
+            if (valid && nk.inv) kk[r] = rms_row8(kk[r], __ldg(nk.inv + (size_t)(bh / nk.H) * N + n), gk);
+            const uint32_t kw[4] = {kk[r].x, kk[r].y, kk[r].z, kk[r].w};
+            uint32_t pw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float f0 = valid ? phi(bf16_lo(kw[e])) : 0.f;
+              const float f1 = valid ? phi(bf16_hi(kw[e])) : 0.f;
+              zacc[2 * e] += f0;
+              zacc[2 * e + 1] += f1;
+              pw[e] = pack_bf16(f0, f1);
+            }
+            // MN-major core matrix: (m/8)*SBO + (tok/8)*128 + (tok%8)*16 + (m%8)*2
+            const uint32_t off = cg * kKvSBO + (row >> 3) * 128 + (row & 7) * 16;
+            *reinterpret_cast<uint4*>(op + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+            *reinterpret_cast<uint4*>(op + kKvHalf + off) = valid ? vv[r] : make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bars->op_full[b]);
+            mbar_arrive(&bars->raw_empty[s]);
+          }
+        }
+        if (!ok) break;
+        // z_j: the 16 row slots' channel sums, added in slot order.
+        float* zr = zred + (zi & 1) * 16 * kD;
+        *reinterpret_cast<float4*>(zr + r0 * kD + cg * 8) = make_float4(zacc[0], zacc[1], zacc[2], zacc[3]);
+        *reinterpret_cast<float4*>(zr + r0 * kD + cg * 8 + 4) = make_float4(zacc[4], zacc[5], zacc[6], zacc[7]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->z_ready[zi & 1]);
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->z_ready[zi & 1], (zi >> 1) & 1, abort, wd));
+        if (!ok) break;
+        if (ct < kD) {
+          float a = 0.f;
+#pragma unroll
+          for (int r = 0; r < 16; ++r) a += zr[r * kD + ct];
+          if (j < nb) z[((size_t)bh * nb + j) * kD + ct] = a;
+        }
+      }
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    // Warp w reads TMEM lanes 32(w%4).. (cv = 32(w%4) + lane) and columns ck
+    // in [64 hc, +64) of the item's accumulators, 16 columns per round.  A
+    // round's pieces (cv, 8-column chunk ch, block jj) go to shared memory at
+    // piece index (cv%32, ch, jj), the index within the lane's kKvP pieces
+    // XOR-ed with a function of cv that spreads eight lanes over the banks;
+    // read back 32 consecutive pieces per instruction, kKvJ consecutive lanes
+    // hold the blocks of one (cv, ch), which are contiguous in a mask-GEMM
+    // tile (element (cv, ck) of h_j at himg_off).
+    const int q = warp & 3, hc = (warp - 2 - kKvConv) >> 2;
+    const int cb = 64 * hc;
+    uint8_t* stg = smem + kKvOffSt + (warp - 2 - kKvConv) * kKvStage;
+    int it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < nitems; item += gridDim.x, ++it) {
+      const int bh = item / nit, j0 = (item - bh * nit) * kKvJ;
+      const int a = it % kKvAcc;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->acc_full[a], (it / kKvAcc) & 1, abort, wd));
+      if (!ok) break;
+      tc_fence_after();
+      uint8_t* hsb = hs + (size_t)bh * nbt * 64 * 16384 * 2;
 #pragma unroll 1
-    for (int c0 = cb; c0 < cb + 64; c0 += 16) {
-      uint32_t r[16];
-      SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0, r);
-      tmem_ld_wait();
+      for (int rd = 0; rd < 4; ++rd) {
+        const int c0 = cb + 16 * rd;
+        const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16) + a * kKvJ * 128 + c0;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t w4[4];
+        for (int jp = 0; jp < kKvJ; jp += 2) {  // two accumulators at a time
+          uint32_t r[2][16];
+          SAGESLA_TMEM_LD16(tl + jp * 128, r[0]);
+          SAGESLA_TMEM_LD16(tl + (jp + 1) * 128, r[1]);
+          tmem_ld_wait();
+          if (rd == 3 && jp + 2 == kKvJ) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
+          }
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          w4[e] = ok ? pack_bf16(__uint_as_float(r[8 * h + 2 * e]), __uint_as_float(r[8 * h + 2 * e + 1])) : 0u;
-        const int chunk = (int)(himg_off(cv, c0 + 8 * h) >> 4);
-        *reinterpret_cast<uint4*>(hsb + hs_chunk(nbt, j, chunk)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                w4[e] = pack_bf16(__uint_as_float(r[x][8 * ch + 2 * e]), __uint_as_float(r[x][8 * ch + 2 * e + 1]));
+              const int pidx = lane * kKvP + ((ch * kKvJ + jp + x) ^ ((lane >> kKvFs) & (kKvP - 1)));
+              *reinterpret_cast<uint4*>(stg + pidx * 16) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int x = 0; x < kKvP; ++x) {
+          const int p = 32 * x + lane;  // piece (cv%32 = p/kKvP, ch, jj = p%kKvJ)
+          const int cvl = p / kKvP, li = p % kKvP, ch = li / kKvJ, jj = li % kKvJ;
+          const uint4 w =
+              *reinterpret_cast<const uint4*>(stg + (cvl * kKvP + (li ^ ((cvl >> kKvFs) & (kKvP - 1)))) * 16);
+          const int chunk = (int)(himg_off(32 * q + cvl, c0 + 8 * ch) >> 4);
+          *reinterpret_cast<uint4*>(hsb + hs_chunk(nbt, j0 + jj, chunk)) = w;
+        }
+        __syncwarp();
       }
     }
   }
+  if (warp == 1) {
+    if (lane == 0) mbar_wait_drain(&bars->fin, 0, wd);
+    __syncwarp();
+  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 128);
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- K4b ----
@@ -325,199 +494,281 @@ __global__ void __launch_bounds__(64 + kAThreads, 1) linear_sum_kernel(const uin
 // ---------------------------------------------------------------- K4c ----
 // linear_apply: y_r = (phi(q_r) H_i / phi(q_r) Z_i) W^T for every row r of
 // query block i, written (bf16) into `out`; the flash kernel adds O_s to it.
-// Block 64: two query blocks per CTA whose M=64 accumulators share TMEM at
-// lane offsets 0 / 16 (all 128 threads hold a row); block 128: M = 128.
-// 128 threads; thread 0 issues the copies and MMAs.  TMEM: num (128 cols) and
-// y (128 cols).  Shared: H images (the W image replaces them once num is
-// done, so two CTAs fit on an SM), phi(Q) (reused for O_l).
+// Persistent, one CTA per SM.  An item is 128 query rows: two query blocks at
+// block 64 (M=64 accumulators at TMEM lane offsets 0 / 16), one at block 128
+// (M=128).  The CTA's items alternate between two groups of four row warps
+// (one row per thread), each with its own shared-memory stage and 256 TMEM
+// columns (num, then y), so one group's copies, MMAs and stores overlap the
+// other group's work:
+//   warp 0      bulk-copies an item's q rows (up to 32 KB) and H_i images
+//               into the group's stage; the W image once;
+//   warp 1      issues num = phi(Q) H_i for every item;
+//   warp 10     issues y = O_l W^T for every item;
+//   warps 2-9   (row groups) read their q rows (chunk c ^ (lane%8) at step c,
+//               so eight lanes hit eight banks, then put back in channel
+//               order), write the phi(Q) operand over them, scale num by
+//               1/(phi(q) . Z_i) into the O_l operand, and store y through a
+//               swizzled staging area so that each instruction writes two
+//               whole rows.
+// Per row, the arithmetic and its order are those of one thread per row
+// reading its q row from global memory.  Every wait is bounded.
+namespace {
+constexpr int kApImg = 32768;
+constexpr int kApStage = 3 * kApImg;  // q rows -> phi(Q) -> O_l -> y staging; then two H images
+constexpr int kApOffW = 2 * kApStage;
+constexpr int kApOffBars = kApOffW + kApImg;
+constexpr int kApThreads = 32 * 11;
+struct ApBars {
+  uint64_t full[2], empty[2], qread[2], a_full[2], num_full[2], o_full[2], y_full[2], w_full, fin[2];
+  uint32_t tmem;
+  int abort;
+};
+constexpr int kApSmem = kApOffBars + (int)sizeof(ApBars) + 16;
+}  // namespace
+
 template <int MODE>
-__global__ void __launch_bounds__(128) linear_apply_kernel(const uint16_t* __restrict__ q,
-                                                           const uint8_t* __restrict__ himg,
-                                                           const float* __restrict__ zl,
-                                                           const uint8_t* __restrict__ wimg, int N, int nb,
-                                                           __nv_bfloat16* __restrict__ out, int* wd,
-                                                           const QKNorm nq) {
-  constexpr int kImg = 32768;
-  constexpr int nH = MODE == 0 ? 2 : 1;
+__global__ void __launch_bounds__(kApThreads, 1) linear_apply_kernel(const uint16_t* __restrict__ q,
+                                                                    const uint8_t* __restrict__ himg,
+                                                                    const float* __restrict__ zl,
+                                                                    const uint8_t* __restrict__ wimg, int N, int nb,
+                                                                    int nitems, __nv_bfloat16* __restrict__ out,
+                                                                    int* wd, const QKNorm nq) {
+  constexpr int M = MODE == 0 ? 64 : 128;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sH = smem;                       // nH x 32 KB: H images, then the W image
-  uint8_t* sW = smem;                       // (W lands where H was once num is done)
-  uint8_t* sA = smem + nH * kImg;           // 32 KB: phi(Q), then O_l
-  __shared__ uint64_t bar_in, bar_n, bar_y, bar_w;
-  __shared__ uint32_t tmem_s;
-  __shared__ int abort_s;
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int bh = blockIdx.y;
-  const int iA = MODE == 0 ? 2 * (int)blockIdx.x : (int)blockIdx.x;
-  const int iB = MODE == 0 ? iA + 1 : -1;
-  const bool hasB = MODE == 0 && iB < nb;
-  if (t == 0) {
-    mbar_init(&bar_in, 1);
-    mbar_init(&bar_n, 1);
-    mbar_init(&bar_y, 1);
-    mbar_init(&bar_w, 1);
-    abort_s = 0;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
+  ApBars* bars = reinterpret_cast<ApBars*>(smem + kApOffBars);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nbi = MODE == 0 ? (nb + 1) / 2 : nb;  // items per head
+  if (threadIdx.x == 0) {
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&bars->full[g], 1);
+      mbar_init(&bars->empty[g], 4);
+      mbar_init(&bars->qread[g], 4);
+      mbar_init(&bars->a_full[g], 4);
+      mbar_init(&bars->num_full[g], 1);
+      mbar_init(&bars->o_full[g], 4);
+      mbar_init(&bars->y_full[g], 1);
+      mbar_init(&bars->fin[g], 1);
+    }
+    mbar_init(&bars->w_full, 1);
+    bars->abort = 0;
     mbar_fence_init();
   }
-  if (warp == 0) tmem_alloc(&tmem_s, 256);
+  if (warp == 1) tmem_alloc(&bars->tmem, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tmem_s;
-  if (t == 0) {
-    mbar_expect_tx(&bar_in, nH * kImg);
-    for (int x = 0; x < nH; ++x) {
-      const int i = (x == 0 || !hasB) ? iA : iB;
-      bulk_g2s(sH + x * kImg, himg + ((size_t)bh * nb + i) * kImg, kImg, &bar_in);
-    }
-  }
-  // Row of this thread (same TMEM lane mapping as the flash kernel).
-  int row, i;
-  bool active;
-  if (MODE == 0) {
-    row = 16 * warp + (lane & 15);
-    i = lane >= 16 ? iB : iA;
-    active = lane >= 16 ? hasB : true;
-  } else {
-    row = 32 * warp + lane;
-    i = iA;
-    active = true;
-  }
-  const int blk = MODE == 0 ? 64 : 128;
-  const int n = i * blk + row;
-  const bool store = active && n < N;
-  const int xo = (MODE == 0 && lane >= 16) ? 1 : 0;
-  uint8_t* arow = sA + xo * (kImg / 2);
-  const uint4* qrow = reinterpret_cast<const uint4*>(q + ((size_t)bh * N + (store ? n : 0)) * kD);
-  const float4* zrow = reinterpret_cast<const float4*>(zl + ((size_t)bh * nb + (active ? i : 0)) * kD);
-  float den = 0.f;
-  uint4 qq[16];
-#pragma unroll
-  for (int ch = 0; ch < 16; ++ch) qq[ch] = store ? __ldg(qrow + ch) : make_uint4(0, 0, 0, 0);
-  if (nq.inv && store) {  // QK RMSNorm of the query row
-    const float inv = __ldg(nq.inv + (size_t)(bh / nq.H) * N + n);
-    const uint4* gq = nq.gamma + (bh % nq.H) * 16;
-#pragma unroll
-    for (int ch = 0; ch < 16; ++ch) qq[ch] = rms_row8(qq[ch], inv, __ldg(gq + ch));
-  }
-#pragma unroll
-  for (int ch = 0; ch < 16; ++ch) {
-    const uint32_t w4[4] = {qq[ch].x, qq[ch].y, qq[ch].z, qq[ch].w};
-    const float4 z0 = __ldg(zrow + 2 * ch), z1 = __ldg(zrow + 2 * ch + 1);
-    const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-    uint32_t pk[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float a = phi(bf16_lo(w4[e])), b = phi(bf16_hi(w4[e]));
-      den = fmaf(a, zz[2 * e], den);
-      den = fmaf(b, zz[2 * e + 1], den);
-      pk[e] = pack_bf16(a, b);
-    }
-    *reinterpret_cast<uint4*>(arow + kmajor_off(row, ch * 16, 128, 2048)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  }
-  fence_proxy_async_smem();
-  __syncthreads();
-  const int M = MODE == 0 ? 64 : 128;
+  const uint32_t tmem = bars->tmem;
   const uint32_t id = idesc_bf16(M, 128);
-  const int nx = MODE == 0 ? (hasB ? 2 : 1) : 1;
-  if (t == 0) {
-    if (mbar_wait(&bar_in, 0, &abort_s, wd)) {
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      mbar_expect_tx(&bars->w_full, kApImg);
+      bulk_g2s(smem + kApOffW, wimg, kApImg, &bars->w_full);
+      int it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+        const int g = it & 1, bh = item / nbi, t = item - bh * nbi;
+        if (it >= 2 && !(ok = mbar_wait(&bars->empty[g], ((it >> 1) - 1) & 1, abort, wd))) break;
+        const int n0 = 128 * t, rows = min(128, N - n0);
+        const int i0 = MODE == 0 ? 2 * t : t;
+        const int nimg = (MODE == 0 && i0 + 1 < nb) ? 2 : 1;
+        uint8_t* st = smem + g * kApStage;
+        mbar_expect_tx(&bars->full[g], (uint32_t)rows * (kD * 2) + nimg * kApImg);
+        bulk_g2s(st, q + ((size_t)bh * N + n0) * kD, (uint32_t)rows * (kD * 2), &bars->full[g]);
+        for (int x = 0; x < nimg; ++x)
+          bulk_g2s(st + kApImg + x * kApImg, himg + ((size_t)bh * nb + i0 + x) * kApImg, kApImg, &bars->full[g]);
+      }
+      // Drain: the last two items' copies (earlier ones were consumed) and W.
+      for (int g2 = max(0, it - 2); g2 < it; ++g2) mbar_wait_drain(&bars->full[g2 & 1], (g2 >> 1) & 1, wd);
+      mbar_wait_drain(&bars->w_full, 0, wd);
+      (void)ok;
+    }
+  } else if (warp == 1 || warp == 10) {
+    // ------------------------------ MMA issuers ---------------------------
+    const int second = warp == 10;  // 0: num = phi(Q) H_i; 1: y = O_l W^T
+    if (lane == 0) {
+      bool ok = !second || mbar_wait(&bars->w_full, 0, abort, wd);
+      int it = 0;
+      for (int item = blockIdx.x; ok && item < nitems; item += gridDim.x, ++it) {
+        const int g = it & 1, t = item - (item / nbi) * nbi;
+        const int nx = (MODE == 0 && 2 * t + 1 < nb) ? 2 : 1;
+        uint64_t* wait_bar = second ? &bars->o_full[g] : &bars->a_full[g];
+        if (!(ok = mbar_wait(wait_bar, (it >> 1) & 1, abort, wd))) break;
+        tc_fence_after();
+        const uint8_t* st = smem + g * kApStage;
+        for (int x = 0; x < (MODE == 0 ? nx : 1); ++x) {
+          const uint32_t d = tmem + g * 256 + (second ? 128 : 0) + ((uint32_t)(x * 16) << 16);
+          const uint8_t* bsrc = second ? smem + kApOffW : st + kApImg + x * kApImg;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(d, smem_desc(st + x * (kApImg / 2) + ks * 256, 128, 2048), smem_desc(bsrc + ks * 256, 128, 2048),
+                     id, ks > 0);
+        }
+        mma_commit(second ? &bars->y_full[g] : &bars->num_full[g]);
+      }
+      mma_commit(&bars->fin[second]);
+      mbar_wait_drain(&bars->fin[second], 0, wd);
+    }
+  } else {
+    // ------------------------------ row groups ----------------------------
+    const int grp = (warp - 2) >> 2, wq = warp & 3;  // TMEM lane quadrant wq
+    const int x = MODE == 0 ? lane >> 4 : 0;
+    const int row = MODE == 0 ? 16 * wq + (lane & 15) : 32 * wq + lane;  // row of the M tile (TMEM lane)
+    const int R = 64 * x + row;                                         // row of the item
+    const uint32_t lb = (uint32_t)(32 * wq) << 16;
+    const int sw = lane & 7;
+    bool ok = true;
+    // This group's items: the CTA's items k = grp, grp + 2, ...; use u = k / 2.
+    for (int k = grp, item = blockIdx.x + grp * gridDim.x; item < nitems; k += 2, item += 2 * gridDim.x) {
+      const int g = grp, u = k >> 1;
+      const int bh = item / nbi, t = item - bh * nbi;
+      const int n = 128 * t + R, i = (MODE == 0 ? 2 * t : t) + x;
+      const bool store = n < N;  // (a block past nb has no rows below N)
+      uint8_t* st = smem + g * kApStage;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->full[g], u & 1, abort, wd));
+      if (!ok) break;
+      // Own q row, chunk (c ^ sw) at step c: eight lanes, eight bank groups.
+      uint4 qq[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        qq[c] = store ? *reinterpret_cast<const uint4*>(st + R * (kD * 2) + ((c ^ sw) * 16)) : make_uint4(0, 0, 0, 0);
+      // Back to channel order: qq[c] <- chunk c (an XOR permutation, one
+      // conditional exchange per bit of sw).
+#pragma unroll
+      for (int b = 0; b < 3; ++b) {
+        const bool sb = (sw >> b) & 1;
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          if (!(c & (1 << b))) {
+            const uint4 lo = qq[c], hi = qq[c | (1 << b)];
+            qq[c] = sb ? hi : lo;
+            qq[c | (1 << b)] = sb ? lo : hi;
+          }
+      }
+      // Every row of the group read before the operand overwrites them.
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->qread[g]);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->qread[g], u & 1, abort, wd));
+      if (!ok) break;
+      if (nq.inv && store) {  // QK RMSNorm of the query row
+        const float inv = __ldg(nq.inv + (size_t)(bh / nq.H) * N + n);
+        const uint4* gq = nq.gamma + (bh % nq.H) * 16;
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch) qq[ch] = rms_row8(qq[ch], inv, __ldg(gq + ch));
+      }
+      const float4* zrow = reinterpret_cast<const float4*>(zl + ((size_t)bh * nb + (store ? i : 0)) * kD);
+      float den = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        const uint32_t w4[4] = {qq[ch].x, qq[ch].y, qq[ch].z, qq[ch].w};
+        const float4 z0 = __ldg(zrow + 2 * ch), z1 = __ldg(zrow + 2 * ch + 1);
+        const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = phi(bf16_lo(w4[e])), b = phi(bf16_hi(w4[e]));
+          den = fmaf(a, zz[2 * e], den);
+          den = fmaf(b, zz[2 * e + 1], den);
+          pk[e] = pack_bf16(a, b);
+        }
+        *reinterpret_cast<uint4*>(st + kmajor_off(R, ch * 16, 128, 2048)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->a_full[g]);
+      // num -> O_l = num / den (bf16), the A operand of the second MMA.
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->num_full[g], u & 1, abort, wd));
+      if (!ok) break;
       tc_fence_after();
-      for (int x = 0; x < nx; ++x) {
-        const uint32_t d = tmem + ((uint32_t)(x * 16) << 16);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_bf16(d, smem_desc(sA + x * (kImg / 2) + ks * 256, 128, 2048), smem_desc(sH + x * kImg + ks * 256, 128, 2048),
-                   id, ks > 0);
-      }
-    }
-    mma_commit(&bar_n);
-  }
-  bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_n, 0, &abort_s, wd));
-  tc_fence_after();
-  // The MMAs are done reading H: bring the W image (L2-resident) into its
-  // place while num becomes O_l.
-  if (t == 0) {
-    mbar_expect_tx(&bar_w, kImg);
-    bulk_g2s(sW, wimg, kImg, &bar_w);
-  }
-  const uint32_t lb = (uint32_t)(32 * warp) << 16;
-  {
-    const float inv_den = (store && den > 0.f) ? 1.f / den : 0.f;
+      {
+        const float inv_den = (store && den > 0.f) ? 1.f / den : 0.f;
 #pragma unroll 1
-    for (int c = 0; c < kD; c += 16) {
-      uint32_t v16[16];
-      SAGESLA_TMEM_LD16(tmem + lb + c, v16);
-      tmem_ld_wait();
-      uint32_t pk[8];
+        for (int c = 0; c < kD; c += 16) {
+          uint32_t v16[16];
+          SAGESLA_TMEM_LD16(tmem + lb + g * 256 + c, v16);
+          tmem_ld_wait();
+          uint32_t pk[8];
 #pragma unroll
-      for (int z2 = 0; z2 < 8; ++z2)
-        pk[z2] = pack_bf16(ok ? __uint_as_float(v16[2 * z2]) * inv_den : 0.f,
-                           ok ? __uint_as_float(v16[2 * z2 + 1]) * inv_den : 0.f);
-      *reinterpret_cast<uint4*>(arow + kmajor_off(row, c * 2, 128, 2048)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4*>(arow + kmajor_off(row, c * 2 + 16, 128, 2048)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-    }
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  if (t == 0) {
-    tc_fence_after();
-    if (ok && mbar_wait(&bar_w, 0, &abort_s, wd)) {
-      for (int x = 0; x < nx; ++x) {
-        const uint32_t d = tmem + 128 + ((uint32_t)(x * 16) << 16);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_bf16(d, smem_desc(sA + x * (kImg / 2) + ks * 256, 128, 2048), smem_desc(sW + ks * 256, 128, 2048), id,
-                   ks > 0);
+          for (int z2 = 0; z2 < 8; ++z2)
+            pk[z2] = pack_bf16(__uint_as_float(v16[2 * z2]) * inv_den, __uint_as_float(v16[2 * z2 + 1]) * inv_den);
+          *reinterpret_cast<uint4*>(st + kmajor_off(R, c * 2, 128, 2048)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(st + kmajor_off(R, c * 2 + 16, 128, 2048)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
       }
-    }
-    mma_commit(&bar_y);
-  }
-  ok = __all_sync(0xffffffffu, mbar_wait(&bar_y, 0, &abort_s, wd)) && ok;
-  tc_fence_after();
-  __nv_bfloat16* orow = out + ((size_t)bh * N + (store ? n : 0)) * kD;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->o_full[g]);
+      // y -> bf16 rows.  Staging (this warp's 8 KB of the stage): piece
+      // (chunk C, lane l) at slot 32 C + (l ^ (C % 8)).
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->y_full[g], u & 1, abort, wd));
+      if (!ok) break;
+      tc_fence_after();
+      uint8_t* stg = st + ((warp - 2) & 3) * 8192;
 #pragma unroll 1
-  for (int c = 0; c < kD; c += 16) {
-    uint32_t v16[16];
-    SAGESLA_TMEM_LD16(tmem + lb + 128 + c, v16);
-    tmem_ld_wait();
-    if (store) {
-      uint32_t pk[8];
+      for (int c = 0; c < kD; c += 16) {
+        uint32_t v16[16];
+        SAGESLA_TMEM_LD16(tmem + lb + g * 256 + 128 + c, v16);
+        tmem_ld_wait();
 #pragma unroll
-      for (int z2 = 0; z2 < 8; ++z2)
-        pk[z2] = pack_bf16(ok ? __uint_as_float(v16[2 * z2]) : 0.f, ok ? __uint_as_float(v16[2 * z2 + 1]) : 0.f);
-      *reinterpret_cast<uint4*>(orow + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4*>(orow + c + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int z2 = 0; z2 < 4; ++z2)
+            pk[z2] = pack_bf16(__uint_as_float(v16[8 * h + 2 * z2]), __uint_as_float(v16[8 * h + 2 * z2 + 1]));
+          const int C = c / 8 + h;
+          *reinterpret_cast<uint4*>(stg + (32 * C + (lane ^ (C & 7))) * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      // Rows of this warp: lane l wrote row R(l) = 64 (l/16) + 16 wq + l%16
+      // (block 64) or 32 wq + l (block 128); lanes 2k and 2k+1 are adjacent
+      // tokens.  Instruction k: lanes 0-15 write row 2k + 0, lanes 16-31 row
+      // 2k + 1, chunk lane % 16.
+#pragma unroll 4
+      for (int k = 0; k < 16; ++k) {
+        const int lr = 2 * k + (lane >> 4), C = lane & 15;
+        const int Rr = MODE == 0 ? 64 * (lr >> 4) + 16 * wq + (lr & 15) : 32 * wq + lr;
+        const int nr = 128 * t + Rr;
+        const uint4 w = *reinterpret_cast<const uint4*>(stg + (32 * C + (lr ^ (C & 7))) * 16);
+        if (nr < N) *reinterpret_cast<uint4*>(out + ((size_t)bh * N + nr) * kD + C * 8) = w;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->empty[g]);
     }
-  }
-  // The inputs' bulk copies must have landed before the CTA exits.
-  if (t == 0) {
-    mbar_wait_drain(&bar_in, 0, wd);
-    mbar_wait_drain(&bar_w, 0, wd);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-int linear_apply_smem(int block) { return (block == 64 ? 3 : 2) * 32768 + 1024; }
+int linear_apply_smem(int) { return kApSmem; }
 
 cudaError_t launch_linear_apply(const void* q, const uint16_t* himg, const float* zl, const uint16_t* wimg,
                                 const Geom& g, void* out, int* wd, cudaStream_t st, QKNorm nq) {
-  const int smem = linear_apply_smem(g.block);
+  const int nbi = g.block == 64 ? (g.nb + 1) / 2 : g.nb;
+  const int nitems = g.BH * nbi;
+  int dev = 0, sms = 0;
   cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = min(nitems, sms);
   if (g.block == 64) {
-    e = cudaFuncSetAttribute(linear_apply_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(linear_apply_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kApSmem);
     if (e != cudaSuccess) return e;
-    linear_apply_kernel<0><<<dim3((g.nb + 1) / 2, g.BH), 128, smem, st>>>(
-        (const uint16_t*)q, (const uint8_t*)himg, zl, (const uint8_t*)wimg, g.N, g.nb, (__nv_bfloat16*)out, wd, nq);
+    linear_apply_kernel<0><<<grid, kApThreads, kApSmem, st>>>((const uint16_t*)q, (const uint8_t*)himg, zl,
+                                                              (const uint8_t*)wimg, g.N, g.nb, nitems,
+                                                              (__nv_bfloat16*)out, wd, nq);
   } else {
-    e = cudaFuncSetAttribute(linear_apply_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(linear_apply_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kApSmem);
     if (e != cudaSuccess) return e;
-    linear_apply_kernel<1><<<dim3(g.nb, g.BH), 128, smem, st>>>(
-        (const uint16_t*)q, (const uint8_t*)himg, zl, (const uint8_t*)wimg, g.N, g.nb, (__nv_bfloat16*)out, wd, nq);
+    linear_apply_kernel<1><<<grid, kApThreads, kApSmem, st>>>((const uint16_t*)q, (const uint8_t*)himg, zl,
+                                                              (const uint8_t*)wimg, g.N, g.nb, nitems,
+                                                              (__nv_bfloat16*)out, wd, nq);
   }
   return cudaGetLastError();
 }
@@ -529,24 +780,28 @@ __global__ void w_tile_kernel(const uint16_t* __restrict__ w, uint16_t* __restri
   wt[himg_off(co, ci) / 2] = w[co * kD + ci];
 }
 
-int linear_kv_smem(int block) { return 2 * block * 128 * 2 + 1024; }
+int linear_kv_smem(int) { return kKvSmem; }
 int linear_sum_smem() { return kLStages * (kHsTile + kSumTiles * kATile) + (int)sizeof(LBars) + 1024; }
 
 cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_t* hs, float* z, int* wd,
                              cudaStream_t st, QKNorm nk) {
   const int nbt = (g.nb + 63) / 64;
-  const int smem = linear_kv_smem(g.block);
+  const int nitems = g.BH * nbt * (64 / kKvJ);
+  int dev = 0, sms = 0;
   cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = min(nitems, sms);
   if (g.block == 64) {
-    e = cudaFuncSetAttribute(linear_kv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(linear_kv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
     if (e != cudaSuccess) return e;
-    linear_kv_kernel<64><<<dim3(nbt * 64, g.BH), 256, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt, hs,
-                                                                  z, wd, nk);
+    linear_kv_kernel<64><<<grid, kKvThreads, kKvSmem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt, nitems,
+                                                            hs, z, wd, nk);
   } else {
-    e = cudaFuncSetAttribute(linear_kv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(linear_kv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
     if (e != cudaSuccess) return e;
-    linear_kv_kernel<128><<<dim3(nbt * 64, g.BH), 256, smem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt,
-                                                                   hs, z, wd, nk);
+    linear_kv_kernel<128><<<grid, kKvThreads, kKvSmem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt,
+                                                             nitems, hs, z, wd, nk);
   }
   return cudaGetLastError();
 }

@@ -92,10 +92,11 @@ __global__ void stats_final_kernel(const double* __restrict__ psum, const float*
 // next kQStages tiles in shared memory with bulk copies (one per tensor,
 // nvalid x 256 bytes, completing on the stage's mbarrier), so that the HBM
 // reads of later tiles overlap the quantisation of this one.
-//   Q/K: thread t holds channels 8*cg..+7 (cg = (t/8) % 16) of the rows
-//        t%8 + 32*(t/128) + 8*i, i < 4.  A warp spans 8 rows and 4 channel
-//        groups, so its 8-byte stores into the K-major tile images cover
-//        all 32 banks twice (no conflict).
+//   Q/K: thread t holds channels 8*cg..+7 (cg = (t/8 + t%8) % 16) of the
+//        rows t%8 + 32*(t/128) + 8*i, i < 4.  The eight lanes of a quarter
+//        warp read eight rows at eight different cg%8, i.e. eight bank
+//        groups, and a warp's 8-byte stores into the K-major tile images
+//        cover all 32 banks twice (no conflict either way).
 //   V:   warp w converts keys 16*(w/2)..+15 of channels 64*(w%2)..+63; lane
 //        l the channel pair c0 = 64*(w%2) + 2l, c0 + 1.  Each channel gives
 //        one 16-byte chunk (16 consecutive keys) of the V^T image; lanes
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   QuantSmem& S = *reinterpret_cast<QuantSmem*>(smem_raw);
   volatile int* abort = &S.abort;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int cg = (t >> 3) & 15, rr = t & 7, h = t >> 7;
+  const int cg = ((t >> 3) + (t & 7)) & 15, rr = t & 7, h = t >> 7;
   const int nmine = (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
   if (t == 0) {
     for (int s = 0; s < kQStages; ++s) mbar_init(&S.full[s], 1);
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const int r = rr + 32 * h + 8 * i;
         const float a = fmaxf(fmaxf(S.rowmax[0][r], S.rowmax[1][r]), fmaxf(S.rowmax[2][r], S.rowmax[3][r]));
         mqr[i] = a > 0.f ? __fdiv_rn(fq, a) : 0.f;
-        if ((t & 0x78) == 0) sq[(size_t)gt * kQB + r] = a > 0.f ? __fdiv_rn(a, fq) : 1.f;  // cg == 0 writes
+        if ((t & 0x78) == 0) sq[(size_t)gt * kQB + r] = a > 0.f ? __fdiv_rn(a, fq) : 1.f;  // one writer per row
       }
     }
 
