@@ -45,6 +45,16 @@ __device__ __forceinline__ size_t hs_chunk(int nbt, int j, int chunk) {
 
 __device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 
+// Shared-memory load kept in program order (not hoisted by the compiler, so
+// a loop over chunks does not hold every chunk's operands in registers).
+__device__ __forceinline__ float4 lds_f4(const float4* p) {
+  float4 r;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "r"(smem_u32(p)));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -500,8 +510,11 @@ __global__ void __launch_bounds__(64 + kAThreads, 1) linear_sum_kernel(const uin
 // (one row per thread), each with its own shared-memory stage and 256 TMEM
 // columns (num, then y), so one group's copies, MMAs and stores overlap the
 // other group's work:
-//   warp 0      bulk-copies an item's q rows (up to 32 KB) and H_i images
-//               into the group's stage; the W image once;
+//   warp 0      bulk-copies an item's H_i images and Z_i rows into the
+//               group's stage once the first MMA of the group's previous
+//               item has read them; the W image once;
+//   warp 11     bulk-copies the item's q rows (up to 32 KB) once the group's
+//               previous item is stored;
 //   warp 1      issues num = phi(Q) H_i for every item;
 //   warp 10     issues y = O_l W^T for every item;
 //   warps 2-9   (row groups) read their q rows (chunk c ^ (lane%8) at step c,
@@ -514,12 +527,13 @@ __global__ void __launch_bounds__(64 + kAThreads, 1) linear_sum_kernel(const uin
 // reading its q row from global memory.  Every wait is bounded.
 namespace {
 constexpr int kApImg = 32768;
-constexpr int kApStage = 3 * kApImg;  // q rows -> phi(Q) -> O_l -> y staging; then two H images
+constexpr int kApOffZ = 3 * kApImg;   // in a stage: q rows -> phi(Q) -> O_l -> y staging; two H images; two Z rows
+constexpr int kApStage = kApOffZ + 2 * kD * 4;
 constexpr int kApOffW = 2 * kApStage;
 constexpr int kApOffBars = kApOffW + kApImg;
-constexpr int kApThreads = 32 * 11;
+constexpr int kApThreads = 32 * 12;
 struct ApBars {
-  uint64_t full[2], empty[2], qread[2], a_full[2], num_full[2], o_full[2], y_full[2], w_full, fin[2];
+  uint64_t full[2], empty[2], h_empty[2], qread[2], a_full[2], num_full[2], o_full[2], y_full[2], w_full, fin[2];
   uint32_t tmem;
   int abort;
 };
@@ -542,8 +556,9 @@ __global__ void __launch_bounds__(kApThreads, 1) linear_apply_kernel(const uint1
   const int nbi = MODE == 0 ? (nb + 1) / 2 : nb;  // items per head
   if (threadIdx.x == 0) {
     for (int g = 0; g < 2; ++g) {
-      mbar_init(&bars->full[g], 1);
+      mbar_init(&bars->full[g], 2);
       mbar_init(&bars->empty[g], 4);
+      mbar_init(&bars->h_empty[g], 1);
       mbar_init(&bars->qread[g], 4);
       mbar_init(&bars->a_full[g], 4);
       mbar_init(&bars->num_full[g], 1);
@@ -562,29 +577,36 @@ __global__ void __launch_bounds__(kApThreads, 1) linear_apply_kernel(const uint1
   const uint32_t tmem = bars->tmem;
   const uint32_t id = idesc_bf16(M, 128);
 
-  if (warp == 0) {
-    // ------------------------------ producer ------------------------------
+  if (warp == 0 || warp == 11) {
+    // ------------------------------ producers -----------------------------
+    const bool hq = warp == 0;  // H images and Z rows (and W), or q rows
     if (lane == 0) {
-      mbar_expect_tx(&bars->w_full, kApImg);
-      bulk_g2s(smem + kApOffW, wimg, kApImg, &bars->w_full);
+      if (hq) {
+        mbar_expect_tx(&bars->w_full, kApImg);
+        bulk_g2s(smem + kApOffW, wimg, kApImg, &bars->w_full);
+      }
       int it = 0;
-      bool ok = true;
       for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
         const int g = it & 1, bh = item / nbi, t = item - bh * nbi;
-        if (it >= 2 && !(ok = mbar_wait(&bars->empty[g], ((it >> 1) - 1) & 1, abort, wd))) break;
-        const int n0 = 128 * t, rows = min(128, N - n0);
-        const int i0 = MODE == 0 ? 2 * t : t;
-        const int nimg = (MODE == 0 && i0 + 1 < nb) ? 2 : 1;
+        if (it >= 2 && !mbar_wait(hq ? &bars->h_empty[g] : &bars->empty[g], ((it >> 1) - 1) & 1, abort, wd)) break;
         uint8_t* st = smem + g * kApStage;
-        mbar_expect_tx(&bars->full[g], (uint32_t)rows * (kD * 2) + nimg * kApImg);
-        bulk_g2s(st, q + ((size_t)bh * N + n0) * kD, (uint32_t)rows * (kD * 2), &bars->full[g]);
-        for (int x = 0; x < nimg; ++x)
-          bulk_g2s(st + kApImg + x * kApImg, himg + ((size_t)bh * nb + i0 + x) * kApImg, kApImg, &bars->full[g]);
+        if (hq) {
+          const int i0 = MODE == 0 ? 2 * t : t;
+          const int nimg = (MODE == 0 && i0 + 1 < nb) ? 2 : 1;
+          mbar_expect_tx(&bars->full[g], nimg * (kApImg + kD * 4));
+          for (int x = 0; x < nimg; ++x) {
+            bulk_g2s(st + kApImg + x * kApImg, himg + ((size_t)bh * nb + i0 + x) * kApImg, kApImg, &bars->full[g]);
+            bulk_g2s(st + kApOffZ + x * kD * 4, zl + ((size_t)bh * nb + i0 + x) * kD, kD * 4, &bars->full[g]);
+          }
+        } else {
+          const int n0 = 128 * t, rows = min(128, N - n0);
+          mbar_expect_tx(&bars->full[g], (uint32_t)rows * (kD * 2));
+          bulk_g2s(st, q + ((size_t)bh * N + n0) * kD, (uint32_t)rows * (kD * 2), &bars->full[g]);
+        }
       }
       // Drain: the last two items' copies (earlier ones were consumed) and W.
       for (int g2 = max(0, it - 2); g2 < it; ++g2) mbar_wait_drain(&bars->full[g2 & 1], (g2 >> 1) & 1, wd);
-      mbar_wait_drain(&bars->w_full, 0, wd);
-      (void)ok;
+      if (hq) mbar_wait_drain(&bars->w_full, 0, wd);
     }
   } else if (warp == 1 || warp == 10) {
     // ------------------------------ MMA issuers ---------------------------
@@ -607,7 +629,12 @@ __global__ void __launch_bounds__(kApThreads, 1) linear_apply_kernel(const uint1
             mma_bf16(d, smem_desc(st + x * (kApImg / 2) + ks * 256, 128, 2048), smem_desc(bsrc + ks * 256, 128, 2048),
                      id, ks > 0);
         }
-        mma_commit(second ? &bars->y_full[g] : &bars->num_full[g]);
+        if (second) {
+          mma_commit(&bars->y_full[g]);
+        } else {
+          mma_commit(&bars->num_full[g]);
+          mma_commit(&bars->h_empty[g]);  // H images and Z rows read
+        }
       }
       mma_commit(&bars->fin[second]);
       mbar_wait_drain(&bars->fin[second], 0, wd);
@@ -625,7 +652,7 @@ __global__ void __launch_bounds__(kApThreads, 1) linear_apply_kernel(const uint1
     for (int k = grp, item = blockIdx.x + grp * gridDim.x; item < nitems; k += 2, item += 2 * gridDim.x) {
       const int g = grp, u = k >> 1;
       const int bh = item / nbi, t = item - bh * nbi;
-      const int n = 128 * t + R, i = (MODE == 0 ? 2 * t : t) + x;
+      const int n = 128 * t + R;
       const bool store = n < N;  // (a block past nb has no rows below N)
       uint8_t* st = smem + g * kApStage;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->full[g], u & 1, abort, wd));
@@ -659,12 +686,13 @@ __global__ void __launch_bounds__(kApThreads, 1) linear_apply_kernel(const uint1
 #pragma unroll
         for (int ch = 0; ch < 16; ++ch) qq[ch] = rms_row8(qq[ch], inv, __ldg(gq + ch));
       }
-      const float4* zrow = reinterpret_cast<const float4*>(zl + ((size_t)bh * nb + (store ? i : 0)) * kD);
+      // Z_i of this row's block, staged (rows of a block past nb are never stored).
+      const float4* zrow = reinterpret_cast<const float4*>(st + kApOffZ + x * kD * 4);
       float den = 0.f;
 #pragma unroll
       for (int ch = 0; ch < 16; ++ch) {
         const uint32_t w4[4] = {qq[ch].x, qq[ch].y, qq[ch].z, qq[ch].w};
-        const float4 z0 = __ldg(zrow + 2 * ch), z1 = __ldg(zrow + 2 * ch + 1);
+        const float4 z0 = lds_f4(zrow + 2 * ch), z1 = lds_f4(zrow + 2 * ch + 1);
         const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
         uint32_t pk[4];
 #pragma unroll
