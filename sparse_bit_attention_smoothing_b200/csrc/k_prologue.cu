@@ -18,7 +18,9 @@ namespace sagesla {
 
 // ---------------------------------------------------------------- K1 ----
 // grid (split, BH), 128 threads.  Thread t covers channels 8*(t%16)..+7 of
-// rows t/16, t/16+8, ... of its split.
+// rows t/16, t/16+8, ... of its split.  NORM: the QK RMSNorm is applied to
+// the key rows (a separate instance, so the plain loop stays branch-free).
+template <bool NORM>
 __global__ void __launch_bounds__(128) stats_partial_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                                             int N, int rows_per_split, double* __restrict__ psum,
                                                             float* __restrict__ pmax, const QKNorm nk) {
@@ -34,13 +36,13 @@ __global__ void __launch_bounds__(128) stats_partial_kernel(const uint4* __restr
     m[i] = 0.f;
   }
   const size_t base = (size_t)bh * N * 16;  // in uint4 (8 bf16) units
-  const uint4 gk = nk.inv ? __ldg(nk.gamma + (bh % nk.H) * 16 + cg) : make_uint4(0, 0, 0, 0);
-  const float* invk = nk.inv ? nk.inv + (size_t)(bh / max(1, nk.H)) * N : nullptr;
+  const uint4 gk = NORM ? __ldg(nk.gamma + (bh % nk.H) * 16 + cg) : make_uint4(0, 0, 0, 0);
+  const float* invk = NORM ? nk.inv + (size_t)(bh / max(1, nk.H)) * N : nullptr;
 #pragma unroll 4
   for (int n = n_begin + r0; n < n_end; n += 8) {  // unrolled: four row pairs of loads in flight
     uint4 kk = __ldg(k + base + (size_t)n * 16 + cg);
     uint4 vv = __ldg(v + base + (size_t)n * 16 + cg);
-    if (invk) kk = rms_row8(kk, __ldg(invk + n), gk);
+    if (NORM) kk = rms_row8(kk, __ldg(invk + n), gk);
     uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};
     uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
@@ -407,8 +409,12 @@ __global__ void untile_kernel(const uint8_t* __restrict__ q8t, const uint8_t* __
 cudaError_t launch_stats_partial(const void* k, const void* v, const Geom& g, double* psum, float* pmax,
                                  cudaStream_t st, QKNorm nk) {
   const int rows = (g.N + g.split - 1) / g.split;
-  stats_partial_kernel<<<dim3(g.split, g.BH), 128, 0, st>>>((const uint4*)k, (const uint4*)v, g.N, rows, psum, pmax,
-                                                            nk);
+  if (nk.inv)
+    stats_partial_kernel<true><<<dim3(g.split, g.BH), 128, 0, st>>>((const uint4*)k, (const uint4*)v, g.N, rows, psum,
+                                                                    pmax, nk);
+  else
+    stats_partial_kernel<false><<<dim3(g.split, g.BH), 128, 0, st>>>((const uint4*)k, (const uint4*)v, g.N, rows, psum,
+                                                                     pmax, nk);
   return cudaGetLastError();
 }
 
