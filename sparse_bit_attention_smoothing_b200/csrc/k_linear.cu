@@ -446,8 +446,17 @@ __global__ void __launch_bounds__(64 + kAThreads, 1) linear_sum_kernel(const uin
     const int u = (tid - 64) >> 7, r = (tid - 64) & 127;
     const int i = i0 + 128 * u + r;
     bool ok = true;
+    // The row's selection words, loaded two K tiles ahead of their use.
+    const uint32_t* sb = selbits + ((size_t)bh * nb + (i < nb ? i : 0)) * nbw;
+    auto sel_word = [&](int kt) -> uint64_t {
+      return (i < nb && kt < nbt) ? ((uint64_t)__ldg(sb + 2 * kt) | ((uint64_t)__ldg(sb + 2 * kt + 1) << 32)) : 0ull;
+    };
+    uint64_t wa = sel_word(0), wb = sel_word(1);
     for (int kt = 0; kt < nbt; ++kt) {
       const int st = kt % kLStages;
+      const uint64_t w = wa;
+      wa = wb;
+      wb = sel_word(kt + 2);
       if (kt >= kLStages) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->empty[st], ((kt / kLStages) - 1) & 1, abort, wd));
         if (!ok) break;
@@ -455,8 +464,6 @@ __global__ void __launch_bounds__(64 + kAThreads, 1) linear_sum_kernel(const uin
       // ones = NOT selected and j < nb (and i < nb), as 64 bits
       uint64_t ones = 0;
       if (i < nb) {
-        const uint64_t w = (uint64_t)selbits[((size_t)bh * nb + i) * nbw + 2 * kt] |
-                           ((uint64_t)selbits[((size_t)bh * nb + i) * nbw + 2 * kt + 1] << 32);
         const int left = nb - kt * 64;  // key blocks of this tile that exist
         ones = ~w & (left >= 64 ? ~0ull : ((1ull << left) - 1ull));
       }

@@ -269,12 +269,14 @@ __global__ void __launch_bounds__(32 * TQ) pool_topk_kernel(const float* __restr
 }
 
 // Sixteen query blocks per CTA, 512 threads (one CTA per SM), for nb <=
-// 1280.  Phase 1: the kbar chunks are double-buffered with cp.async, so the
-// next chunk streams in while this one is scored; thread t takes key t % 64,
-// channel quarter (t / 64) % 4 and query rows 8 * (t / 256) .. + 7.
+// 1280.  Phase 1: the kbar chunks stream through a 3-buffer ring with
+// cp.async, two chunks ahead of the one being scored; thread t takes keys
+// t % 32 and t % 32 + 32 of the chunk, channel eighth (t / 32) % 8 and query
+// rows 8 * (t / 256) .. + 7 (40 shared loads per 256 FMAs); the eight
+// partial dot products of a score are added pairwise.
 // Phase 2 as above, one warp per query row; Z_i gathers 16 rows of z at a
 // time.
-constexpr int kTQ16 = 16, kPER16 = 40;
+constexpr int kTQ16 = 16, kPER16 = 40, kKB16 = 3;
 __global__ void __launch_bounds__(512, 1) pool_topk16_kernel(const float* __restrict__ qbar,
                                                             const float* __restrict__ kbar, int nb, int kc,
                                                             int32_t* __restrict__ idx, const float* __restrict__ zin,
@@ -284,18 +286,18 @@ __global__ void __launch_bounds__(512, 1) pool_topk16_kernel(const float* __rest
   constexpr int kThr = 512;
   extern __shared__ __align__(16) float sm[];
   float* qb = sm;                            // [16][128]
-  float* kb = qb + kTQ16 * kD;               // [2][kKC][kPad]
-  float* psc = kb + 2 * kKC * kPad;          // [4][16][kKC] quarter sums
-  float* sc = psc + 4 * kTQ16 * kKC;         // [16][nb]
+  float* kb = qb + kTQ16 * kD;               // [3][kKC][kPad]
+  float* psc = kb + kKB16 * kKC * kPad;      // [8][16][kKC] eighth sums
+  float* sc = psc + 8 * kTQ16 * kKC;         // [16][nb]
   const int bh = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int i0 = blockIdx.x * kTQ16;
   const float* qh = qbar + (size_t)bh * nb * kD;
   const float* kh = kbar + (size_t)bh * nb * kD;
   const float rs = 1.0f / sqrtf((float)kD);
   const int nchunk = (nb + kKC - 1) / kKC;
-  // Chunk c of kbar into buffer c % 2 (rows past nb read as zeros).
+  // Chunk c of kbar into buffer c % 3 (rows past nb read as zeros).
   auto stage = [&](int c) {
-    float* dst = kb + (c & 1) * kKC * kPad;
+    float* dst = kb + (c % kKB16) * kKC * kPad;
 #pragma unroll
     for (int m = 0; m < kKC * kD / 4 / kThr; ++m) {
       const int e = t + m * kThr;
@@ -306,43 +308,57 @@ __global__ void __launch_bounds__(512, 1) pool_topk16_kernel(const float* __rest
     cp_async_commit();
   };
   stage(0);
+  if (nchunk > 1) stage(1);
   for (int e = t; e < kTQ16 * kD; e += kThr) {
     const int r = e / kD;
     qb[e] = i0 + r < nb ? qh[(size_t)i0 * kD + e] : 0.f;
   }
-  const int jj = t & 63, qg = (t >> 6) & 3, rg = t >> 8;
+  const int jj = t & 31, cs = (t >> 5) & 7, rg = t >> 8;
   for (int c = 0; c < nchunk; ++c) {
-    if (c + 1 < nchunk) {
-      stage(c + 1);
+    // Buffer (c + 2) % 3 was last read in chunk c - 1, before its second barrier.
+    if (c + 2 < nchunk) {
+      stage(c + 2);
+      cp_async_wait<2>();
+    } else if (c + 1 < nchunk) {
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
-    __syncthreads();  // chunk c is in buffer c % 2 for every thread
-    const float* kr = kb + (c & 1) * kKC * kPad + jj * kPad + 32 * qg;
-    float a[8];
+    __syncthreads();  // chunk c is in buffer c % 3 for every thread
+    const float* kr = kb + (c % kKB16) * kKC * kPad + jj * kPad + 16 * cs;
+    float a[8][2];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) a[r] = 0.f;
+    for (int r = 0; r < 8; ++r) a[r][0] = a[r][1] = 0.f;
 #pragma unroll
-    for (int cc = 0; cc < 32; cc += 4) {
-      const float4 k4 = *reinterpret_cast<const float4*>(kr + cc);
+    for (int cc = 0; cc < 16; cc += 4) {
+      const float4 ka = *reinterpret_cast<const float4*>(kr + cc);
+      const float4 kb4 = *reinterpret_cast<const float4*>(kr + 32 * kPad + cc);
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        const float4 x = *reinterpret_cast<const float4*>(qb + (8 * rg + r) * kD + 32 * qg + cc);
-        a[r] = fmaf(x.x, k4.x, a[r]);
-        a[r] = fmaf(x.y, k4.y, a[r]);
-        a[r] = fmaf(x.z, k4.z, a[r]);
-        a[r] = fmaf(x.w, k4.w, a[r]);
+        const float4 x = *reinterpret_cast<const float4*>(qb + (8 * rg + r) * kD + 16 * cs + cc);
+        a[r][0] = fmaf(x.x, ka.x, a[r][0]);
+        a[r][0] = fmaf(x.y, ka.y, a[r][0]);
+        a[r][0] = fmaf(x.z, ka.z, a[r][0]);
+        a[r][0] = fmaf(x.w, ka.w, a[r][0]);
+        a[r][1] = fmaf(x.x, kb4.x, a[r][1]);
+        a[r][1] = fmaf(x.y, kb4.y, a[r][1]);
+        a[r][1] = fmaf(x.z, kb4.z, a[r][1]);
+        a[r][1] = fmaf(x.w, kb4.w, a[r][1]);
       }
     }
 #pragma unroll
-    for (int r = 0; r < 8; ++r) psc[(qg * kTQ16 + 8 * rg + r) * kKC + jj] = a[r];
-    __syncthreads();  // quarter sums complete; buffer c % 2 may be refilled
+    for (int r = 0; r < 8; ++r) {
+      psc[(cs * kTQ16 + 8 * rg + r) * kKC + jj] = a[r][0];
+      psc[(cs * kTQ16 + 8 * rg + r) * kKC + jj + 32] = a[r][1];
+    }
+    __syncthreads();  // eighth sums complete; buffer c % 3 may be refilled
     for (int e = t; e < kTQ16 * kKC; e += kThr) {
       const int r = e / kKC, k = e % kKC, jk = c * kKC + k;
+      const float* p = psc + r * kKC + k;
+      constexpr int kS = kTQ16 * kKC;  // stride between eighths
       if (jk < nb)
-        sc[r * nb + jk] = ((psc[(0 * kTQ16 + r) * kKC + k] + psc[(1 * kTQ16 + r) * kKC + k]) +
-                           (psc[(2 * kTQ16 + r) * kKC + k] + psc[(3 * kTQ16 + r) * kKC + k])) * rs;
+        sc[r * nb + jk] = (((p[0] + p[kS]) + (p[2 * kS] + p[3 * kS])) +
+                           ((p[4 * kS] + p[5 * kS]) + (p[6 * kS] + p[7 * kS]))) * rs;
     }
   }
   __syncthreads();
@@ -453,13 +469,13 @@ cudaError_t launch_pool_topk(const float* qsum, const float* ksum, const Geom& g
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  // Sixteen query blocks per CTA (512 threads, double-buffered kbar chunks,
+  // Sixteen query blocks per CTA (512 threads, a 3-buffer ring of kbar chunks,
   // one CTA per SM) up to nb = 1280, where the order keys fit in registers;
   // else eight query blocks per CTA where the scores fit in shared memory;
   // else four.
   constexpr size_t kSmemMax = 227 * 1024;
   if (g.nb <= 32 * kPER16) {
-    const size_t smem = sizeof(float) * ((size_t)kTQ16 * kD + 2 * (size_t)kKC * kPad + 4 * (size_t)kTQ16 * kKC +
+    const size_t smem = sizeof(float) * ((size_t)kTQ16 * kD + kKB16 * (size_t)kKC * kPad + 8 * (size_t)kTQ16 * kKC +
                                          (size_t)kTQ16 * g.nb);
     e = cudaFuncSetAttribute(pool_topk16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
