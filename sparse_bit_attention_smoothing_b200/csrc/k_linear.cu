@@ -480,26 +480,37 @@ __global__ void __launch_bounds__(64 + kAThreads, 1) linear_sum_kernel(const uin
       fence_proxy_async_smem();
       mbar_arrive(&bars->a_full[st]);
     }
-    // Epilogue: row i of D (256 fp32 columns) -> bf16 image columns.
+    // Epilogue: row i of D (256 fp32 columns) -> 512 bytes of bf16 image
+    // columns.  The MMAs are done, so the operand ring is free: each warp
+    // stages its 32 rows there (16-byte piece c of row l at slot
+    // 32 l + (c ^ (l % 8)): eight lanes, eight bank groups), then stores one
+    // whole row per instruction.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, abort, wd));
     if (ok) {
       tc_fence_after();
       const int q = warp & 3, ue = (warp - 2) >> 2;  // TMEM quadrant, M tile
-      const int row = 32 * q + lane;  // TMEM lane == row of the M=128 tile
-      const int ir = i0 + 128 * ue + row;
-      uint16_t* dst = hout + ((size_t)bh * nb + (ir < nb ? ir : 0)) * 16384 + (size_t)nt * 256;
+      uint4* stg = reinterpret_cast<uint4*>(smem + (warp - 2) * 16384);
 #pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 16) {
-        uint32_t v16[16];
-        SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * q) << 16) + ue * 256 + c0, v16);
+      for (int c0 = 0; c0 < 256; c0 += 32) {
+        uint32_t v[32];
+        SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * q) << 16) + ue * 256 + c0, v);
+        SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * q) << 16) + ue * 256 + c0 + 16, v + 16);
         tmem_ld_wait();
-        if (ir < nb) {
-          uint32_t pk[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(__uint_as_float(v16[2 * e]), __uint_as_float(v16[2 * e + 1]));
-          *reinterpret_cast<uint4*>(dst + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(dst + c0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        for (int h = 0; h < 4; ++h) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pk[e] = pack_bf16(__uint_as_float(v[8 * h + 2 * e]), __uint_as_float(v[8 * h + 2 * e + 1]));
+          const int c = c0 / 8 + h;
+          stg[32 * lane + (c ^ (lane & 7))] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
+      }
+      __syncwarp();
+#pragma unroll 4
+      for (int k = 0; k < 32; ++k) {
+        const int ir = i0 + 128 * ue + 32 * q + k;  // TMEM lane 32q + k == row of the M=128 tile
+        const uint4 w = stg[32 * k + (lane ^ (k & 7))];
+        if (ir < nb) *reinterpret_cast<uint4*>(hout + ((size_t)bh * nb + ir) * 16384 + (size_t)nt * 256 + lane * 8) = w;
       }
     }
   }
