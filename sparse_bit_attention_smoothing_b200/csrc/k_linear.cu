@@ -360,44 +360,51 @@ __global__ void __launch_bounds__(kKvThreads, 1) linear_kv_kernel(const uint4* _
 }
 
 // ---------------------------------------------------------------- K4b ----
-// grid (ceil(nb/256), 64 n-tiles, BH): the CTAs that read the same B tiles
-// are neighbours in launch order.  A CTA covers two M=128 tiles of query
-// blocks, so each B tile it loads feeds two MMA chains.  320 threads: warp 0
-// bulk-loads the B tiles, warp 1 issues MMAs, warps 2-9 expand the 0/1 A
-// tiles from the selection bitmask and run the epilogue.  K tiles of 64 key
-// blocks, 3-stage ring; D = 2 x (128 x 256) fp32 in TMEM.
+// Persistent, one CTA per SM.  Tiles (query-block group it, n-tile nt, head
+// bh) are numbered it fastest, then nt, then bh, and dealt round-robin, so the
+// CTAs that read the same B tiles work on them at the same time.  A tile is
+// two M=128 tiles of query blocks, so each B tile loaded feeds two MMA
+// chains.  320 threads: warp 0 bulk-loads the B tiles, warp 1 issues MMAs,
+// warps 2-9 expand the 0/1 A tiles from the selection bitmask and run the
+// epilogue.  K tiles of 64 key blocks through a 3-stage ring whose stages
+// continue across tiles, so the next tile's first stages fill while this
+// tile's epilogue drains TMEM; D = 2 x (128 x 256) fp32 in TMEM.
 namespace {
 constexpr int kLStages = 3;
-constexpr int kSumTiles = 2;          // M=128 query-block tiles per CTA
+constexpr int kSumTiles = 2;          // M=128 query-block tiles per CTA tile
 constexpr int kATile = 128 * 64 * 2;  // 16 KB per M tile
 constexpr int kAThreads = 128 * kSumTiles;
+constexpr int kAWarps = kAThreads / 32;
+constexpr int kSumStg = 32 * 64 * 2;  // per epilogue warp: 32 rows x 64 bf16 columns
 struct LBars {
-  uint64_t b_full[kLStages], a_full[kLStages], empty[kLStages], done;
+  uint64_t b_full[kLStages], a_full[kLStages], empty[kLStages], acc_full, acc_empty, fin;
   uint32_t tmem;
   int abort;
 };
+constexpr int kSumOffStg = kLStages * (kHsTile + kSumTiles * kATile);
+constexpr int kSumOffBars = kSumOffStg + kAWarps * kSumStg;
 }  // namespace
 
 __global__ void __launch_bounds__(64 + kAThreads, 1) linear_sum_kernel(const uint8_t* __restrict__ hs,
                                                              const uint32_t* __restrict__ selbits, int nb, int nbt,
-                                                             int nbw, uint16_t* __restrict__ hout, int* wd) {
+                                                             int nbw, int ngrp, int ntiles,
+                                                             uint16_t* __restrict__ hout, int* wd) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sB = smem;                               // kLStages x 32 KB
   uint8_t* sA = smem + kLStages * kHsTile;          // kLStages x kSumTiles x 16 KB
-  LBars* bars = reinterpret_cast<LBars*>(sA + kLStages * kSumTiles * kATile);
+  LBars* bars = reinterpret_cast<LBars*>(smem + kSumOffBars);
   volatile int* abort = &bars->abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int it = blockIdx.x, nt = blockIdx.y, bh = blockIdx.z;
-  const int i0 = it * 128 * kSumTiles;
-  const uint8_t* hs_head = hs + (size_t)bh * nbt * 64 * 16384 * 2;
   if (tid == 0) {
     for (int s = 0; s < kLStages; ++s) {
       mbar_init(&bars->b_full[s], 1);
-      mbar_init(&bars->a_full[s], kAThreads);
+      mbar_init(&bars->a_full[s], kAWarps);
       mbar_init(&bars->empty[s], 1);
     }
-    mbar_init(&bars->done, 1);
+    mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->acc_empty, kAWarps);
+    mbar_init(&bars->fin, 1);
     bars->abort = 0;
     mbar_fence_init();
   }
@@ -407,110 +414,136 @@ __global__ void __launch_bounds__(64 + kAThreads, 1) linear_sum_kernel(const uin
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
   if (warp == 0) {
+    // ------------------------------ B producer ----------------------------
     if (lane == 0) {
-      int issued = 0;
-      for (int kt = 0; kt < nbt && !*abort; ++kt) {
-        const int st = kt % kLStages;
-        if (kt >= kLStages && !mbar_wait(&bars->empty[st], ((kt / kLStages) - 1) & 1, abort, wd)) break;
-        mbar_expect_tx(&bars->b_full[st], kHsTile);
-        bulk_g2s(sB + st * kHsTile, hs_head + ((size_t)nt * nbt + kt) * kHsTile, kHsTile, &bars->b_full[st]);
-        issued = kt + 1;
+      int g = 0;  // K stages issued, over all tiles
+      bool ok = true;
+      for (int T = blockIdx.x; ok && T < ntiles; T += gridDim.x) {
+        const int nt = (T / ngrp) % 64, bh = T / (ngrp * 64);
+        const uint8_t* hs_head = hs + (size_t)bh * nbt * 64 * 16384 * 2;
+        for (int kt = 0; kt < nbt; ++kt, ++g) {
+          const int st = g % kLStages;
+          if (g >= kLStages && !(ok = mbar_wait(&bars->empty[st], ((g / kLStages) - 1) & 1, abort, wd))) break;
+          mbar_expect_tx(&bars->b_full[st], kHsTile);
+          bulk_g2s(sB + st * kHsTile, hs_head + ((size_t)nt * nbt + kt) * kHsTile, kHsTile, &bars->b_full[st]);
+        }
       }
-      for (int kt = (issued > kLStages ? issued - kLStages : 0); kt < issued; ++kt)
-        mbar_wait_drain(&bars->b_full[kt % kLStages], (kt / kLStages) & 1, wd);
+      for (int x = max(0, g - kLStages); x < g; ++x) mbar_wait_drain(&bars->b_full[x % kLStages], (x / kLStages) & 1, wd);
     }
   } else if (warp == 1) {
+    // ------------------------------ MMA issuer ----------------------------
     if (lane == 0) {
       const uint32_t id = idesc_bf16(128, 256, 1);  // B MN-major
+      int g = 0, lt = 0;
       bool ok = true;
-      for (int kt = 0; kt < nbt && ok; ++kt) {
-        const int st = kt % kLStages;
-        ok = mbar_wait(&bars->a_full[st], (kt / kLStages) & 1, abort, wd) &&
-             mbar_wait(&bars->b_full[st], (kt / kLStages) & 1, abort, wd);
+      for (int T = blockIdx.x; ok && T < ntiles; T += gridDim.x, ++lt) {
+        if (lt > 0 && !(ok = mbar_wait(&bars->acc_empty, (lt - 1) & 1, abort, wd))) break;
+        for (int kt = 0; kt < nbt; ++kt, ++g) {
+          const int st = g % kLStages;
+          ok = mbar_wait(&bars->a_full[st], (g / kLStages) & 1, abort, wd) &&
+               mbar_wait(&bars->b_full[st], (g / kLStages) & 1, abort, wd);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int u = 0; u < kSumTiles; ++u)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16(tmem + u * 256, smem_desc(sA + (st * kSumTiles + u) * kATile + ks * 256, kQK_LBO, kQK_SBO),
+                       smem_desc(sB + st * kHsTile + ks * 2 * kHs_LBO, kHs_LBO, kHs_SBO), id, (kt > 0 || ks > 0));
+          mma_commit(&bars->empty[st]);
+        }
         if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int u = 0; u < kSumTiles; ++u)
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(tmem + u * 256, smem_desc(sA + (st * kSumTiles + u) * kATile + ks * 256, kQK_LBO, kQK_SBO),
-                     smem_desc(sB + st * kHsTile + ks * 2 * kHs_LBO, kHs_LBO, kHs_SBO), id, (kt > 0 || ks > 0));
-        mma_commit(&bars->empty[st]);
+        mma_commit(&bars->acc_full);
       }
-      mma_commit(&bars->done);
-      mbar_wait_drain(&bars->done, 0, wd);
+      mma_commit(&bars->fin);
+      mbar_wait_drain(&bars->fin, 0, wd);
     }
   } else {
     // A producer: thread -> query block row i = i0 + (tid - 64); 64 key
-    // blocks per K tile from two bitmask words; 1 = NOT selected, j < nb.
+    // blocks per K tile from two bitmask words (loaded two K tiles ahead);
+    // 1 = NOT selected, j < nb.
     const int u = (tid - 64) >> 7, r = (tid - 64) & 127;
-    const int i = i0 + 128 * u + r;
+    const int q = warp & 3, ue = (warp - 2) >> 2;  // epilogue: TMEM quadrant, M tile
+    uint4* stg = reinterpret_cast<uint4*>(smem + kSumOffStg + (warp - 2) * kSumStg);
+    int g = 0, lt = 0;
     bool ok = true;
-    // The row's selection words, loaded two K tiles ahead of their use.
-    const uint32_t* sb = selbits + ((size_t)bh * nb + (i < nb ? i : 0)) * nbw;
-    auto sel_word = [&](int kt) -> uint64_t {
-      return (i < nb && kt < nbt) ? ((uint64_t)__ldg(sb + 2 * kt) | ((uint64_t)__ldg(sb + 2 * kt + 1) << 32)) : 0ull;
-    };
-    uint64_t wa = sel_word(0), wb = sel_word(1);
-    for (int kt = 0; kt < nbt; ++kt) {
-      const int st = kt % kLStages;
-      const uint64_t w = wa;
-      wa = wb;
-      wb = sel_word(kt + 2);
-      if (kt >= kLStages) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->empty[st], ((kt / kLStages) - 1) & 1, abort, wd));
-        if (!ok) break;
-      }
-      // ones = NOT selected and j < nb (and i < nb), as 64 bits
-      uint64_t ones = 0;
-      if (i < nb) {
-        const int left = nb - kt * 64;  // key blocks of this tile that exist
-        ones = ~w & (left >= 64 ? ~0ull : ((1ull << left) - 1ull));
-      }
-      uint8_t* A = sA + (st * kSumTiles + u) * kATile;
+    for (int T = blockIdx.x; ok && T < ntiles; T += gridDim.x, ++lt) {
+      const int it = T % ngrp, nt = (T / ngrp) % 64, bh = T / (ngrp * 64);
+      const int i0 = it * 128 * kSumTiles;
+      const int i = i0 + 128 * u + r;
+      const uint32_t* sb = selbits + ((size_t)bh * nb + (i < nb ? i : 0)) * nbw;
+      auto sel_word = [&](int kt) -> uint64_t {
+        return (i < nb && kt < nbt) ? ((uint64_t)__ldg(sb + 2 * kt) | ((uint64_t)__ldg(sb + 2 * kt + 1) << 32)) : 0ull;
+      };
+      uint64_t wa = sel_word(0), wb = sel_word(1);
+      for (int kt = 0; kt < nbt; ++kt, ++g) {
+        const int st = g % kLStages;
+        const uint64_t w = wa;
+        wa = wb;
+        wb = sel_word(kt + 2);
+        if (g >= kLStages) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars->empty[st], ((g / kLStages) - 1) & 1, abort, wd));
+          if (!ok) break;
+        }
+        // ones = NOT selected and j < nb (and i < nb), as 64 bits
+        uint64_t ones = 0;
+        if (i < nb) {
+          const int left = nb - kt * 64;  // key blocks of this tile that exist
+          ones = ~w & (left >= 64 ? ~0ull : ((1ull << left) - 1ull));
+        }
+        uint8_t* A = sA + (st * kSumTiles + u) * kATile;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {  // 8 keys per 16-byte chunk
-        const uint32_t b8 = (uint32_t)(ones >> (8 * ch)) & 0xFFu;
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)  // bf16 1.0 = 0x3F80 in each half whose bit is set
-          pk[e] = (((b8 >> (2 * e)) & 1u) * 0x3F80u) | (((b8 >> (2 * e + 1)) & 1u) * 0x3F800000u);
-        *reinterpret_cast<uint4*>(A + kmajor_off(r, ch * 16, kQK_LBO, kQK_SBO)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&bars->a_full[st]);
-    }
-    // Epilogue: row i of D (256 fp32 columns) -> 512 bytes of bf16 image
-    // columns.  The MMAs are done, so the operand ring is free: each warp
-    // stages its 32 rows there (16-byte piece c of row l at slot
-    // 32 l + (c ^ (l % 8)): eight lanes, eight bank groups), then stores one
-    // whole row per instruction.
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, abort, wd));
-    if (ok) {
-      tc_fence_after();
-      const int q = warp & 3, ue = (warp - 2) >> 2;  // TMEM quadrant, M tile
-      uint4* stg = reinterpret_cast<uint4*>(smem + (warp - 2) * 16384);
-#pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 32) {
-        uint32_t v[32];
-        SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * q) << 16) + ue * 256 + c0, v);
-        SAGESLA_TMEM_LD16(tmem + ((uint32_t)(32 * q) << 16) + ue * 256 + c0 + 16, v + 16);
-        tmem_ld_wait();
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
+        for (int ch = 0; ch < 8; ++ch) {  // 8 keys per 16-byte chunk
+          const uint32_t b8 = (uint32_t)(ones >> (8 * ch)) & 0xFFu;
           uint32_t pk[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) pk[e] = pack_bf16(__uint_as_float(v[8 * h + 2 * e]), __uint_as_float(v[8 * h + 2 * e + 1]));
-          const int c = c0 / 8 + h;
-          stg[32 * lane + (c ^ (lane & 7))] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          for (int e = 0; e < 4; ++e)  // bf16 1.0 = 0x3F80 in each half whose bit is set
+            pk[e] = (((b8 >> (2 * e)) & 1u) * 0x3F80u) | (((b8 >> (2 * e + 1)) & 1u) * 0x3F800000u);
+          *reinterpret_cast<uint4*>(A + kmajor_off(r, ch * 16, kQK_LBO, kQK_SBO)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->a_full[st]);
       }
-      __syncwarp();
-#pragma unroll 4
-      for (int k = 0; k < 32; ++k) {
-        const int ir = i0 + 128 * ue + 32 * q + k;  // TMEM lane 32q + k == row of the M=128 tile
-        const uint4 w = stg[32 * k + (lane ^ (k & 7))];
-        if (ir < nb) *reinterpret_cast<uint4*>(hout + ((size_t)bh * nb + ir) * 16384 + (size_t)nt * 256 + lane * 8) = w;
+      if (!ok) break;
+      // Epilogue: rows of D (256 fp32 columns) -> bf16 image columns, 64 at a
+      // time through this warp's staging area (16-byte piece p of row l at
+      // slot 8 l + (p ^ (l % 8)): eight lanes, eight bank groups); read back,
+      // eight lanes write one row's 128 contiguous bytes.
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->acc_full, lt & 1, abort, wd));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += 64) {
+        uint32_t v[64];
+        const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + ue * 256 + c0;
+        SAGESLA_TMEM_LD16(ta, v);
+        SAGESLA_TMEM_LD16(ta + 16, v + 16);
+        SAGESLA_TMEM_LD16(ta + 32, v + 32);
+        SAGESLA_TMEM_LD16(ta + 48, v + 48);
+        tmem_ld_wait();
+        if (c0 == 192) {  // every TMEM read of this tile done
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->acc_empty);
+        }
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pk[e] = pack_bf16(__uint_as_float(v[8 * p + 2 * e]), __uint_as_float(v[8 * p + 2 * e + 1]));
+          stg[8 * lane + (p ^ (lane & 7))] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rl = 4 * k + (lane >> 3), p = lane & 7;      // row of this warp, piece
+          const int ir = i0 + 128 * ue + 32 * q + rl;             // TMEM lane 32q + rl == row of the M tile
+          const uint4 w4 = stg[8 * rl + (p ^ (rl & 7))];
+          if (ir < nb)
+            *reinterpret_cast<uint4*>(hout + ((size_t)bh * nb + ir) * 16384 + (size_t)nt * 256 + c0 + 8 * p) = w4;
+        }
+        __syncwarp();
       }
     }
   }
@@ -827,7 +860,7 @@ __global__ void w_tile_kernel(const uint16_t* __restrict__ w, uint16_t* __restri
 }
 
 int linear_kv_smem(int) { return kKvSmem; }
-int linear_sum_smem() { return kLStages * (kHsTile + kSumTiles * kATile) + (int)sizeof(LBars) + 1024; }
+int linear_sum_smem() { return kSumOffBars + (int)sizeof(LBars) + 1024; }
 
 cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_t* hs, float* z, int* wd,
                              cudaStream_t st, QKNorm nk) {
@@ -855,11 +888,17 @@ cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_
 cudaError_t launch_linear_sum(const uint8_t* hs, const uint32_t* selbits, const Geom& g, uint16_t* hout, int* wd,
                               cudaStream_t st) {
   const int nbt = (g.nb + 63) / 64;
+  const int ngrp = (g.nb + 128 * kSumTiles - 1) / (128 * kSumTiles);
+  const int ntiles = ngrp * 64 * g.BH;
   const int smem = linear_sum_smem();
-  cudaError_t e = cudaFuncSetAttribute(linear_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  int dev = 0, sms = 0;
+  cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(linear_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  linear_sum_kernel<<<dim3((g.nb + 128 * kSumTiles - 1) / (128 * kSumTiles), 64, g.BH), 64 + kAThreads, smem, st>>>(
-      hs, selbits, g.nb, nbt, 2 * nbt, hout, wd);
+  linear_sum_kernel<<<min(ntiles, sms), 64 + kAThreads, smem, st>>>(hs, selbits, g.nb, nbt, 2 * nbt, ngrp, ntiles, hout,
+                                                                    wd);
   return cudaGetLastError();
 }
 
