@@ -1,0 +1,358 @@
+"""The mbarrier protocols of the persistent linear-branch kernels, on the CPU.
+
+Each kernel role (a producer thread, an MMA-issuing thread, a warp of
+converters or of the epilogue) is written out as its sequence of steps in
+program order: barrier waits and arrivals, and the begin / end of each access
+to a shared buffer (a shared-memory stage or operand buffer, a TMEM
+accumulator).  Asynchronous work is placed where its completion is signalled:
+a bulk copy writes its stage until the arrival on the stage's full barrier, an
+MMA reads its operands and writes its accumulator until its commit arrives.
+A random scheduler then runs the roles in arbitrary interleavings and checks:
+
+  - no deadlock;
+  - every parity wait is sound: a wait for completion k of a barrier (parity
+    k % 2) must find the barrier at k or k + 1 completions whenever the role
+    stands at it, because the hardware only compares parities (k - 1 would let
+    it through early, k + 2 would hold it for good);
+  - no role writes a buffer while another still reads it (or writes it for a
+    different item), and every read finds the item it expects, completely
+    written.
+
+The role programs follow the kernels in csrc/k_linear.cu (linear_kv_kernel,
+linear_apply_kernel, linear_sum_kernel): the same loop structure, stage and
+phase arithmetic, barrier counts and arrival points.
+"""
+import random
+from collections import defaultdict
+
+import pytest
+
+
+class Violation(AssertionError):
+    pass
+
+
+class Buffers:
+    """Multi-reader buffers with item tags; writers of one tag may overlap."""
+
+    def __init__(self):
+        self.readers = defaultdict(int)
+        self.writers = defaultdict(int)
+        self.wtag = {}
+        self.content = {}
+
+    def wbeg(self, b, tag, who):
+        if self.readers[b]:
+            raise Violation(f"{who} writes {b} ({tag}) while it is read")
+        if self.writers[b] and self.wtag[b] != tag:
+            raise Violation(f"{who} writes {b} ({tag}) while {self.wtag[b]} is being written")
+        self.writers[b] += 1
+        self.wtag[b] = tag
+        self.content[b] = None
+
+    def wend(self, b):
+        self.writers[b] -= 1
+        if self.writers[b] == 0:
+            self.content[b] = self.wtag[b]
+
+    def rbeg(self, b, tag, who):
+        if self.writers[b] or self.content.get(b) != tag:
+            raise Violation(f"{who} reads {b} expecting {tag}, holds {self.content.get(b)} "
+                            f"({self.writers[b]} writers)")
+        self.readers[b] += 1
+
+    def rend(self, b):
+        self.readers[b] -= 1
+
+
+def simulate(programs, counts, seed):
+    """programs: role -> list of steps; counts: barrier -> arrivals per phase."""
+    rng = random.Random(seed)
+    pc = {r: 0 for r in programs}
+    done = defaultdict(int)
+    arrivals = defaultdict(int)
+    buf = Buffers()
+
+    def check_waits():
+        for r, prog in programs.items():
+            if pc[r] < len(prog) and prog[pc[r]][0] == "wait":
+                _, b, k = prog[pc[r]]
+                c = done[b]
+                if c >= k + 2:
+                    raise Violation(f"{r} waits for completion {k} of {b}, which has {c}: parity alias")
+                if c < k and (k - c) % 2 == 1:
+                    raise Violation(f"{r} waits for completion {k} of {b}, which has {c}: passes early")
+
+    while True:
+        check_waits()
+        ready = []
+        for r, prog in programs.items():
+            if pc[r] >= len(prog):
+                continue
+            st = prog[pc[r]]
+            if st[0] != "wait" or done[st[1]] >= st[2] + 1:
+                ready.append(r)
+        if not ready:
+            left = {r: programs[r][pc[r]] for r in programs if pc[r] < len(programs[r])}
+            if left:
+                raise Violation(f"deadlock: {left}")
+            return
+        r = rng.choice(ready)
+        st = programs[r][pc[r]]
+        op = st[0]
+        if op == "arrive":
+            b = st[1]
+            arrivals[b] += 1
+            if arrivals[b] == counts[b]:
+                arrivals[b] = 0
+                done[b] += 1
+        elif op == "wbeg":
+            buf.wbeg(st[1], st[2], r)
+        elif op == "wend":
+            buf.wend(st[1])
+        elif op == "rbeg":
+            buf.rbeg(st[1], st[2], r)
+        elif op == "rend":
+            buf.rend(st[1])
+        pc[r] += 1
+
+
+# --------------------------------------------------------------- linear_kv --
+def linear_kv_programs(nitems, chunks, J=4, stages=3, ops=2, nconv=8, nepi=8):
+    """Single accumulator set (4 blocks per item use all 512 TMEM columns)."""
+    P, C = {}, defaultdict(lambda: 1)
+    U = nitems * J * chunks
+    prod = []
+    for u in range(U):
+        s = u % stages
+        if u >= stages:
+            prod.append(("wait", ("raw_empty", s), u // stages - 1))
+        prod += [("wbeg", ("raw", s), u), ("wend", ("raw", s)), ("arrive", ("raw_full", s))]
+    P["producer"] = prod
+    for w in range(nconv):
+        cv, u, zi = [], 0, 0
+        for it in range(nitems):
+            for jj in range(J):
+                for c in range(chunks):
+                    s, b = u % stages, u % ops
+                    cv.append(("wait", ("raw_full", s), u // stages))
+                    if u >= ops:
+                        cv.append(("wait", ("op_empty", b), u // ops - 1))
+                    cv += [("rbeg", ("raw", s), u), ("wbeg", ("op", b, w), u), ("wend", ("op", b, w)),
+                           ("rend", ("raw", s)), ("arrive", ("op_full", b)), ("arrive", ("raw_empty", s))]
+                    u += 1
+                cv += [("wbeg", ("zred", zi & 1, w), zi), ("wend", ("zred", zi & 1, w)),
+                       ("arrive", ("z_ready", zi & 1)), ("wait", ("z_ready", zi & 1), zi >> 1)]
+                if w < nconv // 2:  # threads ct < 128 add the 16 row slots
+                    cv += [("rbeg", ("zred", zi & 1, x), zi) for x in range(nconv)]
+                    cv += [("rend", ("zred", zi & 1, x)) for x in range(nconv)]
+                zi += 1
+        P[f"conv{w}"] = cv
+    mma, u = [], 0
+    for it in range(nitems):
+        if it > 0:
+            mma.append(("wait", ("acc_empty",), it - 1))
+        for jj in range(J):
+            for c in range(chunks):
+                b = u % ops
+                mma.append(("wait", ("op_full", b), u // ops))
+                mma += [("rbeg", ("op", b, w), u) for w in range(nconv)]
+                if c == 0:
+                    mma.append(("wbeg", ("acc", jj), it))
+                mma += [("rend", ("op", b, w)) for w in range(nconv)]
+                mma.append(("arrive", ("op_empty", b)))
+                u += 1
+        mma += [("wend", ("acc", jj)) for jj in range(J)] + [("arrive", ("acc_full",))]
+    P["mma"] = mma
+    for e in range(nepi):
+        ep = []
+        for it in range(nitems):
+            ep.append(("wait", ("acc_full",), it))
+            ep += [("rbeg", ("acc", jj), it) for jj in range(J)]
+            ep += [("rend", ("acc", jj)) for jj in range(J)] + [("arrive", ("acc_empty",))]
+        P[f"epi{e}"] = ep
+    for s in range(stages):
+        C[("raw_empty", s)] = nconv
+    for b in range(ops):
+        C[("op_full", b)] = nconv
+    C[("z_ready", 0)] = C[("z_ready", 1)] = nconv
+    C[("acc_empty",)] = nepi
+    return P, C
+
+
+# ------------------------------------------------------------ linear_apply --
+def linear_apply_programs(nitems, nrow=4):
+    """Two groups of row warps alternate items; group g = item % 2 owns stage g
+    (q rows -> phi(Q) -> O_l -> y staging in one region, H images and Z rows)
+    and TMEM columns g (num, y).  Region parts: one per row warp; phi(Q) and
+    O_l rows of a warp land in every part, its raw rows and its staging in its
+    own part."""
+    P, C = {}, defaultdict(lambda: 1)
+    parts = range(nrow)
+    hq = [("wbeg", ("W",), 0), ("wend", ("W",)), ("arrive", ("w_full",))]
+    qq = []
+    for k in range(nitems):
+        g, u = k & 1, k >> 1
+        if k >= 2:
+            hq.append(("wait", ("h_empty", g), u - 1))
+            qq.append(("wait", ("empty", g), u - 1))
+        hq += [("wbeg", ("H", g), k), ("wbeg", ("Z", g), k), ("wend", ("H", g)), ("wend", ("Z", g)),
+               ("arrive", ("full", g))]
+        qq += [("wbeg", ("Q", g, p), (k, "q")) for p in parts] + [("wend", ("Q", g, p)) for p in parts]
+        qq.append(("arrive", ("full", g)))
+    P["hprod"], P["qprod"] = hq, qq
+    m1, m2 = [], [("wait", ("w_full",), 0)]
+    for k in range(nitems):
+        g, u = k & 1, k >> 1
+        m1.append(("wait", ("a_full", g), u))
+        m1 += [("rbeg", ("Q", g, p), (k, "a")) for p in parts] + [("rbeg", ("H", g), k), ("wbeg", ("num", g), k)]
+        m1 += [("rend", ("Q", g, p)) for p in parts] + [("rend", ("H", g)), ("wend", ("num", g))]
+        m1 += [("arrive", ("num_full", g)), ("arrive", ("h_empty", g))]
+        m2.append(("wait", ("o_full", g), u))
+        m2 += [("rbeg", ("Q", g, p), (k, "o")) for p in parts] + [("rbeg", ("W",), 0), ("wbeg", ("y", g), k)]
+        m2 += [("rend", ("Q", g, p)) for p in parts] + [("rend", ("W",)), ("wend", ("y", g))]
+        m2.append(("arrive", ("y_full", g)))
+    P["mma1"], P["mma2"] = m1, m2
+    for grp in range(2):
+        for w in range(nrow):
+            rw = []
+            for k in range(grp, nitems, 2):
+                g, u = grp, k >> 1
+                rw += [("wait", ("full", g), u), ("rbeg", ("Q", g, w), (k, "q")), ("rend", ("Q", g, w)),
+                       ("arrive", ("qread", g)), ("wait", ("qread", g), u), ("rbeg", ("Z", g), k)]
+                rw += [("wbeg", ("Q", g, p), (k, "a")) for p in parts] + [("wend", ("Q", g, p)) for p in parts]
+                rw += [("rend", ("Z", g)), ("arrive", ("a_full", g)), ("wait", ("num_full", g), u),
+                       ("rbeg", ("num", g), k)]
+                rw += [("wbeg", ("Q", g, p), (k, "o")) for p in parts] + [("wend", ("Q", g, p)) for p in parts]
+                rw += [("rend", ("num", g)), ("arrive", ("o_full", g)), ("wait", ("y_full", g), u),
+                       ("rbeg", ("y", g), k), ("rend", ("y", g)),
+                       ("wbeg", ("Q", g, w), (k, "y")), ("wend", ("Q", g, w)),
+                       ("rbeg", ("Q", g, w), (k, "y")), ("rend", ("Q", g, w)), ("arrive", ("empty", g))]
+            P[f"row{grp}.{w}"] = rw
+    for g in range(2):
+        C[("full", g)] = 2
+        C[("empty", g)] = C[("qread", g)] = C[("a_full", g)] = C[("o_full", g)] = nrow
+    return P, C
+
+
+# -------------------------------------------------------------- linear_sum --
+def linear_sum_programs(ntiles, nbt, stages=3, nawarps=8):
+    """The K-stage ring continues across tiles; one accumulator set (both M
+    tiles, 512 columns); the A warps also run the epilogue."""
+    P, C = {}, defaultdict(lambda: 1)
+    prod, g = [], 0
+    for T in range(ntiles):
+        for kt in range(nbt):
+            s = g % stages
+            if g >= stages:
+                prod.append(("wait", ("empty", s), g // stages - 1))
+            prod += [("wbeg", ("B", s), g), ("wend", ("B", s)), ("arrive", ("b_full", s))]
+            g += 1
+    P["bprod"] = prod
+    mma, g = [], 0
+    for T in range(ntiles):
+        if T > 0:
+            mma.append(("wait", ("acc_empty",), T - 1))
+        for kt in range(nbt):
+            s = g % stages
+            mma += [("wait", ("a_full", s), g // stages), ("wait", ("b_full", s), g // stages)]
+            mma += [("rbeg", ("A", s, w), g) for w in range(nawarps)] + [("rbeg", ("B", s), g)]
+            if kt == 0:
+                mma.append(("wbeg", ("D",), T))
+            mma += [("rend", ("A", s, w)) for w in range(nawarps)] + [("rend", ("B", s)), ("arrive", ("empty", s))]
+            g += 1
+        mma += [("wend", ("D",)), ("arrive", ("acc_full",))]
+    P["mma"] = mma
+    for w in range(nawarps):
+        aw, g = [], 0
+        for T in range(ntiles):
+            for kt in range(nbt):
+                s = g % stages
+                if g >= stages:
+                    aw.append(("wait", ("empty", s), g // stages - 1))
+                aw += [("wbeg", ("A", s, w), g), ("wend", ("A", s, w)), ("arrive", ("a_full", s))]
+                g += 1
+            aw += [("wait", ("acc_full",), T), ("rbeg", ("D",), T), ("rend", ("D",)), ("arrive", ("acc_empty",))]
+        P[f"aw{w}"] = aw
+    for s in range(stages):
+        C[("a_full", s)] = nawarps
+    C[("acc_empty",)] = nawarps
+    return P, C
+
+
+@pytest.mark.parametrize("nitems,chunks", [(1, 1), (2, 1), (3, 2), (5, 1)])
+def test_linear_kv_protocol(nitems, chunks):
+    P, C = linear_kv_programs(nitems, chunks)
+    for seed in range(40):
+        simulate(P, C, seed)
+
+
+@pytest.mark.parametrize("nitems", [1, 2, 3, 4, 7])
+def test_linear_apply_protocol(nitems):
+    P, C = linear_apply_programs(nitems)
+    for seed in range(60):
+        simulate(P, C, seed)
+
+
+@pytest.mark.parametrize("ntiles,nbt", [(1, 1), (1, 4), (2, 2), (3, 5), (4, 1)])
+def test_linear_sum_protocol(ntiles, nbt):
+    P, C = linear_sum_programs(ntiles, nbt)
+    for seed in range(40):
+        simulate(P, C, seed)
+
+
+# The checker itself: each of these planted protocol mistakes must be caught.
+def _drop_step(P, role, pred):
+    prog = P[role]
+    i = next(i for i, st in enumerate(prog) if pred(st))
+    P[role] = prog[:i] + prog[i + 1:]
+
+
+def _caught(P, C, seeds=200):
+    for seed in range(seeds):
+        try:
+            simulate(P, C, seed)
+        except Violation:
+            return True
+    return False
+
+
+def test_checker_catches_a_missing_empty_wait():
+    # the producer refills stage 0 without waiting for the converters
+    P, C = linear_kv_programs(2, 1)
+    _drop_step(P, "producer", lambda st: st[0] == "wait")
+    assert _caught(P, C)
+
+
+def test_checker_catches_a_missing_qread_barrier():
+    # a row warp writes phi(Q) over rows another warp may still be reading
+    P, C = linear_apply_programs(2)
+    for grp in range(2):
+        for w in range(4):
+            P[f"row{grp}.{w}"] = [st for st in P[f"row{grp}.{w}"] if st[1][0] != "qread"]
+    assert _caught(P, C)
+
+
+def test_checker_catches_an_early_h_refill():
+    # the H producer refills a stage without waiting for the first MMA
+    P, C = linear_apply_programs(4)
+    P["hprod"] = [st for st in P["hprod"] if not (st[0] == "wait" and st[1][0] == "h_empty")]
+    assert _caught(P, C)
+
+
+def test_checker_catches_a_wrong_arrival_count():
+    # one A warp fewer counted on a_full: the MMA may read a stage being written
+    P, C = linear_sum_programs(2, 3)
+    for s in range(3):
+        C[("a_full", s)] = 7
+    assert _caught(P, C)
+
+
+def test_checker_catches_a_parity_alias():
+    # a waiter two phases behind: wait for completion 0 placed after the role
+    # could only get there once completion 2 happened
+    P = {"a": [("arrive", ("x",)), ("arrive", ("x",)), ("arrive", ("x",)), ("arrive", ("y",))],
+         "b": [("wait", ("y",), 0), ("wait", ("x",), 0)]}
+    C = defaultdict(lambda: 1)
+    with pytest.raises(Violation, match="alias"):
+        simulate(P, C, 0)
