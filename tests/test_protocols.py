@@ -1,4 +1,4 @@
-"""The mbarrier protocols of the persistent linear-branch kernels, on the CPU.
+"""The mbarrier protocols of the persistent kernels (linear branch, block-64 flash), on the CPU.
 
 Each kernel role (a producer thread, an MMA-issuing thread, a warp of
 converters or of the epilogue) is written out as its sequence of steps in
@@ -19,8 +19,9 @@ A random scheduler then runs the roles in arbitrary interleavings and checks:
     written.
 
 The role programs follow the kernels in csrc/k_linear.cu (linear_kv_kernel,
-linear_apply_kernel, linear_sum_kernel): the same loop structure, stage and
-phase arithmetic, barrier counts and arrival points.
+linear_apply_kernel, linear_sum_kernel) and csrc/k_flash64.cu (one slot of
+flash64_kernel): the same loop structure, stage and phase arithmetic, barrier
+counts and arrival points.
 """
 import random
 from collections import defaultdict
@@ -356,3 +357,110 @@ def test_checker_catches_a_parity_alias():
     C = defaultdict(lambda: 1)
     with pytest.raises(Violation, match="alias"):
         simulate(P, C, 0)
+
+
+# ---------------------------------------------------------------- flash64 --
+def flash64_programs(nitems, nsteps, rescale, nsoft=4):
+    """One slot of the block-64 flash kernel (the two slots share nothing but
+    the CTA).  Buffers: Q tiles (2), K and V stages (2), step metadata (4),
+    S (TMEM), P~ (2, a part per softmax warp), O (TMEM, a part per softmax
+    warp's lanes).  rescale(gs) says whether the softmax rescales O at step gs
+    (data-dependent in the kernel; only where s > 0)."""
+    P, C = {}, defaultdict(lambda: 1)
+    W = range(nsoft)
+    total = nitems * nsteps
+    kp, vp, gs = [], [], 0
+    for ui in range(nitems):
+        qb = ui & 1
+        if ui >= 2:
+            kp.append(("wait", ("q_empty", qb), (ui >> 1) - 1))
+        kp += [("wbeg", ("Q", qb), ui), ("wend", ("Q", qb)), ("arrive", ("q_full", qb))]
+        for s in range(nsteps):
+            st, ms = gs & 1, gs & 3
+            for prog, nm in ((kp, "K"), (vp, "V")):
+                if gs >= 2:
+                    prog.append(("wait", (nm.lower() + "_empty", st), (gs >> 1) - 1))
+                prog += [("wbeg", (nm, st), gs), ("wend", (nm, st)), ("arrive", (nm.lower() + "_full", st))]
+            if gs >= 4:
+                kp.append(("wait", ("m_empty", ms), (gs >> 2) - 1))
+            kp += [("wbeg", ("meta", ms), gs), ("wend", ("meta", ms)), ("arrive", ("m_full", ms))]
+            gs += 1
+    P["kprod"], P["vprod"] = kp, vp
+    mma = []
+    for gs in range(total + 1):
+        if gs < total:
+            ui, s = divmod(gs, nsteps)
+            qb, st = ui & 1, gs & 1
+            if s == 0:
+                mma.append(("wait", ("q_full", qb), ui >> 1))
+            mma.append(("wait", ("k_full", st), gs >> 1))
+            if gs > 0:
+                mma.append(("wait", ("s_free",), gs - 1))
+            mma += [("rbeg", ("Q", qb), ui), ("rbeg", ("K", st), gs)] + [("wbeg", ("S", w), gs) for w in W]
+            mma += [("rend", ("Q", qb)), ("rend", ("K", st))] + [("wend", ("S", w)) for w in W]
+            mma += [("arrive", ("s_full",)), ("arrive", ("k_empty", st))]
+            if s == nsteps - 1:
+                mma.append(("arrive", ("q_empty", qb)))
+        if gs > 0:
+            gp = gs - 1
+            b = st = gp & 1
+            mma += [("wait", ("v_full", st), gp >> 1), ("wait", ("p_full", b), gp >> 1)]
+            mma += [("rbeg", ("Pt", b, w), gp) for w in W] + [("rbeg", ("V", st), gp)]
+            mma += [("wbeg", ("O", w), gp) for w in W]
+            mma += [("rend", ("Pt", b, w)) for w in W] + [("rend", ("V", st))] + [("wend", ("O", w)) for w in W]
+            mma += [("arrive", ("o_done",)), ("arrive", ("p_empty", b)), ("arrive", ("v_empty", st))]
+    mma.append(("arrive", ("fin",)))
+    P["mma"] = mma
+    for w in W:
+        sm, gs = [], 0
+        for ui in range(nitems):
+            for s in range(nsteps):
+                b = gs & 1
+                sm += [("wait", ("m_full", gs & 3), gs >> 2), ("rbeg", ("meta", gs & 3), gs),
+                       ("rend", ("meta", gs & 3)), ("arrive", ("m_empty", gs & 3))]
+                if gs >= 2:
+                    sm.append(("wait", ("p_empty", b), (gs >> 1) - 1))
+                sm += [("wait", ("s_full",), gs), ("rbeg", ("S", w), gs), ("rend", ("S", w)), ("arrive", ("s_free",)),
+                       ("wbeg", ("Pt", b, w), gs), ("wend", ("Pt", b, w))]
+                if s > 0 and rescale(gs):
+                    sm += [("wait", ("o_done",), gs - 1), ("wbeg", ("O", w), ("r", gs)), ("wend", ("O", w))]
+                sm.append(("arrive", ("p_full", b)))
+                gs += 1
+            # epilogue: the last PV of the item complete (p_empty of its parity)
+            sm += [("wait", ("p_empty", (gs - 1) & 1), (gs - 1) >> 1), ("rbeg", ("O", w), gs - 1), ("rend", ("O", w))]
+        P[f"soft{w}"] = sm
+    for x in range(4):
+        C[("m_empty", x)] = nsoft
+    for b in range(2):
+        C[("p_full", b)] = nsoft
+    C[("s_free",)] = nsoft
+    return P, C
+
+
+@pytest.mark.parametrize("nitems,nsteps", [(1, 1), (1, 3), (2, 1), (2, 2), (3, 3), (4, 2), (2, 5)])
+def test_flash64_protocol(nitems, nsteps):
+    for seed in range(60):
+        pick = random.Random(1000 + seed)
+        flags = {gs: pick.random() < 0.5 for gs in range(nitems * nsteps)}
+        P, C = flash64_programs(nitems, nsteps, lambda gs: flags[gs])
+        simulate(P, C, seed)
+
+
+def test_checker_catches_the_epilogue_waiting_on_o_done():
+    # The epilogue's wait for the last PV taken on o_done instead of p_empty:
+    # o_done may have completed PV(gs-2), PV(gs-1), both or neither, so a
+    # parity wait on it can alias.
+    hits = 0
+    for seed in range(300):
+        pick = random.Random(seed)
+        flags = {gs: pick.random() < 0.2 for gs in range(3 * 3)}
+        P, C = flash64_programs(3, 3, lambda gs: flags[gs])
+        for w in range(4):
+            P[f"soft{w}"] = [("wait", ("o_done",), st[2] * 2 + (st[1][1])) if st[0] == "wait" and st[1][0] == "p_empty"
+                             and i + 1 < len(P[f"soft{w}"]) and P[f"soft{w}"][i + 1][0] == "rbeg"
+                             and P[f"soft{w}"][i + 1][1][0] == "O" else st for i, st in enumerate(P[f"soft{w}"])]
+        try:
+            simulate(P, C, seed)
+        except Violation:
+            hits += 1
+    assert hits > 0
