@@ -1,4 +1,4 @@
-"""The mbarrier protocols of the persistent kernels (linear branch, block-64 flash), on the CPU.
+"""The mbarrier protocols of the persistent kernels (linear branch, block-64 flash, W8A8 GEMM), on the CPU.
 
 Each kernel role (a producer thread, an MMA-issuing thread, a warp of
 converters or of the epilogue) is written out as its sequence of steps in
@@ -19,9 +19,9 @@ A random scheduler then runs the roles in arbitrary interleavings and checks:
     written.
 
 The role programs follow the kernels in csrc/k_linear.cu (linear_kv_kernel,
-linear_apply_kernel, linear_sum_kernel) and csrc/k_flash64.cu (one slot of
-flash64_kernel): the same loop structure, stage and phase arithmetic, barrier
-counts and arrival points.
+linear_apply_kernel, linear_sum_kernel), csrc/k_flash64.cu (one slot of
+flash64_kernel) and csrc/k_w8a8.cu (w8a8_gemm_kernel): the same loop
+structure, stage and phase arithmetic, barrier counts and arrival points.
 """
 import random
 from collections import defaultdict
@@ -464,3 +464,46 @@ def test_checker_catches_the_epilogue_waiting_on_o_done():
         except Violation:
             hits += 1
     assert hits > 0
+
+
+# ------------------------------------------------------------------ w8a8 --
+def w8a8_programs(ntiles, nk, stages=6, accs=4, nepi=8):
+    """w8a8_gemm_kernel: a K-step ring and four TMEM accumulators, both
+    counted over all tiles of the CTA; every K block's INT32 product is read
+    by the eight promotion warps before its accumulator is reused."""
+    P, C = {}, defaultdict(lambda: 1)
+    n = ntiles * nk
+    prod = []
+    for it in range(n):
+        st = it % stages
+        if it >= stages:
+            prod.append(("wait", ("empty", st), it // stages - 1))
+        prod += [("wbeg", ("AB", st), it), ("wend", ("AB", st)), ("arrive", ("full", st))]
+    P["producer"] = prod
+    mma = []
+    for it in range(n):
+        st, b = it % stages, it % accs
+        mma.append(("wait", ("full", st), it // stages))
+        if it >= accs:
+            mma.append(("wait", ("acc_empty", b), it // accs - 1))
+        mma += [("rbeg", ("AB", st), it), ("wbeg", ("acc", b), it), ("rend", ("AB", st)), ("wend", ("acc", b)),
+                ("arrive", ("empty", st)), ("arrive", ("acc_full", b))]
+    mma.append(("arrive", ("fin",)))
+    P["mma"] = mma
+    for e in range(nepi):
+        ep = []
+        for it in range(n):
+            b = it % accs
+            ep += [("wait", ("acc_full", b), it // accs), ("rbeg", ("acc", b), it), ("rend", ("acc", b)),
+                   ("arrive", ("acc_empty", b))]
+        P[f"promo{e}"] = ep
+    for b in range(accs):
+        C[("acc_empty", b)] = nepi
+    return P, C
+
+
+@pytest.mark.parametrize("ntiles,nk", [(1, 1), (1, 7), (2, 3), (3, 40), (5, 2)])
+def test_w8a8_gemm_protocol(ntiles, nk):
+    P, C = w8a8_programs(ntiles, nk)
+    for seed in range(30):
+        simulate(P, C, seed)
