@@ -139,6 +139,21 @@ int sagesla_attn_qknorm(const void* q, const void* k, const void* v, const void*
                         sagesla_stream_t stream);
 
 /*
+ * sagesla_attn_bnhd: the attention on q, k, v in the token-major layout a
+ * DiT's projections emit, bf16 [B][N][H][d] (the row of token n, head h at
+ * ((b*N + n)*H + h)*d), read in place by the kernels that load them; out in
+ * the same layout.  gamma_q and gamma_k both NULL: no norm (then eps is
+ * ignored); both set: the QK RMSNorm of sagesla_attn_qknorm (the per-token
+ * sums run over the H*d contiguous channels of each token).  The result equals
+ * sagesla_attn / sagesla_attn_qknorm on the tensors permuted to [B][H][N][d],
+ * bit for bit.  Note the argument order B, N, H.  Codes as sagesla_attn;
+ * SAGESLA_ERR_INVALID when only one gamma is given.
+ */
+int sagesla_attn_bnhd(const void* q, const void* k, const void* v, const void* gamma_q, const void* gamma_k,
+                      float eps, const void* proj_w, void* out, int B, int N, int H, int d, int block, float topk,
+                      sagesla_stream_t stream);
+
+/*
  * sagesla_get_quant: the smoothing + quantisation step alone (for parity).
  *   q8, k8   int8 [B][H][N][d] device: INT8 codes, row-major.
  *   v8       uint8 [B][H][N][d] device: FP8 E4M3 codes, row-major.

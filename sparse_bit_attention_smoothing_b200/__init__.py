@@ -27,7 +27,7 @@ class SageSLAError(RuntimeError):
         super().__init__(f"{where}: {ERRORS.get(code, 'error')} ({code})")
 
 
-EXPORTS = ["sagesla_attn", "sagesla_attn_opts", "sagesla_attn_qknorm", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
+EXPORTS = ["sagesla_attn", "sagesla_attn_opts", "sagesla_attn_qknorm", "sagesla_attn_bnhd", "dense_int8_attn", "sagesla_attn_host", "sagesla_get_quant", "sagesla_get_mask",
            "sagesla_smooth_stats_noalloc", "sagesla_topk_count", "sagesla_sync_status", "sagesla_strerror",
            "sagesla_release", "sagesla_profile", "sagesla_profile_read", "sagesla_watchdog_selftest",
            "sagesla_debug_flash_stall", "sagesla_w8a8_quant", "sagesla_w8a8_gemm", "sagesla_w8a8_linear"]
@@ -47,6 +47,7 @@ def lib():
         L.dense_int8_attn.argtypes = [P, P, P, P, i, i, i, i, P]
         L.sagesla_attn_opts.argtypes = [P, P, P, P, P, i, i, i, i, i, f, i, i, P]
         L.sagesla_attn_qknorm.argtypes = [P, P, P, P, P, f, P, P, i, i, i, i, i, f, P]
+        L.sagesla_attn_bnhd.argtypes = [P, P, P, P, P, f, P, P, i, i, i, i, i, f, P]
         L.sagesla_attn_host.argtypes = [P, P, P, P, P, i, i, i, i, i, f, P]
         L.sagesla_get_quant.argtypes = [P, P, P, i, i, i, i, P, P, P, P, P, P, P, P]
         L.sagesla_get_mask.argtypes = [P, P, i, i, i, i, i, f, P, P, P, P, P]
@@ -132,6 +133,22 @@ def sagesla_attn_qknorm(q, k, v, gamma_q, gamma_k, eps: float = 1e-6, proj_w=Non
            "sagesla_attn_qknorm")
     return out
 
+
+
+def sagesla_attn_bnhd(q, k, v, proj_w=None, out=None, block: int = 64, topk: float = 0.1, gamma_q=None,
+                      gamma_k=None, eps: float = 1e-6, stream=None):
+    """SageSLA attention on q, k, v in the token-major layout [B, N, H, 128] (out in the same layout), read in place;
+    with gamma_q / gamma_k (bf16 [H*128]) the QK RMSNorm of sagesla_attn_qknorm is fused in as well."""
+    import torch
+    if q.dim() != 4 or q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be a contiguous bf16 [B, N, H, d] tensor")
+    B, N, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().sagesla_attn_bnhd(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma_q), _ptr(gamma_k), ctypes.c_float(eps),
+                                   _ptr(proj_w), _ptr(out), B, N, H, d, block, ctypes.c_float(topk), _stream(stream)),
+           "sagesla_attn_bnhd")
+    return out
 
 def dense_int8_attn(q, k, v, out=None, stream=None):
     import torch

@@ -153,6 +153,8 @@ Geom make_geom(int B, int H, int N, int block, float topk) {
   // the same order whatever B*H a call covers (the host entry point's chunks
   // of heads give the same bits as one call over all heads).
   g.split = (N + 1023) / 1024;
+  g.H = H;
+  g.tok = 0;
   return g;
 }
 
@@ -253,7 +255,7 @@ int run_front(const void* q, const void* k, const void* v, const Geom& g, const 
               cudaStream_t st, int qmax = 127, int q_tok = 0, const NormIn* nrm = nullptr) {
   if (nrm && nrm->gq) {
     ProfScope ps(11, st);
-    SAGESLA_TRY(launch_rc(launch_rms_inv(q, k, nrm->B, nrm->H, g.N, nrm->eps, b.inv_q, b.inv_k, st)));
+    SAGESLA_TRY(launch_rc(launch_rms_inv(q, k, nrm->B, nrm->H, g.N, nrm->eps, b.inv_q, b.inv_k, st, g.tok)));
   }
   const QKNorm nq = qk_norm(b.inv_q, nrm ? nrm->gq : nullptr, nrm, g);
   const QKNorm nk = qk_norm(b.inv_k, nrm ? nrm->gk : nullptr, nrm, g);
@@ -276,12 +278,13 @@ int run_front(const void* q, const void* k, const void* v, const Geom& g, const 
 
 int run_attn(const void* q, const void* k, const void* v, const void* proj_w, void* out, int B, int H, int N, int d,
              int block, float topk, cudaStream_t st, int dbg_grid = 0, int dbg_stall = 0, long dbg_spin = 0,
-             int qmax = 127, int q_tok = 0, const NormIn* nrm = nullptr) {
+             int qmax = 127, int q_tok = 0, const NormIn* nrm = nullptr, int tok = 0) {
   SAGESLA_TRY(validate(q, k, v, out, B, H, N, d, block, topk));
   if (proj_w && !aligned16(proj_w)) return SAGESLA_ERR_MISALIGNED;
   int dev = 0;
   SAGESLA_TRY(check_device(&dev));
-  const Geom g = make_geom(B, H, N, block, topk);
+  Geom g = make_geom(B, H, N, block, topk);
+  g.tok = tok;
   const bool dense = g.kc == g.nb;
   // An empty complement (every key block selected) makes the linear branch 0.
   const bool linear = proj_w != nullptr && !dense;
@@ -385,6 +388,24 @@ int sagesla_attn_qknorm(const void* q, const void* k, const void* v, const void*
   n.H = H;
   return run_attn(q, k, v, proj_w, out, B, H, N, d, block, topk, reinterpret_cast<cudaStream_t>(stream), 0, 0, 0, 127,
                   0, &n);
+}
+
+int sagesla_attn_bnhd(const void* q, const void* k, const void* v, const void* gamma_q, const void* gamma_k,
+                      float eps, const void* proj_w, void* out, int B, int N, int H, int d, int block, float topk,
+                      sagesla_stream_t stream) {
+  if ((gamma_q == nullptr) != (gamma_k == nullptr)) return SAGESLA_ERR_INVALID;
+  NormIn n;
+  if (gamma_q) {
+    if (!(eps >= 0.f) || eps > 1.f) return SAGESLA_ERR_INVALID;
+    if (!aligned16(gamma_q) || !aligned16(gamma_k)) return SAGESLA_ERR_MISALIGNED;
+    n.gq = gamma_q;
+    n.gk = gamma_k;
+    n.eps = (double)eps;
+    n.B = B;
+    n.H = H;
+  }
+  return run_attn(q, k, v, proj_w, out, B, H, N, d, block, topk, reinterpret_cast<cudaStream_t>(stream), 0, 0, 0, 127,
+                  0, gamma_q ? &n : nullptr, 1);
 }
 
 int dense_int8_attn(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,

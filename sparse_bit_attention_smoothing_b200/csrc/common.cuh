@@ -95,6 +95,14 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   return false;
 }
 
+// --------------------------- input layouts --------------------------------
+// Element offset of row (head bh = b*H + h, token n) of a bf16 tensor in the
+// [B][H][N][128] layout (tok = 0) or the token-major [B][N][H][128] layout
+// (tok = 1) in which a DiT's attention projections emit q, k and v.
+__host__ __device__ __forceinline__ size_t row_elems(int tok, int H, int N, int bh, int n) {
+  return tok ? (((size_t)(bh / H) * N + n) * H + bh % H) * kD : ((size_t)bh * N + n) * kD;
+}
+
 // ------------------------------ QK RMSNorm --------------------------------
 // The DiT's RMSNorm of q and k, applied where the path loads them: per token,
 // x / sqrt(mean over its H*d channels of x^2 + eps) * gamma, rounded to bf16

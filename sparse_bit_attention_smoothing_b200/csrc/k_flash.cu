@@ -77,6 +77,7 @@ struct Params {
   int nsteps;  // steps per unit
   int add_out; // 1: out already holds the linear branch (bf16); add O_s to it
   int q_tok;   // 1: one Q scale per token (sq [BH][nq*64])
+  int H, tok;   // heads; out layout: 0 = [B][H][N][d], 1 = [B][N][H][d]
 };
 
 template <int MODE>
@@ -611,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_kernel(const Params p) {
       const int n = i * (MODE == 0 ? 64 : 128) + r;
       const bool store = active && n < p.N;
       const bool has1 = MODE == 1 || p.kc >= 2;
-      __nv_bfloat16* orow = p.out + ((size_t)un.bh * p.N + (store ? n : 0)) * kD;
+      __nv_bfloat16* orow = p.out + row_elems(p.tok, p.H, p.N, un.bh, store ? n : 0);
       const bool add = p.add_out && store;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[0], (gs - 1) & 1, abort, p.wd));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[1], (gs - 1) & 1, abort, p.wd));
@@ -686,6 +687,8 @@ cudaError_t launch_flash128(const FlashArgs& a, const Geom& g, cudaStream_t st, 
   p.v8t = a.v8t;
   p.sq = a.sq;
   p.q_tok = a.q_tok;
+  p.H = g.H;
+  p.tok = g.tok;
   p.sk = a.sk;
   p.sv = a.sv;
   p.idx = a.idx;

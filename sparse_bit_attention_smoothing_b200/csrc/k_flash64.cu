@@ -95,6 +95,7 @@ struct Params {
   int nsteps;  // steps per query block: ceil(kc / 2)
   int add_out; // 1: out already holds the linear branch (bf16); add O_s to it
   int q_tok;    // 1: one Q scale per token (sq [BH][nq*64])
+  int H, tok;   // heads; out layout: 0 = [B][H][N][d], 1 = [B][N][H][d]
   long spin;    // probe limit of every bounded wait that may give up
   int stall_gs; // >= 0: slot 0's K producer omits the copy of this step (watchdog test)
 };
@@ -479,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash64_kernel(const Params p) {
       const float g0 = f0 * inv, g1 = f1 * inv;
       const int n = i * 64 + r;
       const bool store = n < p.N;
-      __nv_bfloat16* orow = p.out + ((size_t)bh * p.N + (store ? n : 0)) * kD + 64 * g;
+      __nv_bfloat16* orow = p.out + row_elems(p.tok, p.H, p.N, bh, store ? n : 0) + 64 * g;
       const float* svh = p.sv + (size_t)bh * kD + 64 * g;
 #pragma unroll 1
       for (int c = 0; c < 64; c += 16) {
@@ -549,6 +550,8 @@ cudaError_t launch_flash(const FlashArgs& a, const Geom& g, cudaStream_t st, int
   p.kc = g.kc;
   p.add_out = a.add_out;
   p.q_tok = a.q_tok;
+  p.H = g.H;
+  p.tok = g.tok;
   p.items = g.BH * g.nb;
   p.nsteps = (g.kc + 1) / 2;
   p.spin = a.dbg_spin > 0 ? a.dbg_spin : kSpinLimit;

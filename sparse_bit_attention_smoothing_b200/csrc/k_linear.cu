@@ -116,7 +116,8 @@ template <int BLK>
 __global__ void __launch_bounds__(kKvThreads, 1) linear_kv_kernel(const uint4* __restrict__ k,
                                                                  const uint4* __restrict__ v, int N, int nb, int nbt,
                                                                  int nitems, uint8_t* __restrict__ hs,
-                                                                 float* __restrict__ z, int* wd, const QKNorm nk) {
+                                                                 float* __restrict__ z, int* wd, const QKNorm nk,
+                                                                 int H, int tok) {
   constexpr int kChunks = BLK / 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -167,10 +168,16 @@ __global__ void __launch_bounds__(kKvThreads, 1) linear_kv_kernel(const uint4* _
             const int rows = j < nb ? max(0, min(64, N - n0)) : 0;
             const uint32_t bytes = (uint32_t)rows * (kD * 2);
             mbar_expect_tx(&bars->raw_full[s], 2 * bytes);
-            if (rows) {
+            if (rows && !tok) {  // the chunk's rows are contiguous
               const size_t off = ((size_t)bh * N + n0) * 16;
               bulk_g2s(smem + s * kKvRaw, k + off, bytes, &bars->raw_full[s]);
               bulk_g2s(smem + s * kKvRaw + kKvHalf, v + off, bytes, &bars->raw_full[s]);
+            } else {  // token-major: one 256-byte row per copy
+              for (int r = 0; r < rows; ++r) {
+                const size_t off = row_elems(1, H, N, bh, n0 + r) / 8;
+                bulk_g2s(smem + s * kKvRaw + r * (kD * 2), k + off, kD * 2, &bars->raw_full[s]);
+                bulk_g2s(smem + s * kKvRaw + kKvHalf + r * (kD * 2), v + off, kD * 2, &bars->raw_full[s]);
+              }
             }
           }
         }
@@ -597,7 +604,7 @@ __global__ void __launch_bounds__(kApThreads, 1) linear_apply_kernel(const uint1
                                                                     const float* __restrict__ zl,
                                                                     const uint8_t* __restrict__ wimg, int N, int nb,
                                                                     int nitems, __nv_bfloat16* __restrict__ out,
-                                                                    int* wd, const QKNorm nq) {
+                                                                    int* wd, const QKNorm nq, int H, int tok) {
   constexpr int M = MODE == 0 ? 64 : 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
@@ -652,7 +659,11 @@ __global__ void __launch_bounds__(kApThreads, 1) linear_apply_kernel(const uint1
         } else {
           const int n0 = 128 * t, rows = min(128, N - n0);
           mbar_expect_tx(&bars->full[g], (uint32_t)rows * (kD * 2));
-          bulk_g2s(st, q + ((size_t)bh * N + n0) * kD, (uint32_t)rows * (kD * 2), &bars->full[g]);
+          if (!tok)  // the item's rows are contiguous
+            bulk_g2s(st, q + ((size_t)bh * N + n0) * kD, (uint32_t)rows * (kD * 2), &bars->full[g]);
+          else  // token-major: one 256-byte row per copy
+            for (int r = 0; r < rows; ++r)
+              bulk_g2s(st + r * (kD * 2), q + row_elems(1, H, N, bh, n0 + r), kD * 2, &bars->full[g]);
         }
       }
       // Drain: the last two items' copies (earlier ones were consumed) and W.
@@ -814,7 +825,7 @@ __global__ void __launch_bounds__(kApThreads, 1) linear_apply_kernel(const uint1
         const int Rr = MODE == 0 ? 64 * (lr >> 4) + 16 * wq + (lr & 15) : 32 * wq + lr;
         const int nr = 128 * t + Rr;
         const uint4 w = *reinterpret_cast<const uint4*>(stg + (32 * C + (lr ^ (C & 7))) * 16);
-        if (nr < N) *reinterpret_cast<uint4*>(out + ((size_t)bh * N + nr) * kD + C * 8) = w;
+        if (nr < N) *reinterpret_cast<uint4*>(out + row_elems(tok, H, N, bh, nr) + C * 8) = w;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->empty[g]);
@@ -841,13 +852,13 @@ cudaError_t launch_linear_apply(const void* q, const uint16_t* himg, const float
     if (e != cudaSuccess) return e;
     linear_apply_kernel<0><<<grid, kApThreads, kApSmem, st>>>((const uint16_t*)q, (const uint8_t*)himg, zl,
                                                               (const uint8_t*)wimg, g.N, g.nb, nitems,
-                                                              (__nv_bfloat16*)out, wd, nq);
+                                                              (__nv_bfloat16*)out, wd, nq, g.H, g.tok);
   } else {
     e = cudaFuncSetAttribute(linear_apply_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kApSmem);
     if (e != cudaSuccess) return e;
     linear_apply_kernel<1><<<grid, kApThreads, kApSmem, st>>>((const uint16_t*)q, (const uint8_t*)himg, zl,
                                                               (const uint8_t*)wimg, g.N, g.nb, nitems,
-                                                              (__nv_bfloat16*)out, wd, nq);
+                                                              (__nv_bfloat16*)out, wd, nq, g.H, g.tok);
   }
   return cudaGetLastError();
 }
@@ -875,12 +886,12 @@ cudaError_t launch_linear_kv(const void* k, const void* v, const Geom& g, uint8_
     e = cudaFuncSetAttribute(linear_kv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
     if (e != cudaSuccess) return e;
     linear_kv_kernel<64><<<grid, kKvThreads, kKvSmem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt, nitems,
-                                                            hs, z, wd, nk);
+                                                            hs, z, wd, nk, g.H, g.tok);
   } else {
     e = cudaFuncSetAttribute(linear_kv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
     if (e != cudaSuccess) return e;
     linear_kv_kernel<128><<<grid, kKvThreads, kKvSmem, st>>>((const uint4*)k, (const uint4*)v, g.N, g.nb, nbt,
-                                                             nitems, hs, z, wd, nk);
+                                                             nitems, hs, z, wd, nk, g.H, g.tok);
   }
   return cudaGetLastError();
 }

@@ -19,11 +19,13 @@ namespace sagesla {
 // ---------------------------------------------------------------- K1 ----
 // grid (split, BH), 128 threads.  Thread t covers channels 8*(t%16)..+7 of
 // rows t/16, t/16+8, ... of its split.  NORM: the QK RMSNorm is applied to
-// the key rows (a separate instance, so the plain loop stays branch-free).
-template <bool NORM>
+// the key rows; TOK: token-major input rows (H of them per token).  Each is a
+// separate instance, so the plain loop stays branch-free.
+template <bool NORM, bool TOK>
 __global__ void __launch_bounds__(128) stats_partial_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
-                                                            int N, int rows_per_split, double* __restrict__ psum,
-                                                            float* __restrict__ pmax, const QKNorm nk) {
+                                                            int N, int H, int rows_per_split,
+                                                            double* __restrict__ psum, float* __restrict__ pmax,
+                                                            const QKNorm nk) {
   const int bh = blockIdx.y, sp = blockIdx.x, t = threadIdx.x;
   const int cg = t & 15, r0 = t >> 4;
   const int n_begin = sp * rows_per_split;
@@ -35,13 +37,15 @@ __global__ void __launch_bounds__(128) stats_partial_kernel(const uint4* __restr
     s[i] = 0.0;
     m[i] = 0.f;
   }
-  const size_t base = (size_t)bh * N * 16;  // in uint4 (8 bf16) units
+  // row n of this head at base + n * pitch, in uint4 (8 bf16) units
+  const size_t base = TOK ? ((size_t)(bh / H) * N * H + bh % H) * 16 : (size_t)bh * N * 16;
+  const size_t pitch = TOK ? (size_t)H * 16 : 16;
   const uint4 gk = NORM ? __ldg(nk.gamma + (bh % nk.H) * 16 + cg) : make_uint4(0, 0, 0, 0);
   const float* invk = NORM ? nk.inv + (size_t)(bh / max(1, nk.H)) * N : nullptr;
 #pragma unroll 4
   for (int n = n_begin + r0; n < n_end; n += 8) {  // unrolled: four row pairs of loads in flight
-    uint4 kk = __ldg(k + base + (size_t)n * 16 + cg);
-    uint4 vv = __ldg(v + base + (size_t)n * 16 + cg);
+    uint4 kk = __ldg(k + base + (size_t)n * pitch + cg);
+    uint4 vv = __ldg(v + base + (size_t)n * pitch + cg);
     if (NORM) kk = rms_row8(kk, __ldg(invk + n), gk);
     uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};
     uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
@@ -132,7 +136,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
                  const float* __restrict__ mu, const float* __restrict__ mv, int N, int nq, int ntiles,
                  uint8_t* __restrict__ q8t, uint8_t* __restrict__ k8t, uint8_t* __restrict__ v8t,
                  float* __restrict__ sq, float* __restrict__ sk, float* __restrict__ qsum, float* __restrict__ ksum,
-                 int* wd, int qmax, int q_tok, const QKNorm nrq, const QKNorm nrk) {
+                 int* wd, int qmax, int q_tok, const QKNorm nrq, const QKNorm nrk, int H, int tok) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   QuantSmem& S = *reinterpret_cast<QuantSmem*>(smem_raw);
   volatile int* abort = &S.abort;
@@ -154,12 +158,22 @@ __global__ void __launch_bounds__(kQThreads, 1)
       mbar_arrive(bar);
       return;
     }
-    const uint32_t bytes = (uint32_t)min(kQB, N - n0) * kRowBytes;
-    const size_t off = ((size_t)bh * N + n0) * kRowBytes;
+    const int rows = min(kQB, N - n0);
+    const uint32_t bytes = (uint32_t)rows * kRowBytes;
     mbar_expect_tx(bar, 3 * bytes);
-    bulk_g2s(S.stage[j % kQStages][0], q + off, bytes, bar);
-    bulk_g2s(S.stage[j % kQStages][1], k + off, bytes, bar);
-    bulk_g2s(S.stage[j % kQStages][2], v + off, bytes, bar);
+    if (!tok) {  // the tile's rows are contiguous
+      const size_t off = ((size_t)bh * N + n0) * kRowBytes;
+      bulk_g2s(S.stage[j % kQStages][0], q + off, bytes, bar);
+      bulk_g2s(S.stage[j % kQStages][1], k + off, bytes, bar);
+      bulk_g2s(S.stage[j % kQStages][2], v + off, bytes, bar);
+    } else {  // token-major: one 256-byte row per copy
+      for (int r = 0; r < rows; ++r) {
+        const size_t off = row_elems(1, H, N, bh, n0 + r) * 2;
+        bulk_g2s(S.stage[j % kQStages][0] + r * kRowBytes, q + off, kRowBytes, bar);
+        bulk_g2s(S.stage[j % kQStages][1] + r * kRowBytes, k + off, kRowBytes, bar);
+        bulk_g2s(S.stage[j % kQStages][2] + r * kRowBytes, v + off, kRowBytes, bar);
+      }
+    }
   };
   int issued = 0;
   if (t == 0)
@@ -355,13 +369,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
 // (H d) + eps)), computed in fp64.
 __global__ void __launch_bounds__(256) rms_inv_kernel(const uint2* __restrict__ q, const uint2* __restrict__ k, int H,
                                                       int N, double eps, float* __restrict__ inv_q,
-                                                      float* __restrict__ inv_k) {
+                                                      float* __restrict__ inv_k, int tok) {
   const int b = blockIdx.y, lane = threadIdx.x & 31;
   const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (n >= N) return;
   double sq = 0.0, sk = 0.0;
   for (int h = 0; h < H; ++h) {
-    const size_t row = (((size_t)b * H + h) * N + n) * 32 + lane;  // uint2 = 4 bf16
+    const size_t row = row_elems(tok, H, N, b * H + h, n) / 4 + lane;  // uint2 = 4 bf16
     const uint2 a = __ldg(q + row), c = __ldg(k + row);
     const uint32_t wa[2] = {a.x, a.y}, wc[2] = {c.x, c.y};
 #pragma unroll
@@ -384,9 +398,9 @@ __global__ void __launch_bounds__(256) rms_inv_kernel(const uint2* __restrict__ 
 }
 
 cudaError_t launch_rms_inv(const void* q, const void* k, int B, int H, int N, double eps, float* inv_q, float* inv_k,
-                           cudaStream_t st) {
+                           cudaStream_t st, int tok) {
   rms_inv_kernel<<<dim3((N + 7) / 8, B), 256, 0, st>>>(static_cast<const uint2*>(q), static_cast<const uint2*>(k), H, N,
-                                                        eps, inv_q, inv_k);
+                                                        eps, inv_q, inv_k, tok);
   return cudaGetLastError();
 }
 
@@ -409,12 +423,16 @@ __global__ void untile_kernel(const uint8_t* __restrict__ q8t, const uint8_t* __
 cudaError_t launch_stats_partial(const void* k, const void* v, const Geom& g, double* psum, float* pmax,
                                  cudaStream_t st, QKNorm nk) {
   const int rows = (g.N + g.split - 1) / g.split;
-  if (nk.inv)
-    stats_partial_kernel<true><<<dim3(g.split, g.BH), 128, 0, st>>>((const uint4*)k, (const uint4*)v, g.N, rows, psum,
-                                                                    pmax, nk);
+  const dim3 grid(g.split, g.BH);
+  const uint4 *k4 = (const uint4*)k, *v4 = (const uint4*)v;
+  if (nk.inv && g.tok)
+    stats_partial_kernel<true, true><<<grid, 128, 0, st>>>(k4, v4, g.N, g.H, rows, psum, pmax, nk);
+  else if (nk.inv)
+    stats_partial_kernel<true, false><<<grid, 128, 0, st>>>(k4, v4, g.N, g.H, rows, psum, pmax, nk);
+  else if (g.tok)
+    stats_partial_kernel<false, true><<<grid, 128, 0, st>>>(k4, v4, g.N, g.H, rows, psum, pmax, nk);
   else
-    stats_partial_kernel<false><<<dim3(g.split, g.BH), 128, 0, st>>>((const uint4*)k, (const uint4*)v, g.N, rows, psum,
-                                                                     pmax, nk);
+    stats_partial_kernel<false, false><<<grid, 128, 0, st>>>(k4, v4, g.N, g.H, rows, psum, pmax, nk);
   return cudaGetLastError();
 }
 
@@ -436,7 +454,7 @@ cudaError_t launch_quant(const void* q, const void* k, const void* v, const floa
   const int ntiles = g.BH * g.nq;
   quant_kernel<<<min(ntiles, sms), kQThreads, smem, st>>>((const uint8_t*)q, (const uint8_t*)k, (const uint8_t*)v, mu,
                                                           mv, g.N, g.nq, ntiles, q8t, k8t, v8t, sq, sk, qsum, ksum, wd,
-                                                          qmax, q_tok, nq, nk);
+                                                          qmax, q_tok, nq, nk, g.H, g.tok);
   return cudaGetLastError();
 }
 

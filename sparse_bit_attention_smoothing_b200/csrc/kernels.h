@@ -16,6 +16,8 @@ struct Geom {
   int nq;      // 64-token quantisation tiles per head, padded: 2*ceil(N/128)
   int kc;      // key blocks kept per query block
   int split;   // row splits of the statistics pass
+  int H = 1;   // heads (B = BH / H)
+  int tok = 0; // q, k, v, out layout: 0 = [B][H][N][d], 1 = [B][N][H][d] (token-major, as a DiT emits it)
 };
 
 // QK RMSNorm applied where a kernel loads q or k (inv == nullptr: off):
@@ -27,7 +29,7 @@ struct QKNorm {
 };
 // Per-token 1 / rms of q and k (QK RMSNorm), [B][N] each.
 cudaError_t launch_rms_inv(const void* q, const void* k, int B, int H, int N, double eps, float* inv_q, float* inv_k,
-                           cudaStream_t st);
+                           cudaStream_t st, int tok = 0);
 // K1: per-split fp64 sums of K and fp32 max|V| per channel.
 cudaError_t launch_stats_partial(const void* k, const void* v, const Geom& g, double* psum, float* pmax,
                                  cudaStream_t st, QKNorm nk = QKNorm());
@@ -69,7 +71,7 @@ struct FlashArgs {
   const float* sk;
   const float* sv;
   const int32_t* idx;  // [BH][nb][kc]; NULL = dense (every block, ascending)
-  void* out;           // bf16 [BH][N][128]
+  void* out;           // bf16 rows of 128 in the Geom's layout
   int add_out;          // 1: out already holds the linear branch y (bf16); add O_s to it
   int q_tok;            // 1: sq holds one Q scale per token ([BH][nq*64]) instead of per 64-token tile
   // Watchdog test of the block-64 kernel (all 0 in a normal call): a grid of

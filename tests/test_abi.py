@@ -85,6 +85,11 @@ def test_rejects_bad_arguments_without_launch(L):
     assert L.sagesla_attn_qknorm(a, a, a, None, a, F(1e-6), None, a, 1, 1, 64, 128, 64, F(0.1), None) == -1
     assert L.sagesla_attn_qknorm(a, a, a, a, a, F(-1.0), None, a, 1, 1, 64, 128, 64, F(0.1), None) == -1
     assert L.sagesla_attn_qknorm(a, a, a, P(0x10008), a, F(1e-6), None, a, 1, 1, 64, 128, 64, F(0.1), None) == -2
+    # token-major entry (B, N, H order): one weight without the other, eps out of range, misaligned weights, d != 128
+    assert L.sagesla_attn_bnhd(a, a, a, a, None, F(1e-6), None, a, 1, 64, 1, 128, 64, F(0.1), None) == -1
+    assert L.sagesla_attn_bnhd(a, a, a, a, a, F(2.0), None, a, 1, 64, 1, 128, 64, F(0.1), None) == -1
+    assert L.sagesla_attn_bnhd(a, a, a, P(0x10008), a, F(1e-6), None, a, 1, 64, 1, 128, 64, F(0.1), None) == -2
+    assert L.sagesla_attn_bnhd(a, a, a, None, None, F(0.0), None, a, 1, 64, 1, 64, 64, F(0.1), None) == -1
     # quantisation options out of range
     assert L.sagesla_attn_opts(a, a, a, None, a, 1, 1, 64, 128, 64, F(0.1), 5, 0, None) == -1
     assert L.sagesla_attn_opts(a, a, a, None, a, 1, 1, 64, 128, 64, F(0.1), 8, 2, None) == -1
