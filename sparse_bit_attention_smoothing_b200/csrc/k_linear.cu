@@ -9,7 +9,7 @@
 //   H_i = sum_{j not in S_i} h_j   (a 0/1 complement-mask GEMM per head)
 //
 // K4a linear_kv:  per key block, h_j on tcgen05 (kind::f16, both operands
-//   MN-major, staged from the token-major rows), fp32 accumulate, stored in
+//   MN-major, staged from the 128-channel rows of K and V), fp32 accumulate, stored in
 //   bf16 as the B tiles of the mask GEMM; z_j in fp32.
 // K4b linear_sum: per head, H = (1 - M) . Hstack with tcgen05 (M=128 query
 //   blocks x N=256 columns of the d*d matrices, K = key blocks); the 0/1 A

@@ -363,7 +363,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
 // Per-token 1 / rms of q and k over all H heads x d channels (QK RMSNorm):
 // grid (ceil(N / 8), B), 256 threads, one warp per token; lane l reads
-// channels 4l .. 4l+3 of every head's row.  The squares of bf16 values are
+// channels 4l .. 4l+3 of every head's row (in either input layout; in the
+// token-major one the H rows of a token are contiguous).  The squares of bf16 values are
 // exact in fp64 and their sum is rounded far below the fp32 rounding of the
 // result, so the order of the sum does not change inv = fl32(1 / sqrt(sum /
 // (H d) + eps)), computed in fp64.
