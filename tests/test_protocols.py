@@ -1,4 +1,4 @@
-"""The mbarrier protocols of the persistent kernels (linear branch, block-64 flash, W8A8 GEMM), on the CPU.
+"""The barrier protocols of the persistent kernels (quantiser, linear branch, block-64 flash, W8A8 GEMM), on the CPU.
 
 Each kernel role (a producer thread, an MMA-issuing thread, a warp of
 converters or of the epilogue) is written out as its sequence of steps in
@@ -20,8 +20,10 @@ A random scheduler then runs the roles in arbitrary interleavings and checks:
 
 The role programs follow the kernels in csrc/k_linear.cu (linear_kv_kernel,
 linear_apply_kernel, linear_sum_kernel), csrc/k_flash64.cu (one slot of
-flash64_kernel) and csrc/k_w8a8.cu (w8a8_gemm_kernel): the same loop
-structure, stage and phase arithmetic, barrier counts and arrival points.
+flash64_kernel), csrc/k_w8a8.cu (w8a8_gemm_kernel) and csrc/k_prologue.cu
+(quant_kernel, whose block barriers are modelled as one barrier phase per use
+that every warp arrives at and waits for): the same loop structure, stage and
+phase arithmetic, barrier counts and arrival points.
 """
 import random
 from collections import defaultdict
@@ -507,3 +509,61 @@ def test_w8a8_gemm_protocol(ntiles, nk):
     P, C = w8a8_programs(ntiles, nk)
     for seed in range(30):
         simulate(P, C, seed)
+
+
+# ------------------------------------------------------------------ quant --
+def quant_programs(ntiles, q_tok, nwarps=4, stages=3):
+    """quant_kernel: thread 0 (in warp 0) keeps a 3-stage ring of bulk copies
+    of the Q, K, V rows one tile ahead per stage; block barriers (one phase
+    per use, all warps) order the reads of a stage before its refill and the
+    reuse of the tile images, partial sums and per-warp maxima across tiles."""
+    P, C = {}, defaultdict(lambda: 1)
+    for w in range(nwarps):
+        pr = []
+        issued = 0
+        if w == 0:
+            while issued < min(stages, ntiles):
+                st = issued % stages
+                pr += [("wbeg", ("stage", st), issued), ("wend", ("stage", st)), ("arrive", ("full", st))]
+                issued += 1
+        for j in range(ntiles):
+            st = j % stages
+            pr += [("wait", ("full", st), j // stages), ("arrive", ("A", j)), ("wait", ("A", j), 0),
+                   ("rbeg", ("stage", st), j), ("wbeg", ("img", 2), j), ("wend", ("img", 2)),
+                   ("rend", ("stage", st)), ("wbeg", ("red", w), j), ("wend", ("red", w)),
+                   ("arrive", ("B", j)), ("wait", ("B", j), 0)]
+            if w == 0 and issued < ntiles:  # refill the stage just read
+                pr += [("wbeg", ("stage", issued % stages), issued), ("wend", ("stage", issued % stages)),
+                       ("arrive", ("full", issued % stages))]
+                issued += 1
+            pr += [("rbeg", ("red", x), j) for x in range(nwarps)] + [("rend", ("red", x)) for x in range(nwarps)]
+            if q_tok:
+                pr += [("wbeg", ("rowmax", w), j), ("wend", ("rowmax", w)), ("arrive", ("R", j)), ("wait", ("R", j), 0)]
+                pr += [("rbeg", ("rowmax", x), j) for x in range(nwarps)] + [("rend", ("rowmax", x)) for x in range(nwarps)]
+            pr += [("wbeg", ("img", 0), j), ("wend", ("img", 0)), ("wbeg", ("psum", w), j), ("wend", ("psum", w)),
+                   ("arrive", ("C", j)), ("wait", ("C", j), 0)]
+            pr += [("rbeg", ("psum", x), j) for x in range(nwarps)] + [("rend", ("psum", x)) for x in range(nwarps)]
+            pr += [("rbeg", ("img", x), j) for x in (0, 2)] + [("rend", ("img", x)) for x in (0, 2)]
+        P[f"warp{w}"] = pr
+    for j in range(ntiles):
+        for b in ("A", "B", "R", "C"):
+            C[(b, j)] = nwarps
+    return P, C
+
+
+@pytest.mark.parametrize("ntiles,q_tok", [(1, 0), (2, 1), (3, 0), (4, 1), (7, 0), (8, 1)])
+def test_quant_ring_protocol(ntiles, q_tok):
+    P, C = quant_programs(ntiles, q_tok)
+    for seed in range(40):
+        simulate(P, C, seed)
+
+
+def test_checker_catches_a_refill_before_the_barrier():
+    # thread 0 refilling the stage before every warp has passed barrier B
+    P, C = quant_programs(4, 0)
+    prog = P["warp0"]
+    i = next(i for i, st in enumerate(prog) if st == ("arrive", ("B", 0)))
+    k = next(i for i, st in enumerate(prog) if st[0] == "wbeg" and st[1] == ("stage", 0) and st[2] == 3)
+    refill = prog[k:k + 3]
+    P["warp0"] = prog[:i] + refill + prog[i:k] + prog[k + 3:]
+    assert _caught(P, C)
