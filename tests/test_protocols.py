@@ -1,4 +1,5 @@
-"""The barrier protocols of the persistent kernels (quantiser, linear branch, block-64 flash, W8A8 GEMM), on the CPU.
+"""The barrier protocols of the persistent and ring-buffered kernels (quantiser, pooled top-k, linear branch,
+block-64 flash, W8A8 GEMM), on the CPU.
 
 Each kernel role (a producer thread, an MMA-issuing thread, a warp of
 converters or of the epilogue) is written out as its sequence of steps in
@@ -21,9 +22,10 @@ A random scheduler then runs the roles in arbitrary interleavings and checks:
 The role programs follow the kernels in csrc/k_linear.cu (linear_kv_kernel,
 linear_apply_kernel, linear_sum_kernel), csrc/k_flash64.cu (one slot of
 flash64_kernel), csrc/k_w8a8.cu (w8a8_gemm_kernel) and csrc/k_prologue.cu
-(quant_kernel, whose block barriers are modelled as one barrier phase per use
-that every warp arrives at and waits for): the same loop structure, stage and
-phase arithmetic, barrier counts and arrival points.
+(quant_kernel) and csrc/k_topk.cu (pool_topk16_kernel's chunk ring), whose
+block barriers are modelled as one barrier phase per use that every warp or
+thread arrives at and waits for: the same loop structure, stage and phase
+arithmetic, barrier counts and arrival points.
 """
 import random
 from collections import defaultdict
@@ -566,4 +568,61 @@ def test_checker_catches_a_refill_before_the_barrier():
     k = next(i for i, st in enumerate(prog) if st[0] == "wbeg" and st[1] == ("stage", 0) and st[2] == 3)
     refill = prog[k:k + 3]
     P["warp0"] = prog[:i] + refill + prog[i:k] + prog[k + 3:]
+    assert _caught(P, C)
+
+
+# --------------------------------------------------------------- pool_topk --
+def pool_topk16_programs(nchunk, nthreads=4, nbuf=3):
+    """pool_topk16_kernel phase 1: every thread copies its share of kbar chunk
+    c into buffer c % 3 with cp.async (one commit group per chunk), two chunks
+    ahead; cp.async.wait_group<2> (or <1>, <0> at the tail) retires its own
+    groups up to chunk c, a block barrier publishes them, the chunk is scored,
+    and a second barrier ends every read of the buffer before it is refilled.
+    A thread's copy of chunk c is 'being written' from its issue until the
+    wait that retires its group."""
+    P, C = {}, defaultdict(lambda: 1)
+    for t in range(nthreads):
+        pr, pending = [], []
+
+        def issue(c):
+            pr.append(("wbeg", ("kb", c % nbuf, t), c))
+            pending.append(c)
+
+        def wait_group(n):  # all but the n most recent of this thread's groups complete
+            while len(pending) > n:
+                c = pending.pop(0)
+                pr.append(("wend", ("kb", c % nbuf, t)))
+
+        issue(0)
+        if nchunk > 1:
+            issue(1)
+        for c in range(nchunk):
+            if c + 2 < nchunk:
+                issue(c + 2)
+                wait_group(2)
+            elif c + 1 < nchunk:
+                wait_group(1)
+            else:
+                wait_group(0)
+            pr += [("arrive", ("S1", c)), ("wait", ("S1", c), 0)]
+            pr += [("rbeg", ("kb", c % nbuf, x), c) for x in range(nthreads)]
+            pr += [("rend", ("kb", c % nbuf, x)) for x in range(nthreads)]
+            pr += [("wbeg", ("psc", t), c), ("wend", ("psc", t)), ("arrive", ("S2", c)), ("wait", ("S2", c), 0)]
+            pr += [("rbeg", ("psc", x), c) for x in range(nthreads)] + [("rend", ("psc", x)) for x in range(nthreads)]
+        P[f"t{t}"] = pr
+    for c in range(nchunk):
+        C[("S1", c)] = C[("S2", c)] = nthreads
+    return P, C
+
+
+@pytest.mark.parametrize("nchunk", [1, 2, 3, 4, 7, 19])
+def test_pool_topk16_ring_protocol(nchunk):
+    P, C = pool_topk16_programs(nchunk)
+    for seed in range(40):
+        simulate(P, C, seed)
+
+
+def test_checker_catches_a_two_buffer_ring_two_chunks_ahead():
+    # two buffers with the same two-chunk lookahead: chunk c + 2 overwrites the buffer still being scored
+    P, C = pool_topk16_programs(5, nbuf=2)
     assert _caught(P, C)
